@@ -1,0 +1,129 @@
+"""Plain CPU oracle for block-scaled FP8 GEMM (test infrastructure only).
+
+Only ``tests/``, ``__graft_entry__.smoke()`` and ``bench.py``'s CPU-baseline
+leg (and its ``--impl reference`` arm) may import this package.  The product
+path (``fp8_block_scaled_bsgemm_b200``) never imports it and shares no code
+with it: the arithmetic lives in ``bsgemm_oracle.c``; this module only
+compiles that file with the host C compiler and marshals numpy arrays.
+
+What the oracle computes is stated in the header of ``bsgemm_oracle.c``
+(hncyxsy.com/news/191052, §2.2 block scaling, §3.1 granularity, §3.2
+segment-wise FP32 accumulation, §4.2 API and layouts, §5.2 scale direction).
+
+Parity pins: ``tests/test_oracle_pins.py`` and ``tests/golden/``.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+import threading
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "bsgemm_oracle.c")
+_LIB = os.path.join(_HERE, "liboracle.so")
+_lock = threading.Lock()
+_lib = None
+
+LAYOUTS = {"nt": 0, "tn": 1, "nn": 2, "tt": 3}
+
+
+def build(force: bool = False) -> str:
+    """Compile ``bsgemm_oracle.c`` into ``liboracle.so`` (gcc, OpenMP)."""
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+        tmp = _LIB + f".tmp{os.getpid()}"
+        cmd = ["gcc", "-O2", "-fopenmp", "-fPIC", "-shared", "-std=c11", "-Wall", "-Wextra",
+               "-o", tmp, _SRC, "-lm"]
+        subprocess.run(cmd, check=True)
+        os.replace(tmp, _LIB)
+    return _LIB
+
+
+def _load():
+    global _lib
+    with _lock:
+        if _lib is None:
+            lib = ctypes.CDLL(build())
+            p = ctypes.c_void_p
+            i64 = ctypes.c_int64
+            lib.oracle_e4m3_value.restype = ctypes.c_double
+            lib.oracle_e4m3_value.argtypes = [ctypes.c_uint8]
+            lib.oracle_bf16_rne.restype = ctypes.c_uint16
+            lib.oracle_bf16_rne.argtypes = [ctypes.c_double]
+            lib.oracle_bsgemm.restype = ctypes.c_int
+            lib.oracle_bsgemm.argtypes = [ctypes.c_int, p, p, p, p, i64, i64, i64, i64, p, p]
+            lib.oracle_bsgemm_at.restype = ctypes.c_int
+            lib.oracle_bsgemm_at.argtypes = [ctypes.c_int, p, p, p, p, i64, i64, i64, i64, i64,
+                                             p, p, p, p]
+            lib.oracle_num_threads.restype = ctypes.c_int
+            lib.oracle_num_threads.argtypes = []
+            _lib = lib
+    return _lib
+
+
+def _ptr(x: np.ndarray):
+    return x.ctypes.data_as(ctypes.c_void_p)
+
+
+def e4m3_value(code: int) -> float:
+    """Exact value of one E4M3 code (NaN for 0x7F / 0xFF)."""
+    return _load().oracle_e4m3_value(int(code))
+
+
+def e4m3_table() -> np.ndarray:
+    """All 256 E4M3 codes decoded to float64."""
+    return np.array([e4m3_value(c) for c in range(256)], dtype=np.float64)
+
+
+def bf16_rne(x: float) -> int:
+    """BF16 bit pattern of ``x`` rounded once, to nearest-even, from FP64."""
+    return int(_load().oracle_bf16_rne(float(x)))
+
+
+def num_threads() -> int:
+    return int(_load().oracle_num_threads())
+
+
+def _check_inputs(layout, a, b, sa, sb, M, N, K, gran):
+    if layout not in LAYOUTS:
+        raise ValueError(f"layout must be one of {sorted(LAYOUTS)}")
+    a = np.ascontiguousarray(a, dtype=np.uint8)
+    b = np.ascontiguousarray(b, dtype=np.uint8)
+    sa = np.ascontiguousarray(sa, dtype=np.float32)
+    sb = np.ascontiguousarray(sb, dtype=np.float32)
+    kb = -(-K // gran)
+    if a.size != M * K or b.size != N * K:
+        raise ValueError("operand sizes do not match M, N, K")
+    if sa.size != -(-M // gran) * kb or sb.size != -(-N // gran) * kb:
+        raise ValueError("scale sizes do not match the granularity")
+    return a, b, sa, sb
+
+
+def bsgemm(layout: str, a, b, sa, sb, M: int, N: int, K: int, gran: int):
+    """Full oracle product. Returns (ref float64 [M,N], out bf16 bits uint16 [M,N])."""
+    a, b, sa, sb = _check_inputs(layout, a, b, sa, sb, M, N, K, gran)
+    ref = np.empty((M, N), dtype=np.float64)
+    out = np.empty((M, N), dtype=np.uint16)
+    rc = _load().oracle_bsgemm(LAYOUTS[layout], _ptr(a), _ptr(b), _ptr(sa), _ptr(sb),
+                               M, N, K, gran, _ptr(ref), _ptr(out))
+    if rc != 0:
+        raise RuntimeError(f"oracle_bsgemm failed with code {rc}")
+    return ref, out
+
+
+def bsgemm_at(layout: str, a, b, sa, sb, M: int, N: int, K: int, gran: int, mi, ni):
+    """Oracle outputs at (mi[i], ni[i]) only. Returns (ref float64, out uint16)."""
+    a, b, sa, sb = _check_inputs(layout, a, b, sa, sb, M, N, K, gran)
+    mi = np.ascontiguousarray(mi, dtype=np.int64)
+    ni = np.ascontiguousarray(ni, dtype=np.int64)
+    if mi.shape != ni.shape:
+        raise ValueError("mi and ni must have the same shape")
+    ref = np.empty(mi.shape, dtype=np.float64)
+    out = np.empty(mi.shape, dtype=np.uint16)
+    rc = _load().oracle_bsgemm_at(LAYOUTS[layout], _ptr(a), _ptr(b), _ptr(sa), _ptr(sb),
+                                  M, N, K, gran, mi.size, _ptr(mi), _ptr(ni), _ptr(ref), _ptr(out))
+    if rc != 0:
+        raise RuntimeError(f"oracle_bsgemm_at failed with code {rc}")
+    return ref, out

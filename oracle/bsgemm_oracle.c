@@ -1,0 +1,238 @@
+/*
+ * Plain CPU oracle for block-scaled FP8 GEMM.
+ *
+ * TEST INFRASTRUCTURE ONLY. Nothing on the product path may call, link or load
+ * this file: only the tests, the smoke check and the bench's CPU-baseline leg
+ * use it. It shares no code, header, table or constant with the CUDA library.
+ *
+ * What it computes (hncyxsy.com/news/191052, "DeepGEMM实战: FP8矩阵乘法加速与
+ * Hopper架构优化指南"):
+ *   - inputs are FP8 E4M3 codes, accumulation is FP32 or wider (§2.2, §3.2);
+ *   - each operand carries one FP32 scale per g x g block, g in {64,128,256},
+ *     default 128 (§2.2, §3.1 table);
+ *   - dequantisation multiplies by the scale (§5.2: "quantise divides,
+ *     dequantise multiplies");
+ *   - K is cut into segments that are accumulated separately and then added
+ *     (§3.2), which is where the per-block scales enter;
+ *   - out is BF16 [M,N], A is [M,K] and B is [N,K] in the "NT" layout, and the
+ *     NT/TN/NN/TT flags say how A and B are stored (§3.3, §4.2).
+ *
+ * The exact definition written out here, for every (m, n):
+ *
+ *   ref[m,n] = sum_{kb=0}^{Kb-1} sA[m/g][kb] * sB[n/g][kb]
+ *                                * sum_{k in block kb} dec(A[m,k]) * dec(B[n,k])
+ *   out[m,n] = bf16_rne(ref[m,n])          (one rounding, straight from FP64)
+ *
+ * Arithmetic, chosen so that every step is either exact or one FP64 rounding:
+ *   - dec(code) is an integer count of 2^-9 (every E4M3 value is a multiple
+ *     of 2^-9, the smallest subnormal, and |value| <= 448 = 229376 * 2^-9);
+ *   - the inner block sum is an exact int64 count of 2^-18 (|product| < 2^36,
+ *     at most 256 terms, so |sum| < 2^44);
+ *   - sA*sB is exact in FP64 (24 + 24 significant bits <= 53);
+ *   - term = blocksum * 2^-18 * (sA*sB) is one FP64 rounding, and the terms
+ *     are added in ascending kb in FP64.
+ *
+ * Readings of points the pages leave open (each one is also listed in the
+ * design notes): both operands use g x g blocks; the scale tensors are
+ * row-major FP32 [ceil(rows/g)][ceil(K/g)] in logical block coordinates for
+ * every storage layout; a partial last block (rows or K not a multiple of g)
+ * simply has fewer terms; for the layout flags the first letter is A and the
+ * second is B, "N" for A means stored [M,K], "T" for A means stored [K,M],
+ * "T" for B means stored [N,K] and "N" for B means stored [K,N].
+ *
+ * parity pins: see tests/test_oracle_pins.py (closed forms, power-of-two
+ * invariants, exact-rational brute force, hand-worked cases in tests/golden/).
+ */
+#include <math.h>
+#include <stdint.h>
+#include <string.h>
+
+#define OR_LAYOUT_NT 0
+#define OR_LAYOUT_TN 1
+#define OR_LAYOUT_NN 2
+#define OR_LAYOUT_TT 3
+
+#define OR_OK 0
+#define OR_ERR_ARG 1
+#define OR_ERR_NAN_INPUT 2
+
+/* ---- E4M3 ("fn": no infinities) decode -------------------------------------
+ * Bit layout: s eeee mmm, exponent bias 7.
+ *   eeee == 0            : subnormal, value = (-1)^s * m/8 * 2^-6 = m * 2^-9
+ *   eeee == 1111, mmm=111: NaN (the only non-finite code)
+ *   otherwise            : value = (-1)^s * (1 + m/8) * 2^(e-7)
+ *                                = (-1)^s * (8 + m) * 2^(e-1) * 2^-9
+ * The result is the value as a signed integer count of 2^-9.               */
+static int e4m3_units(uint8_t code, int64_t *units)
+{
+    int s = code >> 7;
+    int e = (code >> 3) & 0xF;
+    int m = code & 0x7;
+    int64_t mag;
+    if (e == 0xF && m == 0x7)
+        return 0; /* NaN */
+    if (e == 0)
+        mag = m;
+    else
+        mag = (int64_t)(8 + m) << (e - 1);
+    *units = s ? -mag : mag;
+    return 1;
+}
+
+/* Value of one E4M3 code as a double (NaN for the NaN codes). */
+double oracle_e4m3_value(uint8_t code)
+{
+    int64_t u;
+    if (!e4m3_units(code, &u))
+        return NAN;
+    return ldexp((double)u, -9);
+}
+
+/* ---- FP64 -> BF16, round to nearest, ties to even --------------------------
+ * BF16 keeps 8 significant bits and FP32's exponent range (normal minimum
+ * 2^-126, subnormal quantum 2^-133, largest finite (2 - 2^-7) * 2^127).
+ * The rounding is done once, on the exact double, with no detour through
+ * FP32 (which would round twice).                                         */
+uint16_t oracle_bf16_rne(double x)
+{
+    double r;
+    float f;
+    uint32_t bits;
+    if (isnan(x))
+        return 0x7FC0;
+    if (x == 0.0)
+        return signbit(x) ? 0x8000 : 0x0000;
+    if (isinf(x))
+        return signbit(x) ? 0xFF80 : 0x7F80;
+    if (fabs(x) < ldexp(1.0, -126)) {
+        /* subnormal range: quantum 2^-133 */
+        r = ldexp(nearbyint(ldexp(x, 133)), -133);
+    } else {
+        int e;
+        double fr = frexp(x, &e);            /* x = fr * 2^e, 0.5 <= |fr| < 1 */
+        double q = nearbyint(ldexp(fr, 8));  /* 8 significant bits, ties-to-even */
+        r = ldexp(q, e - 8);                 /* q == +-256 carries into the next binade */
+    }
+    if (fabs(r) > ldexp(255.0, 120)) /* 255 * 2^120 = (2 - 2^-7) * 2^127 */
+        r = x > 0 ? INFINITY : -INFINITY;
+    f = (float)r; /* exact: r has <= 8 significant bits in FP32's range */
+    memcpy(&bits, &f, sizeof bits);
+    return (uint16_t)(bits >> 16);
+}
+
+/* ---- element access by layout (§3.3 / §4.2 flags) ---------------------- */
+static inline uint8_t elem_a(int layout, const uint8_t *a, int64_t M, int64_t K, int64_t m, int64_t k)
+{
+    /* first letter: N -> A stored [M,K]; T -> A stored [K,M] */
+    if (layout == OR_LAYOUT_NT || layout == OR_LAYOUT_NN)
+        return a[m * K + k];
+    return a[k * M + m];
+}
+
+static inline uint8_t elem_b(int layout, const uint8_t *b, int64_t N, int64_t K, int64_t n, int64_t k)
+{
+    /* second letter: T -> B stored [N,K]; N -> B stored [K,N] */
+    if (layout == OR_LAYOUT_NT || layout == OR_LAYOUT_TT)
+        return b[n * K + k];
+    return b[k * N + n];
+}
+
+/* One output element: the definition above, term by term.
+ * Returns 0 on success, OR_ERR_NAN_INPUT if a NaN code was met.          */
+static int one_element(int layout, const uint8_t *a, const uint8_t *b, const float *sa,
+                       const float *sb, int64_t M, int64_t N, int64_t K, int64_t g,
+                       int64_t m, int64_t n, double *ref)
+{
+    int64_t Kb = (K + g - 1) / g;
+    double acc = 0.0;
+    for (int64_t kb = 0; kb < Kb; ++kb) {
+        int64_t k0 = kb * g;
+        int64_t k1 = k0 + g < K ? k0 + g : K;
+        int64_t blocksum = 0; /* exact, units of 2^-18 */
+        for (int64_t k = k0; k < k1; ++k) {
+            int64_t ua, ub;
+            if (!e4m3_units(elem_a(layout, a, M, K, m, k), &ua) ||
+                !e4m3_units(elem_b(layout, b, N, K, n, k), &ub)) {
+                *ref = NAN;
+                return OR_ERR_NAN_INPUT;
+            }
+            blocksum += ua * ub;
+        }
+        double scale = (double)sa[(m / g) * Kb + kb] * (double)sb[(n / g) * Kb + kb]; /* exact */
+        acc += ldexp((double)blocksum, -18) * scale;
+    }
+    *ref = acc;
+    return OR_OK;
+}
+
+static int check_args(int layout, const void *a, const void *b, const float *sa, const float *sb,
+                      int64_t M, int64_t N, int64_t K, int64_t g)
+{
+    if (layout < OR_LAYOUT_NT || layout > OR_LAYOUT_TT)
+        return OR_ERR_ARG;
+    if (!a || !b || !sa || !sb || M <= 0 || N <= 0 || K <= 0 || g <= 0)
+        return OR_ERR_ARG;
+    return OR_OK;
+}
+
+/* Full output. ref: FP64 [M*N] (may be NULL); out: BF16 bits [M*N] (may be NULL).
+ * Parallel over rows with OpenMP when compiled with it; each element is
+ * computed independently, so the result does not depend on the thread count. */
+int oracle_bsgemm(int layout, const uint8_t *a, const uint8_t *b, const float *sa, const float *sb,
+                  int64_t M, int64_t N, int64_t K, int64_t g, double *ref, uint16_t *out)
+{
+    int rc = check_args(layout, a, b, sa, sb, M, N, K, g);
+    int bad = 0;
+    if (rc)
+        return rc;
+#pragma omp parallel for schedule(dynamic, 1) reduction(| : bad)
+    for (int64_t m = 0; m < M; ++m) {
+        for (int64_t n = 0; n < N; ++n) {
+            double r;
+            bad |= one_element(layout, a, b, sa, sb, M, N, K, g, m, n, &r);
+            if (ref)
+                ref[m * N + n] = r;
+            if (out)
+                out[m * N + n] = oracle_bf16_rne(r);
+        }
+    }
+    return bad ? OR_ERR_NAN_INPUT : OR_OK;
+}
+
+/* Selected outputs only: element i is (mi[i], ni[i]). For parity checks at
+ * sizes where the full product would take the oracle too long.            */
+int oracle_bsgemm_at(int layout, const uint8_t *a, const uint8_t *b, const float *sa,
+                     const float *sb, int64_t M, int64_t N, int64_t K, int64_t g, int64_t count,
+                     const int64_t *mi, const int64_t *ni, double *ref, uint16_t *out)
+{
+    int rc = check_args(layout, a, b, sa, sb, M, N, K, g);
+    int bad = 0;
+    if (rc)
+        return rc;
+    if (count < 0 || (count > 0 && (!mi || !ni)))
+        return OR_ERR_ARG;
+    for (int64_t i = 0; i < count; ++i)
+        if (mi[i] < 0 || mi[i] >= M || ni[i] < 0 || ni[i] >= N)
+            return OR_ERR_ARG;
+#pragma omp parallel for schedule(dynamic, 16) reduction(| : bad)
+    for (int64_t i = 0; i < count; ++i) {
+        double r;
+        bad |= one_element(layout, a, b, sa, sb, M, N, K, g, mi[i], ni[i], &r);
+        if (ref)
+            ref[i] = r;
+        if (out)
+            out[i] = oracle_bf16_rne(r);
+    }
+    return bad ? OR_ERR_NAN_INPUT : OR_OK;
+}
+
+/* Number of OpenMP threads the oracle would use (1 without OpenMP). */
+int oracle_num_threads(void)
+{
+#ifdef _OPENMP
+    extern int omp_get_max_threads(void);
+    return omp_get_max_threads();
+#else
+    return 1;
+#endif
+}
