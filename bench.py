@@ -1,0 +1,385 @@
+"""Benchmark of the B200 block-scaled FP8 GEMM (one JSON line on rank 0).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+A step is one call of the GEMM (the whole hot path: TMA operand fetch, scale
+fetch, tcgen05 MMA per K-block, FP32 scale promotion, split-K fix-up where the
+plan uses it, BF16 epilogue) on one batch of synthetic inputs.
+
+Default workload: the square 4096^3 NT GEMM with 128x128 block scales and 41
+outlier rows of A (x50).  Other workloads (``--workload``): tiny, ffn, ffn_tn,
+ffn_tt, small_m:<M>, long_k:<g>.
+
+Timing: W warm-up steps, then K timed steps.  Inputs are resident in HBM; the
+L2 cache is flushed (a 512 MiB memset) before every timed step, outside the
+events that bracket the GEMM itself.  CUDA events on the launching stream give
+the device time of each launch; the reported time per step is their mean and
+the whole-job value is total FLOPs / time, max over ranks.  ``e2e`` repeats the
+measurement through the public API with the inputs in pinned host memory:
+host->device copies, the GEMM and the device->host copy of the output are all
+inside the timed region.
+
+Multi-GPU (torchrun, one rank per GPU): every rank runs the same GEMM on its
+own GPU (replicas; the GEMM has no exchange step), the step time is the max
+over ranks and the value sums the ranks' work ("scaling": "weak").
+
+``--impl reference`` times the CPU oracle (the plain FP64 restatement used by
+the tests) on the host cores on a bounded sample of the same workload: rank 0
+only, the other ranks exit at once.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import workloads  # noqa: E402
+
+METRIC = "FP8 block-scaled GEMM TFLOP/s and % of B200 FP8/HBM roofline (1 GPU)"
+L2_FLUSH_BYTES = 512 << 20
+
+
+def parse_args(argv=None):
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=30)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default="square")
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0, help="target CPU seconds of the oracle sample")
+    return ap.parse_args(argv)
+
+
+# ---------------------------------------------------------------- workloads
+def make_workload(name: str) -> workloads.Problem:
+    if name == "square":
+        return workloads.square()
+    if name == "tiny":
+        return workloads.tiny()
+    if name in ("ffn", "ffn_nt"):
+        return workloads.ffn(layout="nt")
+    if name == "ffn_tn":
+        return workloads.ffn(layout="tn")
+    if name == "ffn_tt":
+        return workloads.ffn(layout="tt")
+    if name.startswith("small_m:"):
+        return workloads.small_m(int(name.split(":")[1]))
+    if name.startswith("long_k:"):
+        return workloads.long_k(gran=int(name.split(":")[1]))
+    raise SystemExit(f"unknown workload {name}")
+
+
+def workload_config(p: workloads.Problem, name: str) -> dict:
+    return {"workload": p.name, "name": name, "M": p.M, "N": p.N, "K": p.K, "gran": p.gran,
+            "layout": p.layout, "inputs": "E4M3 codes + FP32 block scales, seeded synthetic",
+            "l2": "flushed (512 MiB memset) before every timed step"}
+
+
+def algorithmic_bytes(p: workloads.Problem) -> int:
+    kb = -(-p.K // p.gran)
+    return p.M * p.K + p.N * p.K + 2 * p.M * p.N + 4 * (-(-p.M // p.gran) + -(-p.N // p.gran)) * kb
+
+
+def measured_peaks() -> dict:
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return {"hbm_gbs": float(d["hbm_gbs"]), "bf16_tflops": float(d["bf16_tflops"]), "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "source": "fallback"}
+
+
+# ---------------------------------------------------------------- clocks
+class ClockSampler:
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+
+    def __enter__(self):
+        try:
+            fd, self.path = tempfile.mkstemp(prefix="bsgemm_clocks_", suffix=".csv")
+            os.close(fd)
+            self.fh = open(self.path, "w")
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.QUERY}",
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                         stdout=self.fh, stderr=subprocess.DEVNULL)
+            time.sleep(0.3)
+        except Exception:
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            time.sleep(0.2)
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+            self.fh.close()
+
+    def summary(self):
+        if self.proc is None or not self.path or not os.path.exists(self.path):
+            return None
+        rows = []
+        for ln in open(self.path):
+            parts = [x.strip() for x in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                rows.append((float(parts[1]), float(parts[2]), parts[5:9]))
+            except ValueError:
+                continue
+        os.unlink(self.path)
+        if not rows:
+            return None
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for _, _, fl in rows for i, v in enumerate(fl) if v.lower() == "active"})
+        return {"sm_mhz": statistics.median(r[0] for r in rows), "sm_max_mhz": max(r[1] for r in rows),
+                "reasons": reasons, "samples": len(rows)}
+
+
+# ---------------------------------------------------------------- oracle baseline
+def cpu_baseline(p: workloads.Problem, seconds: float) -> dict:
+    """The oracle, as it stands, on a bounded sample of whole output rows."""
+    import oracle
+    # a first small probe sizes the sample to about `seconds` of CPU work
+    probe_rows = max(1, min(p.M, 2))
+    mi, ni = _rows_sample(p, probe_rows)
+    t0 = time.perf_counter()
+    oracle.bsgemm_at(p.layout, p.a, p.b, p.sa, p.sb, p.M, p.N, p.K, p.gran, mi, ni)
+    dt = max(time.perf_counter() - t0, 1e-6)
+    rows = int(max(1, min(p.M, probe_rows * seconds / dt)))
+    mi, ni = _rows_sample(p, rows)
+    t0 = time.perf_counter()
+    oracle.bsgemm_at(p.layout, p.a, p.b, p.sa, p.sb, p.M, p.N, p.K, p.gran, mi, ni)
+    dt = time.perf_counter() - t0
+    flops = 2.0 * rows * p.N * p.K
+    return {"value": flops / dt / 1e12, "unit": "TFLOP/s", "cores": oracle.num_threads(),
+            "kind": "oracle", "sample": f"{rows} full output rows of {p.M} ({rows * p.N} outputs), {dt:.1f} s",
+            "seconds": dt}
+
+
+def _rows_sample(p, rows):
+    step = max(1, p.M // rows)
+    r = (np.arange(rows, dtype=np.int64) * step) % p.M
+    mi = np.repeat(r, p.N)
+    ni = np.tile(np.arange(p.N, dtype=np.int64), rows)
+    return mi, ni
+
+
+# ---------------------------------------------------------------- distributed plumbing
+def dist_setup(n_gpus: int):
+    import torch
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(0)
+    return rank, world, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ---------------------------------------------------------------- our arm
+def run_ours(args):
+    import torch
+    import fp8_block_scaled_bsgemm_b200 as bsg
+
+    rank, world, local = dist_setup(args.gpus)
+    p = make_workload(args.workload)
+    dev = torch.device("cuda", local if world > 1 else 0)
+    stream = torch.cuda.current_stream(dev)
+    a = torch.from_numpy(p.a).to(dev)
+    b = torch.from_numpy(p.b).to(dev)
+    sa = torch.from_numpy(p.sa).to(dev)
+    sb = torch.from_numpy(p.sb).to(dev)
+    out = torch.empty((p.M, p.N), dtype=torch.bfloat16, device=dev)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    num_sms = torch.cuda.get_device_properties(dev).multi_processor_count
+    plan = bsg.make_plan(p.M, p.N, p.K, p.gran, p.layout, num_sms)
+
+    def gemm():
+        bsg.gemm(a, b, sa, sb, out=out, layout=p.layout, gran=p.gran, stream=stream)
+
+    for _ in range(args.warmup):
+        flush.zero_()
+        gemm()
+    torch.cuda.synchronize()
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    barrier(world)
+    torch.cuda.synchronize()
+    with ClockSampler(torch.cuda.current_device()) as clk:
+        t_wall = time.perf_counter()
+        for i in range(args.steps):
+            flush.zero_()
+            starts[i].record(stream)
+            gemm()
+            ends[i].record(stream)
+        torch.cuda.synchronize()
+        t_wall = time.perf_counter() - t_wall
+    barrier(world)
+    times_ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
+    ms = sum(times_ms) / len(times_ms)
+    ms_max = max_over_ranks(ms, world)
+    status = bsg.get_last_device_status(stream)
+    if status != 0:
+        raise SystemExit(f"device status {status} after the timed region")
+
+    # ---- e2e through the public API from pinned host memory
+    e2e = None
+    if not args.no_e2e:
+        ha = torch.from_numpy(p.a).pin_memory()
+        hb = torch.from_numpy(p.b).pin_memory()
+        hsa = torch.from_numpy(p.sa).pin_memory()
+        hsb = torch.from_numpy(p.sb).pin_memory()
+        hout = torch.empty((p.M, p.N), dtype=torch.bfloat16).pin_memory()
+        da, db, dsa, dsb = (torch.empty_like(x, device=dev) for x in (ha, hb, hsa, hsb))
+
+        def e2e_step():
+            da.copy_(ha, non_blocking=True)
+            db.copy_(hb, non_blocking=True)
+            dsa.copy_(hsa, non_blocking=True)
+            dsb.copy_(hsb, non_blocking=True)
+            bsg.gemm(da, db, dsa, dsb, out=out, layout=p.layout, gran=p.gran, stream=stream)
+            hout.copy_(out, non_blocking=True)
+
+        for _ in range(max(1, args.warmup)):
+            e2e_step()
+        torch.cuda.synchronize()
+        es = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+        ee = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+        barrier(world)
+        for i in range(args.steps):
+            flush.zero_()
+            es[i].record(stream)
+            e2e_step()
+            ee[i].record(stream)
+        torch.cuda.synchronize()
+        barrier(world)
+        e_ms = max_over_ranks(sum(s.elapsed_time(e) for s, e in zip(es, ee)) / args.steps, world)
+        h2d = sum(x.numel() * x.element_size() for x in (ha, hb, hsa, hsb))
+        e2e = {"value": world * p.flops / (e_ms * 1e-3) / 1e12, "unit": "TFLOP/s", "ms_per_step": e_ms,
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": hout.numel() * hout.element_size()}
+
+    if rank != 0:
+        _finish(world)
+        return
+    peaks = measured_peaks()
+    bound = "hbm" if p.M <= 128 else "tensor"
+    if bound == "tensor":
+        # FP8 dense peak = measured BF16 burst x the nominal FP8/BF16 ratio (4.5 / 2.25)
+        peak = peaks["bf16_tflops"] * 2.0
+        achieved = p.flops / (ms * 1e-3) / 1e12
+        roof = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                "frac": achieved / peak, "traffic": None,
+                "peak_source": f"{peaks['source']} bf16 burst x 2 (FP8/BF16 nominal ratio)",
+                "frac_of_nominal_4500": achieved / 4500.0}
+    else:
+        bytes_ = algorithmic_bytes(p)
+        peak = peaks["hbm_gbs"]
+        achieved = bytes_ / (ms * 1e-3) / 1e9
+        roof = {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                "frac": achieved / peak, "traffic": None, "peak_source": f"{peaks['source']} hbm copy",
+                "algorithmic_bytes_per_launch": bytes_}
+    line = {
+        "metric": METRIC, "value": world * p.flops / (ms_max * 1e-3) / 1e12, "unit": "TFLOP/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_max,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "fp8_e4m3",
+        "data": "synthetic", "config": workload_config(p, args.workload) | {"parallelism": f"replicas{world}",
+                                                                              "plan": plan},
+        "roofline": roof, "e2e": e2e, "gpu_launches": args.steps * plan["kernels"],
+        "clocks": clk.summary(), "wall_s_timed_region": t_wall,
+        "min_ms": min(times_ms), "median_ms": statistics.median(times_ms),
+    }
+    if not args.no_cpu_baseline and world == 1:
+        line["cpu_baseline"] = cpu_baseline(p, args.cpu_seconds)
+    else:
+        line["cpu_baseline"] = None
+    print(json.dumps(line), flush=True)
+    _finish(world)
+
+
+def _finish(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+# ---------------------------------------------------------------- reference arm (the oracle)
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    import oracle
+    p = make_workload(args.workload)
+    budget = max(1.0, 150.0 / max(1, args.steps + args.warmup))  # whole run within a few minutes
+    per = []
+    for i in range(args.warmup + args.steps):
+        r = cpu_baseline(p, min(budget, args.cpu_seconds))
+        if i >= args.warmup:
+            per.append(r)
+    value = statistics.mean(r["value"] for r in per)
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": statistics.mean(r["seconds"] for r in per) * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "config": workload_config(p, args.workload),
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": oracle.num_threads(), "kind": "oracle",
+                         "sample": per[-1]["sample"] + " per step"},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main(argv=None):
+    args = parse_args(argv)
+    if args.warmup < 3 and args.impl == "ours":
+        print("warning: fewer than 3 warm-up steps", file=sys.stderr)
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,180 @@
+"""Python binding of the B200 block-scaled FP8 GEMM C ABI (``include/bsgemm.h``).
+
+Argument marshalling only: every step of the GEMM runs in ``libbsgemm.so``'s
+CUDA kernels.  PyTorch supplies device memory and streams.  There is no CPU
+path: if the library is missing (and cannot be built here) every call raises.
+
+    out = bsgemm_fp8_nt(a, b, scale_a, scale_b)          # a [M,K], b [N,K]
+    out = gemm(a, b, scale_a, scale_b, layout="tn")      # a [K,M], b [K,N]
+
+Operation (hncyxsy.com/news/191052 §2.2, §3.2, §4.2):
+out[m,n] = bf16(sum_kb sA[m/g][kb] * sB[n/g][kb] * sum_{k in kb} A[m,k] B[n,k]).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libbsgemm.so")
+
+LAYOUTS = {"nt": 0, "tn": 1, "nn": 2, "tt": 3}
+VARIANTS = {"auto": 0, "data_parallel": 1, "swap_ab": 2}
+STATUS = {0: "ok", 1: "invalid argument", 2: "unsupported granularity", 3: "misaligned",
+          4: "unsupported device", 5: "CUDA error", 6: "device wait timeout"}
+
+_lock = threading.Lock()
+_lib = None
+
+
+class BsgemmError(RuntimeError):
+    def __init__(self, status: int, what: str = ""):
+        self.status = status
+        super().__init__(f"{what}: {STATUS.get(status, 'unknown')} (status {status})")
+
+
+class Tuning(ctypes.Structure):
+    _fields_ = [("variant", ctypes.c_int), ("bnq", ctypes.c_int), ("splits", ctypes.c_int)]
+
+
+class Plan(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_int) for n in ("layout", "gran", "swap_ab", "bnq", "tiles_p", "tiles_q",
+                                            "splits", "kb_per_split", "grid", "group_p", "kernels")]
+
+    def as_dict(self):
+        return {n: getattr(self, n) for n, _ in self._fields_}
+
+
+EXPORTS = ("bsgemm_fp8_nt", "bsgemm_fp8_tn", "bsgemm_fp8_nn", "bsgemm_fp8_tt", "bsgemm_fp8_gemm_ex",
+           "bsgemm_make_plan", "bsgemm_status_string", "bsgemm_get_last_device_status",
+           "bsgemm_last_device_status_detail", "bsgemm_diag_wait_timeout", "bsgemm_version")
+
+
+def lib():
+    """Load ``libbsgemm.so`` (building it first if it is missing and nvcc exists)."""
+    global _lib
+    with _lock:
+        if _lib is None:
+            if not os.path.exists(LIB_PATH):
+                from . import build as _build
+                _build.build()
+            L = ctypes.CDLL(LIB_PATH)
+            p, i64, i32 = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int
+            gemm_args = [p, p, p, p, p, i64, i64, i64, i32, p]
+            for name in ("bsgemm_fp8_nt", "bsgemm_fp8_tn", "bsgemm_fp8_nn", "bsgemm_fp8_tt"):
+                getattr(L, name).argtypes = gemm_args
+                getattr(L, name).restype = i32
+            L.bsgemm_fp8_gemm_ex.argtypes = [i32, p, p, p, p, p, i64, i64, i64, i32,
+                                             ctypes.POINTER(Tuning), p]
+            L.bsgemm_fp8_gemm_ex.restype = i32
+            L.bsgemm_make_plan.argtypes = [i32, i64, i64, i64, i32, i32, ctypes.POINTER(Tuning),
+                                           ctypes.POINTER(Plan)]
+            L.bsgemm_make_plan.restype = i32
+            L.bsgemm_status_string.argtypes = [i32]
+            L.bsgemm_status_string.restype = ctypes.c_char_p
+            L.bsgemm_get_last_device_status.argtypes = [p]
+            L.bsgemm_get_last_device_status.restype = i32
+            L.bsgemm_last_device_status_detail.argtypes = []
+            L.bsgemm_last_device_status_detail.restype = i32
+            L.bsgemm_diag_wait_timeout.argtypes = [ctypes.c_ulonglong, p]
+            L.bsgemm_diag_wait_timeout.restype = i32
+            L.bsgemm_version.argtypes = []
+            L.bsgemm_version.restype = i32
+            _lib = L
+    return _lib
+
+
+def status_string(status: int) -> str:
+    return lib().bsgemm_status_string(int(status)).decode()
+
+
+def _stream_handle(stream) -> int:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return int(stream.cuda_stream) if hasattr(stream, "cuda_stream") else int(stream)
+
+
+def _tuning(tuning):
+    if tuning is None:
+        return None
+    if isinstance(tuning, Tuning):
+        return ctypes.byref(tuning)
+    t = Tuning(VARIANTS[tuning.get("variant", "auto")], int(tuning.get("bnq", 0)),
+               int(tuning.get("splits", 0)))
+    return ctypes.byref(t)
+
+
+def _as_bytes(x: torch.Tensor, name: str) -> torch.Tensor:
+    if x.dtype not in (torch.float8_e4m3fn, torch.uint8):
+        raise TypeError(f"{name} must be float8_e4m3fn or uint8 codes, got {x.dtype}")
+    if not x.is_cuda or not x.is_contiguous():
+        raise ValueError(f"{name} must be a contiguous CUDA tensor")
+    return x
+
+
+def shapes(layout: str, a: torch.Tensor, b: torch.Tensor):
+    """(M, N, K) from the stored shapes of a and b for a layout."""
+    if a.dim() != 2 or b.dim() != 2:
+        raise ValueError("a and b must be 2-D")
+    M, Ka = (a.shape[1], a.shape[0]) if layout[0] == "t" else (a.shape[0], a.shape[1])
+    N, Kb = (b.shape[0], b.shape[1]) if layout[1] == "t" else (b.shape[1], b.shape[0])
+    if Ka != Kb:
+        raise ValueError(f"K mismatch: {Ka} vs {Kb}")
+    return int(M), int(N), int(Ka)
+
+
+def gemm(a, b, scale_a, scale_b, out=None, layout="nt", gran=128, tuning=None, stream=None):
+    """out[M,N] (BF16) of the block-scaled FP8 GEMM; see ``include/bsgemm.h``."""
+    if layout not in LAYOUTS:
+        raise ValueError(f"layout must be one of {sorted(LAYOUTS)}")
+    a = _as_bytes(a, "a")
+    b = _as_bytes(b, "b")
+    M, N, K = shapes(layout, a, b)
+    for s, nm in ((scale_a, "scale_a"), (scale_b, "scale_b")):
+        if s.dtype != torch.float32 or not s.is_cuda or not s.is_contiguous():
+            raise ValueError(f"{nm} must be a contiguous float32 CUDA tensor")
+    if out is None:
+        out = torch.empty((M, N), dtype=torch.bfloat16, device=a.device)
+    if out.dtype != torch.bfloat16 or tuple(out.shape) != (M, N) or not out.is_contiguous():
+        raise ValueError("out must be a contiguous bfloat16 [M, N] tensor")
+    st = lib().bsgemm_fp8_gemm_ex(LAYOUTS[layout], a.data_ptr(), b.data_ptr(), scale_a.data_ptr(),
+                                  scale_b.data_ptr(), out.data_ptr(), M, N, K, int(gran),
+                                  _tuning(tuning), _stream_handle(stream))
+    if st != 0:
+        raise BsgemmError(st, f"bsgemm {layout} M={M} N={N} K={K} g={gran}")
+    return out
+
+
+def bsgemm_fp8_nt(a, b, scale_a, scale_b, out=None, gran=128, stream=None):
+    return gemm(a, b, scale_a, scale_b, out, "nt", gran, None, stream)
+
+
+def bsgemm_fp8_tn(a, b, scale_a, scale_b, out=None, gran=128, stream=None):
+    return gemm(a, b, scale_a, scale_b, out, "tn", gran, None, stream)
+
+
+def bsgemm_fp8_nn(a, b, scale_a, scale_b, out=None, gran=128, stream=None):
+    return gemm(a, b, scale_a, scale_b, out, "nn", gran, None, stream)
+
+
+def bsgemm_fp8_tt(a, b, scale_a, scale_b, out=None, gran=128, stream=None):
+    return gemm(a, b, scale_a, scale_b, out, "tt", gran, None, stream)
+
+
+def make_plan(M, N, K, gran=128, layout="nt", num_sms=148, tuning=None) -> dict:
+    pl = Plan()
+    st = lib().bsgemm_make_plan(LAYOUTS[layout], M, N, K, gran, num_sms, _tuning(tuning), ctypes.byref(pl))
+    if st != 0:
+        raise BsgemmError(st, "bsgemm_make_plan")
+    return pl.as_dict()
+
+
+def get_last_device_status(stream=None) -> int:
+    return int(lib().bsgemm_get_last_device_status(_stream_handle(stream)))
+
+
+def diag_wait_timeout(timeout_ns: int, stream=None) -> int:
+    return int(lib().bsgemm_diag_wait_timeout(int(timeout_ns), _stream_handle(stream)))

@@ -1,0 +1,340 @@
+// C ABI of the block-scaled FP8 GEMM library: argument checks, plan choice,
+// TMA descriptor encoding, split-K workspace, launches and device status.
+// The operation and every argument convention are documented in bsgemm.h.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <cstdint>
+#include <cstdlib>
+#include <cstring>
+#include <map>
+#include <mutex>
+#include <utility>
+
+#include "bsgemm.h"
+#include "bsgemm_host.h"
+#include "bsgemm_kernel.cuh"
+
+using bsg::Params;
+using bsg_host::DeviceInfo;
+using bsg_host::Workspace;
+
+namespace {
+__device__ int g_device_status;  // BSGEMM_OK or a timeout code (low byte) | where << 8
+}  // namespace
+
+namespace bsg_host {
+namespace {
+
+// ------------------------------------------------------------------ driver entry point
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+  });
+  return fn;
+}
+
+}  // namespace
+
+// 2D tensor map with 128-byte swizzle. `inner` is the contiguous extent.
+bool make_map_2d(CUtensorMap* m, const void* base, CUtensorMapDataType dt, uint64_t inner,
+                 uint64_t outer, uint64_t row_stride_bytes, uint32_t box_inner, uint32_t box_outer) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {inner, outer};
+  cuuint64_t strides[1] = {row_stride_bytes};
+  cuuint32_t box[2] = {box_inner, box_outer};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(m, dt, 2, const_cast<void*>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+// ------------------------------------------------------------------ per-device state
+std::mutex g_mu;
+std::map<int, DeviceInfo> g_dev;
+std::map<std::pair<int, uintptr_t>, Workspace> g_ws;
+
+bsgemm_status device_info(DeviceInfo& out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return BSGEMM_ERR_CUDA;
+  std::lock_guard<std::mutex> lk(g_mu);
+  auto it = g_dev.find(dev);
+  if (it == g_dev.end()) {
+    DeviceInfo d;
+    int major = 0, minor = 0;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&d.num_sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+      return BSGEMM_ERR_CUDA;
+    d.ok = (major == 10 && minor == 0);
+    if (d.ok) {
+      void* p = nullptr;
+      if (cudaGetSymbolAddress(&p, g_device_status) != cudaSuccess) return BSGEMM_ERR_CUDA;
+      d.status = static_cast<int*>(p);
+    }
+    it = g_dev.emplace(dev, d).first;
+  }
+  out = it->second;
+  return out.ok ? BSGEMM_OK : BSGEMM_ERR_UNSUPPORTED_DEVICE;
+}
+
+// Workspace of at least `ws_bytes` and `n_counters` zeroed counters for
+// (current device, stream). Growing frees the old buffers (cudaFree waits for
+// the device, so no launch still uses them).
+bsgemm_status get_workspace(cudaStream_t stream, size_t ws_bytes, size_t n_counters, Workspace& out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return BSGEMM_ERR_CUDA;
+  std::lock_guard<std::mutex> lk(g_mu);
+  Workspace& w = g_ws[{dev, reinterpret_cast<uintptr_t>(stream)}];
+  if (w.ws_bytes < ws_bytes) {
+    if (w.ws) cudaFree(w.ws);
+    w.ws = nullptr;
+    w.ws_bytes = 0;
+    size_t want = ws_bytes + ws_bytes / 4;
+    if (cudaMalloc(&w.ws, want) != cudaSuccess) return BSGEMM_ERR_CUDA;
+    w.ws_bytes = want;
+  }
+  if (w.n_counters < n_counters) {
+    if (w.counters) cudaFree(w.counters);
+    w.counters = nullptr;
+    w.n_counters = 0;
+    size_t want = n_counters < 1024 ? 1024 : n_counters * 2;
+    if (cudaMalloc(&w.counters, want * sizeof(int)) != cudaSuccess) return BSGEMM_ERR_CUDA;
+    if (cudaMemset(w.counters, 0, want * sizeof(int)) != cudaSuccess) return BSGEMM_ERR_CUDA;
+    w.n_counters = want;
+  }
+  out = w;
+  return BSGEMM_OK;
+}
+
+unsigned long long wait_timeout_ns() {
+  static unsigned long long t = [] {
+    const char* e = std::getenv("BSGEMM_WAIT_TIMEOUT_NS");
+    unsigned long long v = e ? std::strtoull(e, nullptr, 10) : 0ull;
+    return v ? v : 1000000000ull;  // 1 s
+  }();
+  return t;
+}
+
+}  // namespace bsg_host
+
+namespace {
+using bsg_host::device_info;
+
+// ------------------------------------------------------------------ checks
+bool aligned(const void* p, uintptr_t n) { return (reinterpret_cast<uintptr_t>(p) % n) == 0; }
+
+bsgemm_status check_args(int layout, const void* a, const void* b, const float* sa, const float* sb,
+                         const void* out, int64_t M, int64_t N, int64_t K, int gran) {
+  if (layout < BSGEMM_LAYOUT_NT || layout > BSGEMM_LAYOUT_TT) return BSGEMM_ERR_INVALID_ARG;
+  if (!a || !b || !sa || !sb || !out) return BSGEMM_ERR_INVALID_ARG;
+  if (M <= 0 || N <= 0 || K <= 0) return BSGEMM_ERR_INVALID_ARG;
+  // TMA coordinates and the kernel's index math are 32-bit
+  if (M > (1 << 30) || N > (1 << 30) || K > (1 << 30)) return BSGEMM_ERR_INVALID_ARG;
+  if (gran != 64 && gran != 128 && gran != 256) return BSGEMM_ERR_UNSUPPORTED_GRAN;
+  if (!aligned(a, 16) || !aligned(b, 16) || !aligned(out, 16) || !aligned(sa, 4) || !aligned(sb, 4))
+    return BSGEMM_ERR_MISALIGNED;
+  const bool a_mn = (layout == BSGEMM_LAYOUT_TN || layout == BSGEMM_LAYOUT_TT);
+  const bool b_mn = (layout == BSGEMM_LAYOUT_TN || layout == BSGEMM_LAYOUT_NN);
+  if (a_mn ? (M % 16) : (K % 16)) return BSGEMM_ERR_MISALIGNED;
+  if (b_mn ? (N % 16) : (K % 16)) return BSGEMM_ERR_MISALIGNED;
+  if (N % 8) return BSGEMM_ERR_MISALIGNED;
+  return BSGEMM_OK;
+}
+
+int pow2_at_least(int x, int lo) {
+  int v = lo;
+  while (v < x) v *= 2;
+  return v;
+}
+
+}  // namespace
+
+// ------------------------------------------------------------------ plan
+extern "C" bsgemm_status bsgemm_make_plan(int layout, int64_t M, int64_t N, int64_t K, int gran,
+                                          int num_sms, const bsgemm_tuning* t, bsgemm_plan* plan) {
+  if (!plan || num_sms <= 0) return BSGEMM_ERR_INVALID_ARG;
+  if (layout < BSGEMM_LAYOUT_NT || layout > BSGEMM_LAYOUT_TT) return BSGEMM_ERR_INVALID_ARG;
+  if (M <= 0 || N <= 0 || K <= 0) return BSGEMM_ERR_INVALID_ARG;
+  if (gran != 64 && gran != 128 && gran != 256) return BSGEMM_ERR_UNSUPPORTED_GRAN;
+  bsgemm_plan pl{};
+  const int Kb = static_cast<int>((K + gran - 1) / gran);
+  int variant = t ? t->variant : BSGEMM_VARIANT_AUTO;
+  if (variant == BSGEMM_VARIANT_AUTO) variant = (M <= 128) ? BSGEMM_VARIANT_SWAP_AB : BSGEMM_VARIANT_DATA_PARALLEL;
+  if (variant != BSGEMM_VARIANT_SWAP_AB && variant != BSGEMM_VARIANT_DATA_PARALLEL) return BSGEMM_ERR_INVALID_ARG;
+  pl.swap_ab = (variant == BSGEMM_VARIANT_SWAP_AB);
+  const int64_t P = pl.swap_ab ? N : M;
+  const int64_t Q = pl.swap_ab ? M : N;
+  int bnq = t ? t->bnq : 0;
+  if (bnq == 0) bnq = pl.swap_ab ? pow2_at_least(static_cast<int>(Q < 128 ? Q : 128), 16) : (Q <= 128 ? 128 : 256);
+  if (pl.swap_ab ? (bnq != 16 && bnq != 32 && bnq != 64 && bnq != 128) : (bnq != 128 && bnq != 256))
+    return BSGEMM_ERR_INVALID_ARG;
+  pl.bnq = bnq;
+  pl.tiles_p = static_cast<int>((P + bsg::BM - 1) / bsg::BM);
+  pl.tiles_q = static_cast<int>((Q + bnq - 1) / bnq);
+  const int64_t tiles = static_cast<int64_t>(pl.tiles_p) * pl.tiles_q;
+  if (tiles > (1 << 30)) return BSGEMM_ERR_INVALID_ARG;
+  int splits = t ? t->splits : 0;
+  if (splits <= 0) {
+    // fill the SMs when there are too few tiles; keep >= 4 K-blocks per split
+    splits = 1;
+    if (tiles < num_sms) {
+      int s = static_cast<int>(num_sms / tiles);
+      int max_s = Kb / 4 > 1 ? Kb / 4 : 1;
+      splits = s < max_s ? s : max_s;
+      if (splits < 1) splits = 1;
+    }
+  }
+  if (splits > Kb) splits = Kb;
+  int per = (Kb + splits - 1) / splits;
+  if (gran == 64 && (per & 1)) ++per;  // a split starts on a 128-element stage
+  pl.kb_per_split = per;
+  pl.splits = (Kb + per - 1) / per;
+  const int64_t work = tiles * pl.splits;
+  pl.grid = static_cast<int>(work < num_sms ? work : num_sms);
+  pl.group_p = 16;
+  pl.layout = layout;
+  pl.gran = gran;
+  pl.kernels = 1;
+  *plan = pl;
+  return BSGEMM_OK;
+}
+
+// ------------------------------------------------------------------ entry points
+extern "C" bsgemm_status bsgemm_fp8_gemm_ex(int layout, const void* a, const void* b,
+                                            const float* scale_a, const float* scale_b, void* out,
+                                            int64_t M, int64_t N, int64_t K, int gran,
+                                            const bsgemm_tuning* tuning, bsgemm_stream_t stream) {
+  bsgemm_status st = check_args(layout, a, b, scale_a, scale_b, out, M, N, K, gran);
+  if (st != BSGEMM_OK) return st;
+  DeviceInfo dev;
+  st = device_info(dev);
+  if (st != BSGEMM_OK) return st;
+  bsgemm_plan pl;
+  st = bsgemm_make_plan(layout, M, N, K, gran, dev.num_sms, tuning, &pl);
+  if (st != BSGEMM_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const int m = static_cast<int>(M), n = static_cast<int>(N), k = static_cast<int>(K);
+#define BSG_RUN(G, L) bsg_host::run_g##G##_##L(pl, a, b, scale_a, scale_b, out, m, n, k, s, dev)
+#define BSG_RUN_LAYOUTS(G)                              \
+  switch (layout) {                                     \
+    case BSGEMM_LAYOUT_NT: return BSG_RUN(G, nt);       \
+    case BSGEMM_LAYOUT_TN: return BSG_RUN(G, tn);       \
+    case BSGEMM_LAYOUT_NN: return BSG_RUN(G, nn);       \
+    default:               return BSG_RUN(G, tt);       \
+  }
+  switch (gran) {
+    case 64:  BSG_RUN_LAYOUTS(64)
+    case 128: BSG_RUN_LAYOUTS(128)
+    default:  BSG_RUN_LAYOUTS(256)
+  }
+#undef BSG_RUN_LAYOUTS
+#undef BSG_RUN
+}
+
+extern "C" bsgemm_status bsgemm_fp8_nt(const void* a, const void* b, const float* sa, const float* sb,
+                                       void* out, int64_t M, int64_t N, int64_t K, int gran,
+                                       bsgemm_stream_t stream) {
+  return bsgemm_fp8_gemm_ex(BSGEMM_LAYOUT_NT, a, b, sa, sb, out, M, N, K, gran, nullptr, stream);
+}
+
+extern "C" bsgemm_status bsgemm_fp8_tn(const void* a, const void* b, const float* sa, const float* sb,
+                                       void* out, int64_t M, int64_t N, int64_t K, int gran,
+                                       bsgemm_stream_t stream) {
+  return bsgemm_fp8_gemm_ex(BSGEMM_LAYOUT_TN, a, b, sa, sb, out, M, N, K, gran, nullptr, stream);
+}
+
+extern "C" bsgemm_status bsgemm_fp8_nn(const void* a, const void* b, const float* sa, const float* sb,
+                                       void* out, int64_t M, int64_t N, int64_t K, int gran,
+                                       bsgemm_stream_t stream) {
+  return bsgemm_fp8_gemm_ex(BSGEMM_LAYOUT_NN, a, b, sa, sb, out, M, N, K, gran, nullptr, stream);
+}
+
+extern "C" bsgemm_status bsgemm_fp8_tt(const void* a, const void* b, const float* sa, const float* sb,
+                                       void* out, int64_t M, int64_t N, int64_t K, int gran,
+                                       bsgemm_stream_t stream) {
+  return bsgemm_fp8_gemm_ex(BSGEMM_LAYOUT_TT, a, b, sa, sb, out, M, N, K, gran, nullptr, stream);
+}
+
+extern "C" const char* bsgemm_status_string(bsgemm_status s) {
+  switch (s) {
+    case BSGEMM_OK: return "ok";
+    case BSGEMM_ERR_INVALID_ARG: return "invalid argument";
+    case BSGEMM_ERR_UNSUPPORTED_GRAN: return "unsupported granularity (use 64, 128 or 256)";
+    case BSGEMM_ERR_MISALIGNED: return "misaligned pointer or stride (TMA needs 16-byte rows)";
+    case BSGEMM_ERR_UNSUPPORTED_DEVICE: return "current device is not sm_100 (B200)";
+    case BSGEMM_ERR_CUDA: return "CUDA runtime or driver call failed";
+    case BSGEMM_ERR_DEVICE_TIMEOUT: return "a bounded device-side wait timed out";
+  }
+  return "unknown status";
+}
+
+extern "C" bsgemm_status bsgemm_get_last_device_status(bsgemm_stream_t stream) {
+  DeviceInfo dev;
+  bsgemm_status st = device_info(dev);
+  if (st != BSGEMM_OK) return st;
+  if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return BSGEMM_ERR_CUDA;
+  int v = 0;
+  if (cudaMemcpyFromSymbol(&v, g_device_status, sizeof v) != cudaSuccess) return BSGEMM_ERR_CUDA;
+  if (v == 0) return BSGEMM_OK;
+  const int zero = 0;
+  if (cudaMemcpyToSymbol(g_device_status, &zero, sizeof zero) != cudaSuccess) return BSGEMM_ERR_CUDA;
+  // an aborted split-K launch may have left tile counters raised: clear them
+  int cur = 0;
+  cudaGetDevice(&cur);
+  {
+    std::lock_guard<std::mutex> lk(bsg_host::g_mu);
+    for (auto& kv : bsg_host::g_ws)
+      if (kv.first.first == cur && kv.second.counters)
+        cudaMemset(kv.second.counters, 0, kv.second.n_counters * sizeof(int));
+  }
+  if (cudaDeviceSynchronize() != cudaSuccess) return BSGEMM_ERR_CUDA;
+  return static_cast<bsgemm_status>(v & 0xFF);
+}
+
+extern "C" int bsgemm_last_device_status_detail(void) {
+  int v = 0;
+  if (cudaMemcpyFromSymbol(&v, g_device_status, sizeof v) != cudaSuccess) return -1;
+  return v;
+}
+
+// ------------------------------------------------------------------ diagnostics
+namespace {
+// One CTA waits on an mbarrier that nothing ever completes; the bounded wait
+// must give up after `timeout_ns`, record the timeout and return.
+__global__ void wait_timeout_probe(Params p) {
+  __shared__ bsg::Barriers bars;
+  if (threadIdx.x == 0) {
+    bsg::mbar_init(bsg::smem_addr(&bars.full[0]), 1);
+    bars.abort_flag = 0;
+    bsg::fence_barrier_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) bsg::bounded_wait(bsg::smem_addr(&bars.full[0]), 0, p, &bars, 7);
+  __syncwarp();
+  __syncthreads();
+}
+}  // namespace
+
+extern "C" bsgemm_status bsgemm_diag_wait_timeout(unsigned long long timeout_ns, bsgemm_stream_t stream) {
+  DeviceInfo dev;
+  bsgemm_status st = device_info(dev);
+  if (st != BSGEMM_OK) return st;
+  if (timeout_ns == 0 || timeout_ns > 10000000000ull) return BSGEMM_ERR_INVALID_ARG;
+  Params p{};
+  p.status = dev.status;
+  p.timeout_ns = timeout_ns;
+  wait_timeout_probe<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(p);
+  return cudaGetLastError() == cudaSuccess ? BSGEMM_OK : BSGEMM_ERR_CUDA;
+}
+
+extern "C" int bsgemm_version(void) { return 100; }

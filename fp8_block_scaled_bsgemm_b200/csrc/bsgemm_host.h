@@ -1,0 +1,47 @@
+// Host-side pieces shared by the C ABI (bsgemm_api.cu) and the kernel
+// instance units (bsgemm_inst.cu, compiled once per granularity and layout).
+#pragma once
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cstddef>
+#include <cstdint>
+
+#include "bsgemm.h"
+
+namespace bsg_host {
+
+struct DeviceInfo {
+  bool ok = false;
+  int num_sms = 0;
+  int* status = nullptr;  // device address of the status word
+};
+
+struct Workspace {
+  float* ws = nullptr;
+  size_t ws_bytes = 0;
+  int* counters = nullptr;
+  size_t n_counters = 0;
+};
+
+// 2D tensor map with 128-byte swizzle; `inner` is the contiguous extent.
+bool make_map_2d(CUtensorMap* m, const void* base, CUtensorMapDataType dt, uint64_t inner,
+                 uint64_t outer, uint64_t row_stride_bytes, uint32_t box_inner, uint32_t box_outer);
+
+// Split-K workspace of at least `ws_bytes` bytes and `n_counters` zeroed
+// counters for (current device, stream).
+bsgemm_status get_workspace(cudaStream_t stream, size_t ws_bytes, size_t n_counters, Workspace& out);
+
+// Limit of every bounded device-side wait, in nanoseconds.
+unsigned long long wait_timeout_ns();
+
+#define BSG_RUN_DECL(G, L)                                                                       \
+  bsgemm_status run_g##G##_##L(const bsgemm_plan& plan, const void* a, const void* b,          \
+                               const float* sa, const float* sb, void* out, int M, int N, int K, \
+                               cudaStream_t stream, const DeviceInfo& dev);
+BSG_RUN_DECL(64, nt) BSG_RUN_DECL(64, tn) BSG_RUN_DECL(64, nn) BSG_RUN_DECL(64, tt)
+BSG_RUN_DECL(128, nt) BSG_RUN_DECL(128, tn) BSG_RUN_DECL(128, nn) BSG_RUN_DECL(128, tt)
+BSG_RUN_DECL(256, nt) BSG_RUN_DECL(256, tn) BSG_RUN_DECL(256, nn) BSG_RUN_DECL(256, tt)
+#undef BSG_RUN_DECL
+
+}  // namespace bsg_host

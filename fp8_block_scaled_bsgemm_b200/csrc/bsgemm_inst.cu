@@ -1,0 +1,123 @@
+// Kernel instances and launch code for one (granularity, layout) pair.
+// The build compiles this file once per pair with -DBSG_GRAN=<64|128|256>
+// and -DBSG_LAYOUT=<nt|tn|nn|tt>, so the twelve pairs build in parallel.
+#include <cstring>
+
+#include "bsgemm_host.h"
+#include "bsgemm_kernel.cuh"
+
+#ifndef BSG_GRAN
+#error "compile with -DBSG_GRAN=64|128|256"
+#endif
+#ifndef BSG_LAYOUT
+#error "compile with -DBSG_LAYOUT=nt|tn|nn|tt"
+#endif
+
+#define BSG_CAT2(a, b, c, d) a##b##_##c
+#define BSG_RUN_NAME(G, L) BSG_CAT2(run_g, G, L, )
+#define BSG_STR2(x) #x
+#define BSG_STR(x) BSG_STR2(x)
+
+namespace bsg_host {
+namespace {
+
+// A stored [K,M] for tn/tt; B stored [K,N] for tn/nn (first letter A, second B).
+constexpr const char* kLayout = BSG_STR(BSG_LAYOUT);
+constexpr bool kAMn = kLayout[0] == 't';
+constexpr bool kBMn = kLayout[1] == 'n';
+
+template <int BNQ, int GRAN, bool SWAP, bool P_MN, bool Q_MN, bool SPLIT>
+bsgemm_status launch(const bsgemm_plan& plan, const void* a, const void* b, const float* sa,
+                     const float* sb, void* out, int M, int N, int K, cudaStream_t stream,
+                     const DeviceInfo& dev) {
+  using SC = bsg::StageCfg<BNQ, Q_MN, SWAP>;
+  auto kern = bsg::bsgemm_kernel<BNQ, GRAN, SWAP, P_MN, Q_MN, SPLIT>;
+
+  // P/Q operands: normally P = A (M rows), Q = B (N rows); swapped P = B, Q = A
+  const void* p_ptr = SWAP ? b : a;
+  const void* q_ptr = SWAP ? a : b;
+  const int P = SWAP ? N : M;
+  const int Q = SWAP ? M : N;
+  CUtensorMap tm_p, tm_q, tm_out;
+  bool ok = true;
+  if (P_MN) ok &= make_map_2d(&tm_p, p_ptr, CU_TENSOR_MAP_DATA_TYPE_UINT8, P, K, P, 128, bsg::BK);
+  else      ok &= make_map_2d(&tm_p, p_ptr, CU_TENSOR_MAP_DATA_TYPE_UINT8, K, P, K, bsg::BK, bsg::BM);
+  if (Q_MN) ok &= make_map_2d(&tm_q, q_ptr, CU_TENSOR_MAP_DATA_TYPE_UINT8, Q, K, Q, 128, bsg::BK);
+  else      ok &= make_map_2d(&tm_q, q_ptr, CU_TENSOR_MAP_DATA_TYPE_UINT8, K, Q, K, bsg::BK, BNQ);
+  if (!SWAP) ok &= make_map_2d(&tm_out, out, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, N, M, (uint64_t)N * 2, 64, 32);
+  else       std::memset(&tm_out, 0, sizeof tm_out);
+  if (!ok) return BSGEMM_ERR_CUDA;
+
+  bsg::Params prm{};
+  prm.M = M; prm.N = N; prm.K = K;
+  prm.P = P; prm.Q = Q;
+  prm.Kb = (K + GRAN - 1) / GRAN;
+  prm.Pb = (P + GRAN - 1) / GRAN;
+  prm.Qb = (Q + GRAN - 1) / GRAN;
+  prm.tiles_p = plan.tiles_p;
+  prm.tiles_q = plan.tiles_q;
+  prm.num_tiles = plan.tiles_p * plan.tiles_q;
+  prm.splits = plan.splits;
+  prm.kb_per_split = plan.kb_per_split;
+  prm.num_work = prm.num_tiles * plan.splits;
+  prm.group_p = plan.group_p;
+  prm.sP = SWAP ? sb : sa;
+  prm.sQ = SWAP ? sa : sb;
+  prm.out = static_cast<__nv_bfloat16*>(out);
+  prm.status = dev.status;
+  prm.timeout_ns = wait_timeout_ns();
+  if (SPLIT && plan.splits > 1) {
+    Workspace w;
+    bsgemm_status st = get_workspace(stream, (size_t)prm.num_work * BNQ * bsg::BM * sizeof(float),
+                                     (size_t)prm.num_tiles, w);
+    if (st != BSGEMM_OK) return st;
+    prm.ws = w.ws;
+    prm.counters = w.counters;
+  }
+
+  static bool attr_set = false;  // once per instance
+  if (!attr_set) {
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SC::kSmemBytes) != cudaSuccess)
+      return BSGEMM_ERR_CUDA;
+    if (bsg::RegSplit<BNQ>::kEnabled) {
+      // the setmaxnreg split is only safe with exactly the planned launch registers
+      cudaFuncAttributes fa{};
+      if (cudaFuncGetAttributes(&fa, kern) != cudaSuccess || fa.numRegs != bsg::kLaunchRegs)
+        return BSGEMM_ERR_CUDA;
+    }
+    attr_set = true;
+  }
+  kern<<<plan.grid, bsg::kNumThreads, SC::kSmemBytes, stream>>>(tm_p, tm_q, tm_out, prm);
+  return cudaGetLastError() == cudaSuccess ? BSGEMM_OK : BSGEMM_ERR_CUDA;
+}
+
+}  // namespace
+
+bsgemm_status BSG_RUN_NAME(BSG_GRAN, BSG_LAYOUT)(const bsgemm_plan& pl, const void* a, const void* b,
+                                                 const float* sa, const float* sb, void* out, int M,
+                                                 int N, int K, cudaStream_t s, const DeviceInfo& d) {
+  constexpr int G = BSG_GRAN;
+  if (pl.swap_ab) {
+    // P = B, Q = A
+    switch (pl.bnq) {
+      case 16:  return launch<16, G, true, kBMn, kAMn, true>(pl, a, b, sa, sb, out, M, N, K, s, d);
+      case 32:  return launch<32, G, true, kBMn, kAMn, true>(pl, a, b, sa, sb, out, M, N, K, s, d);
+      case 64:  return launch<64, G, true, kBMn, kAMn, true>(pl, a, b, sa, sb, out, M, N, K, s, d);
+      case 128: return launch<128, G, true, kBMn, kAMn, true>(pl, a, b, sa, sb, out, M, N, K, s, d);
+      default:  return BSGEMM_ERR_INVALID_ARG;
+    }
+  }
+  const bool split = pl.splits > 1;
+  switch (pl.bnq) {
+    case 128:
+      return split ? launch<128, G, false, kAMn, kBMn, true>(pl, a, b, sa, sb, out, M, N, K, s, d)
+                   : launch<128, G, false, kAMn, kBMn, false>(pl, a, b, sa, sb, out, M, N, K, s, d);
+    case 256:
+      return split ? launch<256, G, false, kAMn, kBMn, true>(pl, a, b, sa, sb, out, M, N, K, s, d)
+                   : launch<256, G, false, kAMn, kBMn, false>(pl, a, b, sa, sb, out, M, N, K, s, d);
+    default:
+      return BSGEMM_ERR_INVALID_ARG;
+  }
+}
+
+}  // namespace bsg_host

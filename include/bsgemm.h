@@ -1,0 +1,176 @@
+/*
+ * bsgemm.h -- C ABI of the B200 (sm_100a) block-scaled FP8 GEMM library.
+ *
+ * Operation (hncyxsy.com/news/191052, "DeepGEMM实战: FP8矩阵乘法加速与Hopper
+ * 架构优化指南", §2.2 block-wise scaling, §3.2 segment-wise FP32 accumulation,
+ * §4.2 the gemm_fp8_fp8_bf16_nt call and its NT/TN/NN/TT flags):
+ *
+ *   out[m,n] = bf16( sum_kb  sA[m/g][kb] * sB[n/g][kb]
+ *                            * sum_{k in K-block kb} A[m,k] * B[n,k] )
+ *
+ * A and B hold FP8 E4M3 codes (OCP "e4m3fn": no infinities, 0x7F/0xFF NaN).
+ * Each operand carries one FP32 scale per g x g block (§2.2, §3.1 table:
+ * g = 128 by default, 64 and 256 as variants); the scale multiplies the code
+ * (§5.2: quantisation divides, dequantisation multiplies).  Each K-block's
+ * partial sum is taken on the tensor cores and promoted into an FP32
+ * accumulator with sA*sB applied (§3.2); the result is rounded to BF16
+ * (round to nearest even).
+ *
+ * Argument conventions shared by every entry point:
+ *   a, b      device pointers to E4M3 bytes, dense (no padding between rows):
+ *               _nt: A stored [M,K] row-major, B stored [N,K] row-major
+ *               _tn: A stored [K,M],           B stored [K,N]
+ *               _nn: A stored [M,K],           B stored [K,N]
+ *               _tt: A stored [K,M],           B stored [N,K]
+ *             (first letter A, second letter B; for A "N" means [M,K] and "T"
+ *             means [K,M]; for B "T" means [N,K] and "N" means [K,N]).  The
+ *             transposed forms are read through the TMA descriptors; no
+ *             transposed copy is made (§3.3).
+ *   scale_a   device pointer, FP32 [ceil(M/g)][ceil(K/g)] row-major
+ *   scale_b   device pointer, FP32 [ceil(N/g)][ceil(K/g)] row-major
+ *             Scales are indexed by logical block, whatever the layout.  A
+ *             partial last block (M, N or K not a multiple of g) has its own
+ *             scale and simply covers fewer rows/columns.
+ *   out       device pointer, BF16 [M,N] row-major, preallocated by the caller
+ *   M, N, K   logical sizes, each > 0
+ *   gran      g, one of 64, 128, 256 (the same for A, B and the K blocks)
+ *   stream    CUDA stream; the call is asynchronous with respect to the host
+ *
+ * Ownership: all pointers belong to the caller, who keeps them alive until
+ * the stream has passed the call.  The library keeps no pointer beyond the
+ * call.  It owns an internal split-K workspace per (device, stream), grown on
+ * demand with cudaMalloc and never shrunk; two calls that run concurrently on
+ * different streams never share it.
+ *
+ * Alignment (TMA rules), checked on the host before any launch:
+ *   a, b, out 16-byte aligned; scale_a, scale_b 4-byte aligned;
+ *   every row stride a multiple of 16 bytes: K % 16 == 0 for K-major
+ *   operands, M % 16 == 0 when A is stored [K,M], N % 16 == 0 when B is
+ *   stored [K,N]; N % 8 == 0 for out.
+ *
+ * Errors: argument and alignment problems and a device that is not sm_100
+ * are reported before anything is launched, and nothing is written to out.
+ * A failed launch returns BSGEMM_ERR_CUDA.  Waits inside the kernels are
+ * bounded: a wait that runs out records BSGEMM_ERR_DEVICE_TIMEOUT in a device
+ * status word (read with bsgemm_get_last_device_status) and the kernel
+ * returns without trapping, so the context stays usable.
+ *
+ * Results are deterministic: the same inputs give bit-identical outputs
+ * (split-K partials are added in a fixed order).
+ */
+#ifndef BSGEMM_H
+#define BSGEMM_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Opaque CUDA stream handle (cudaStream_t); 0 is the legacy default stream. */
+typedef void *bsgemm_stream_t;
+
+typedef enum {
+    BSGEMM_OK = 0,
+    BSGEMM_ERR_INVALID_ARG = 1,      /* null pointer, size <= 0, bad layout */
+    BSGEMM_ERR_UNSUPPORTED_GRAN = 2, /* gran not in {64, 128, 256} */
+    BSGEMM_ERR_MISALIGNED = 3,       /* a TMA alignment rule above is broken */
+    BSGEMM_ERR_UNSUPPORTED_DEVICE = 4, /* current device is not sm_100 */
+    BSGEMM_ERR_CUDA = 5,             /* a CUDA runtime/driver call failed */
+    BSGEMM_ERR_DEVICE_TIMEOUT = 6    /* a bounded device-side wait ran out */
+} bsgemm_status;
+
+/* NT: A [M,K], B [N,K] -- the native form (§3.3: fastest). */
+bsgemm_status bsgemm_fp8_nt(const void *a, const void *b, const float *scale_a,
+                            const float *scale_b, void *out, int64_t M, int64_t N, int64_t K,
+                            int gran, bsgemm_stream_t stream);
+
+/* TN: A stored [K,M], B stored [K,N]. */
+bsgemm_status bsgemm_fp8_tn(const void *a, const void *b, const float *scale_a,
+                            const float *scale_b, void *out, int64_t M, int64_t N, int64_t K,
+                            int gran, bsgemm_stream_t stream);
+
+/* NN: A stored [M,K], B stored [K,N]. */
+bsgemm_status bsgemm_fp8_nn(const void *a, const void *b, const float *scale_a,
+                            const float *scale_b, void *out, int64_t M, int64_t N, int64_t K,
+                            int gran, bsgemm_stream_t stream);
+
+/* TT: A stored [K,M], B stored [N,K]. */
+bsgemm_status bsgemm_fp8_tt(const void *a, const void *b, const float *scale_a,
+                            const float *scale_b, void *out, int64_t M, int64_t N, int64_t K,
+                            int gran, bsgemm_stream_t stream);
+
+/* ---- explicit-layout form, plan inspection and tuning ------------------ */
+
+typedef enum {
+    BSGEMM_LAYOUT_NT = 0, /* A [M,K], B [N,K] */
+    BSGEMM_LAYOUT_TN = 1, /* A [K,M], B [K,N] */
+    BSGEMM_LAYOUT_NN = 2, /* A [M,K], B [K,N] */
+    BSGEMM_LAYOUT_TT = 3  /* A [K,M], B [N,K] */
+} bsgemm_layout;
+
+typedef enum {
+    BSGEMM_VARIANT_AUTO = 0,          /* library heuristic */
+    BSGEMM_VARIANT_DATA_PARALLEL = 1, /* 128 rows of A per tile on the MMA M side */
+    BSGEMM_VARIANT_SWAP_AB = 2        /* 128 rows of B per tile on the MMA M side (small M) */
+} bsgemm_variant;
+
+/* Optional overrides of the plan; 0 in any field means "choose". */
+typedef struct {
+    int variant; /* bsgemm_variant */
+    int bnq;     /* tile width on the MMA N side: 128/256 (data-parallel), 16..128 (swap-AB) */
+    int splits;  /* K splits per output tile (split-K) */
+} bsgemm_tuning;
+
+/* What one call will launch (filled by bsgemm_make_plan). */
+typedef struct {
+    int layout, gran;
+    int swap_ab;        /* 1 if B feeds the MMA M side */
+    int bnq;            /* tile width on the MMA N side */
+    int tiles_p, tiles_q; /* tiles along the MMA M side (128 rows) and N side (bnq rows) */
+    int splits;         /* K splits per tile */
+    int kb_per_split;   /* K blocks per split */
+    int grid;           /* persistent CTAs launched (<= number of SMs) */
+    int group_p;        /* raster group height in tiles */
+    int kernels;        /* kernel launches per call */
+} bsgemm_plan;
+
+/* The operation above with the layout as an argument and optional tuning
+ * (NULL = heuristic). Same argument rules and errors as bsgemm_fp8_nt. */
+bsgemm_status bsgemm_fp8_gemm_ex(int layout, const void *a, const void *b, const float *scale_a,
+                                 const float *scale_b, void *out, int64_t M, int64_t N, int64_t K,
+                                 int gran, const bsgemm_tuning *tuning, bsgemm_stream_t stream);
+
+/* Host-only: the plan a call with these sizes would use on a device with
+ * `num_sms` SMs. Touches no device. */
+bsgemm_status bsgemm_make_plan(int layout, int64_t M, int64_t N, int64_t K, int gran, int num_sms,
+                               const bsgemm_tuning *tuning, bsgemm_plan *plan);
+
+/* Human-readable name of a status code (static string, never NULL). */
+const char *bsgemm_status_string(bsgemm_status status);
+
+/* Synchronises `stream`, then returns and clears the device status word of
+ * the current device: BSGEMM_OK, or BSGEMM_ERR_DEVICE_TIMEOUT if a bounded
+ * wait ran out in any kernel since the last call. BSGEMM_ERR_CUDA if the
+ * synchronisation itself failed. */
+bsgemm_status bsgemm_get_last_device_status(bsgemm_stream_t stream);
+
+/* Raw device status word (0, or the timeout code in the low byte and the
+ * place of the wait that gave up in bits 8..15), without clearing it. */
+int bsgemm_last_device_status_detail(void);
+
+/* Diagnostic: launches one CTA that waits on an mbarrier nothing completes,
+ * with a wait limit of `timeout_ns` (1 ns .. 10 s). The wait must give up,
+ * record BSGEMM_ERR_DEVICE_TIMEOUT and return; read it back with
+ * bsgemm_get_last_device_status. Exercises the bounded-wait path of the
+ * GEMM kernels without hanging or faulting the GPU. */
+bsgemm_status bsgemm_diag_wait_timeout(unsigned long long timeout_ns, bsgemm_stream_t stream);
+
+/* Library version as major*10000 + minor*100 + patch. */
+int bsgemm_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* BSGEMM_H */

@@ -1,0 +1,174 @@
+"""GPU parity: the CUDA path (through the C ABI) against the CPU oracle.
+
+Every case compares element by element with the tolerance in gpu_util.py;
+integer-exact cases must match bit for bit. Sizes are chosen so the oracle
+finishes in seconds yet the GPU path crosses several tiles and ragged tails.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import workloads
+import fp8_block_scaled_bsgemm_b200 as bsg
+
+from gpu_util import check_close, full_parity, gpu_as_f64, run_gpu, to_device
+
+pytestmark = pytest.mark.gpu
+
+
+def test_library_is_native_and_device_supported():
+    assert bsg.lib()._name.endswith("libbsgemm.so")
+    assert torch.cuda.get_device_capability() == (10, 0)
+
+
+# ---------------------------------------------------------------- the tiny config, all layouts
+@pytest.mark.parametrize("layout", ["nt", "tn", "nn", "tt"])
+def test_tiny_256_cubed(layout):
+    full_parity(workloads.tiny(layout=layout))
+
+
+# ---------------------------------------------------------------- ragged shapes, each granularity
+@pytest.mark.parametrize("gran", [64, 128, 256])
+@pytest.mark.parametrize("layout", ["nt", "tn", "nn", "tt"])
+def test_ragged_shapes(gran, layout):
+    # M, N multiples of 16 (MN-major layouts need them); neither a tile multiple
+    p = workloads.make_problem(400, 336, 1040, gran, layout, seed=gran)
+    full_parity(p, what=f"ragged {layout} g={gran}")
+
+
+@pytest.mark.parametrize("M,N,K", [(129, 8, 16), (257, 264, 48), (130, 520, 4112), (7, 1000, 656)])
+def test_odd_sizes_nt(M, N, K):
+    for g in (64, 128, 256):
+        full_parity(workloads.make_problem(M, N, K, g, "nt", seed=M + g), what=f"{M}x{N}x{K} g={g}")
+
+
+# ---------------------------------------------------------------- every kernel variant
+@pytest.mark.parametrize("variant,bnq", [("data_parallel", 128), ("data_parallel", 256),
+                                         ("swap_ab", 16), ("swap_ab", 32), ("swap_ab", 64),
+                                         ("swap_ab", 128)])
+@pytest.mark.parametrize("splits", [1, 3, 7])
+def test_forced_variants(variant, bnq, splits):
+    p = workloads.make_problem(200, 392, 2048, 128, "nt", seed=splits)
+    full_parity(p, tuning={"variant": variant, "bnq": bnq, "splits": splits},
+                what=f"{variant} bnq={bnq} splits={splits}")
+
+
+@pytest.mark.parametrize("gran", [64, 128, 256])
+@pytest.mark.parametrize("layout", ["nt", "tn", "nn", "tt"])
+def test_split_k_each_granularity_and_layout(gran, layout):
+    p = workloads.make_problem(160, 272, 3072, gran, layout, seed=3)
+    for v, bnq in (("data_parallel", 128), ("swap_ab", 64)):
+        full_parity(p, tuning={"variant": v, "bnq": bnq, "splits": 5}, what=f"{layout} g={gran} {v}")
+
+
+# ---------------------------------------------------------------- small M (decode-style)
+@pytest.mark.parametrize("M", [1, 8, 32, 64, 128])
+def test_small_m_reduced_k(M):
+    p = workloads.make_problem(M, 7168, 1024, 128, "nt", seed=M)
+    full_parity(p, what=f"small-M {M}")
+
+
+# ---------------------------------------------------------------- exactness and invariants
+def _integer_problem(M, N, K, gran, layout, seed):
+    """Values |v| <= 2 and power-of-two scales: every partial sum and every
+    scaled accumulation is exact in FP32, so GPU and oracle round the same
+    exact value to BF16."""
+    rng = np.random.default_rng(seed)
+    vals = np.array([0x00, 0x38, 0x40, 0xB8, 0xC0], np.uint8)   # 0, 1, 2, -1, -2
+    a = vals[rng.integers(0, vals.size, size=(M, K))]
+    b = vals[rng.integers(0, vals.size, size=(N, K))]
+    Kb = -(-K // gran)
+    sa = np.exp2(rng.integers(-4, -1, size=(-(-M // gran), Kb))).astype(np.float32)
+    sb = np.exp2(rng.integers(-4, -1, size=(-(-N // gran), Kb))).astype(np.float32)
+    p = workloads.Problem(M, N, K, gran, "nt", a, b, sa, sb, "integer-exact")
+    return workloads.relayout(p, layout)
+
+
+@pytest.mark.parametrize("layout", ["nt", "tn", "nn", "tt"])
+@pytest.mark.parametrize("tuning", [None, {"variant": "swap_ab", "bnq": 32, "splits": 2},
+                                    {"variant": "data_parallel", "bnq": 256, "splits": 3}])
+def test_integer_exact_bit_for_bit(layout, tuning):
+    p = _integer_problem(272, 304, 1024, 128, layout, seed=5)
+    ref, want = oracle.bsgemm(p.layout, p.a, p.b, p.sa, p.sb, p.M, p.N, p.K, p.gran)
+    # |ref| < 256 on a 2^-8 grid: 16 significant bits, exact in the FP32 accumulator
+    assert np.all(np.abs(ref) < 256) and np.all(ref == np.round(ref * 256) / 256)
+    out = run_gpu(p, tuning)
+    got = out.view(torch.int16).cpu().numpy().astype(np.uint16)
+    assert np.array_equal(got, want)
+
+
+def test_power_of_two_scale_is_exact_on_gpu():
+    p = workloads.make_problem(256, 512, 1024, 128, "nt", seed=7)
+    out1 = run_gpu(p)
+    p2 = workloads.Problem(p.M, p.N, p.K, p.gran, p.layout, p.a, p.b, p.sa * np.float32(4.0), p.sb)
+    out2 = run_gpu(p2)
+    assert torch.equal(out2.float(), out1.float() * 4.0)
+
+
+def test_single_block_scale_lands_on_its_block():
+    # one K-block of one row block scaled by 2^10: only rows of that block change
+    p = workloads.make_problem(384, 256, 768, 128, "nt", seed=8)
+    base = gpu_as_f64(run_gpu(p))
+    sa = p.sa.copy()
+    sa[1, 2] *= np.float32(1024.0)
+    p2 = workloads.Problem(p.M, p.N, p.K, p.gran, p.layout, p.a, p.b, sa, p.sb)
+    got = gpu_as_f64(run_gpu(p2))
+    assert np.array_equal(got[:128], base[:128]) and np.array_equal(got[256:], base[256:])
+    ref, _ = oracle.bsgemm("nt", p2.a, p2.b, p2.sa, p2.sb, p.M, p.N, p.K, p.gran)
+    check_close(got, ref, "scaled block")
+
+
+def test_layouts_agree_bit_for_bit():
+    p = workloads.make_problem(256, 384, 1536, 128, "nt", seed=10)
+    outs = [run_gpu(workloads.relayout(p, lay)) for lay in ("nt", "tn", "nn", "tt")]
+    for o in outs[1:]:
+        assert torch.equal(o, outs[0])
+
+
+@pytest.mark.parametrize("tuning", [None, {"variant": "swap_ab", "bnq": 16, "splits": 6}])
+def test_deterministic_repeats(tuning):
+    p = workloads.make_problem(64, 2048, 4096, 128, "nt", seed=11)
+    a, b, sa, sb = to_device(p)
+    first = bsg.gemm(a, b, sa, sb, gran=128, tuning=tuning)
+    for _ in range(20):
+        again = bsg.gemm(a, b, sa, sb, gran=128, tuning=tuning)
+        assert torch.equal(again, first)
+
+
+def test_poisoned_output_is_fully_written():
+    p = workloads.make_problem(136, 264, 512, 64, "nt", seed=12)
+    a, b, sa, sb = to_device(p)
+    out = torch.full((p.M, p.N), float("nan"), dtype=torch.bfloat16, device="cuda")
+    bsg.gemm(a, b, sa, sb, out=out, gran=64)
+    torch.cuda.synchronize()
+    assert not torch.isnan(out).any()
+
+
+# ---------------------------------------------------------------- errors and the bounded wait
+def test_host_side_errors_leave_output_untouched():
+    p = workloads.tiny()
+    a, b, sa, sb = to_device(p)
+    out = torch.full((256, 256), 7.0, dtype=torch.bfloat16, device="cuda")
+    A, B, SA, SB, O = a.data_ptr(), b.data_ptr(), sa.data_ptr(), sb.data_ptr(), out.data_ptr()
+    cases = [
+        ((A, B, SA, SB, O, 256, 256, 256, 96), 2),       # unsupported granularity
+        ((0, B, SA, SB, O, 256, 256, 256, 128), 1),      # null pointer
+        ((A, B, SA, SB, O, 0, 256, 256, 128), 1),        # empty M
+        ((A + 1, B, SA, SB, O, 256, 256, 256, 128), 3),  # misaligned base
+        ((A, B, SA, SB, O, 256, 256, 200, 128), 3),      # K % 16 != 0
+        ((A, B, SA, SB, O, 256, 250, 256, 128), 3),      # N % 8 != 0
+    ]
+    L = bsg.lib()
+    for args, want in cases:
+        assert L.bsgemm_fp8_nt(*args, None) == want, args
+    torch.cuda.synchronize()
+    assert torch.all(out == 7.0)
+
+
+def test_bounded_wait_times_out_and_context_survives():
+    assert bsg.get_last_device_status() == 0
+    assert bsg.diag_wait_timeout(2_000_000) == 0          # 2 ms limit
+    assert bsg.get_last_device_status() == 6              # BSGEMM_ERR_DEVICE_TIMEOUT
+    assert bsg.get_last_device_status() == 0              # cleared
+    full_parity(workloads.tiny(), what="after a timed-out wait")
