@@ -59,6 +59,10 @@ def parse_args(argv=None):
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="target CPU seconds of the oracle sample")
+    ap.add_argument("--variant", default="auto", choices=["auto", "data_parallel", "swap_ab"],
+                    help="override the plan's variant (default: library heuristic)")
+    ap.add_argument("--bnq", type=int, default=0, help="override the tile width on the MMA N side")
+    ap.add_argument("--splits", type=int, default=0, help="override the K splits per tile")
     return ap.parse_args(argv)
 
 
@@ -234,10 +238,13 @@ def run_ours(args):
     out = torch.empty((p.M, p.N), dtype=torch.bfloat16, device=dev)
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
     num_sms = torch.cuda.get_device_properties(dev).multi_processor_count
-    plan = bsg.make_plan(p.M, p.N, p.K, p.gran, p.layout, num_sms)
+    tuning = None
+    if args.variant != "auto" or args.bnq or args.splits:
+        tuning = {"variant": args.variant, "bnq": args.bnq, "splits": args.splits}
+    plan = bsg.make_plan(p.M, p.N, p.K, p.gran, p.layout, num_sms, tuning)
 
     def gemm():
-        bsg.gemm(a, b, sa, sb, out=out, layout=p.layout, gran=p.gran, stream=stream)
+        bsg.gemm(a, b, sa, sb, out=out, layout=p.layout, gran=p.gran, tuning=tuning, stream=stream)
 
     for _ in range(args.warmup):
         flush.zero_()
@@ -279,7 +286,7 @@ def run_ours(args):
             db.copy_(hb, non_blocking=True)
             dsa.copy_(hsa, non_blocking=True)
             dsb.copy_(hsb, non_blocking=True)
-            bsg.gemm(da, db, dsa, dsb, out=out, layout=p.layout, gran=p.gran, stream=stream)
+            bsg.gemm(da, db, dsa, dsb, out=out, layout=p.layout, gran=p.gran, tuning=tuning, stream=stream)
             hout.copy_(out, non_blocking=True)
 
         for _ in range(max(1, args.warmup)):

@@ -183,22 +183,34 @@ extern "C" bsgemm_status bsgemm_make_plan(int layout, int64_t M, int64_t N, int6
   pl.tiles_q = static_cast<int>((Q + bnq - 1) / bnq);
   const int64_t tiles = static_cast<int64_t>(pl.tiles_p) * pl.tiles_q;
   if (tiles > (1 << 30)) return BSGEMM_ERR_INVALID_ARG;
+  // split-K only when the tiles alone cannot fill the SMs; among the split
+  // counts, take the one with the least estimated time:
+  //   waves(tiles * splits) * (K-blocks per split + per-item overhead),
+  // the overhead standing for the FP32 partial tile written and re-read
+  auto split_fix = [&](int s, int& per) {
+    per = (Kb + s - 1) / s;
+    if (gran == 64 && (per & 1)) ++per;  // a split starts on a 128-element stage
+    return (Kb + per - 1) / per;
+  };
   int splits = t ? t->splits : 0;
   if (splits <= 0) {
-    // fill the SMs when there are too few tiles; keep >= 4 K-blocks per split
     splits = 1;
     if (tiles < num_sms) {
-      int s = static_cast<int>(num_sms / tiles);
-      int max_s = Kb / 4 > 1 ? Kb / 4 : 1;
-      splits = s < max_s ? s : max_s;
-      if (splits < 1) splits = 1;
+      const double overhead = 1.0 + bnq / 64.0;
+      double best = 1e30;
+      for (int s = 1; s <= Kb && s <= 64; ++s) {
+        int per = 0;
+        const int se = split_fix(s, per);
+        const int64_t waves = (tiles * se + num_sms - 1) / num_sms;
+        const double cost = static_cast<double>(waves) * (per + (se > 1 ? overhead : 0.0));
+        if (cost < best - 1e-9) { best = cost; splits = se; }
+      }
     }
   }
   if (splits > Kb) splits = Kb;
-  int per = (Kb + splits - 1) / splits;
-  if (gran == 64 && (per & 1)) ++per;  // a split starts on a 128-element stage
+  int per = 0;
+  pl.splits = split_fix(splits, per);
   pl.kb_per_split = per;
-  pl.splits = (Kb + per - 1) / per;
   const int64_t work = tiles * pl.splits;
   pl.grid = static_cast<int>(work < num_sms ? work : num_sms);
   pl.group_p = 16;

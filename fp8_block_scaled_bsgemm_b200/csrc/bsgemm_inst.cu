@@ -38,14 +38,12 @@ bsgemm_status launch(const bsgemm_plan& plan, const void* a, const void* b, cons
   const void* q_ptr = SWAP ? a : b;
   const int P = SWAP ? N : M;
   const int Q = SWAP ? M : N;
-  CUtensorMap tm_p, tm_q, tm_out;
+  CUtensorMap tm_p, tm_q;
   bool ok = true;
   if (P_MN) ok &= make_map_2d(&tm_p, p_ptr, CU_TENSOR_MAP_DATA_TYPE_UINT8, P, K, P, 128, bsg::BK);
   else      ok &= make_map_2d(&tm_p, p_ptr, CU_TENSOR_MAP_DATA_TYPE_UINT8, K, P, K, bsg::BK, bsg::BM);
   if (Q_MN) ok &= make_map_2d(&tm_q, q_ptr, CU_TENSOR_MAP_DATA_TYPE_UINT8, Q, K, Q, 128, bsg::BK);
   else      ok &= make_map_2d(&tm_q, q_ptr, CU_TENSOR_MAP_DATA_TYPE_UINT8, K, Q, K, bsg::BK, BNQ);
-  if (!SWAP) ok &= make_map_2d(&tm_out, out, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, N, M, (uint64_t)N * 2, 64, 32);
-  else       std::memset(&tm_out, 0, sizeof tm_out);
   if (!ok) return BSGEMM_ERR_CUDA;
 
   bsg::Params prm{};
@@ -87,7 +85,7 @@ bsgemm_status launch(const bsgemm_plan& plan, const void* a, const void* b, cons
     }
     attr_set = true;
   }
-  kern<<<plan.grid, bsg::kNumThreads, SC::kSmemBytes, stream>>>(tm_p, tm_q, tm_out, prm);
+  kern<<<plan.grid, bsg::kNumThreads, SC::kSmemBytes, stream>>>(tm_p, tm_q, prm);
   return cudaGetLastError() == cudaSuccess ? BSGEMM_OK : BSGEMM_ERR_CUDA;
 }
 

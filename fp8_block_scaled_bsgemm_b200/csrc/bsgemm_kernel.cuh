@@ -15,13 +15,13 @@
 //   warp 0   TMA producer: P and Q tiles of 128 K-bytes into a STAGES-deep
 //            ring of 128B-swizzled shared-memory buffers (mbarrier full/empty);
 //   warp 1   TMEM owner and MMA issuer: for each K-block, tcgen05.mma
-//            (kind::f8f6f4, K = 32 per instruction) into one of two TMEM
+//            (kind::f8f6f4, K = 32 per instruction) into one of 2..8 TMEM
 //            partial buffers, then tcgen05.commit to tell the promoters;
 //   warps 2-3 idle (they complete the first warpgroup);
 //   warps 4-11 promotion + epilogue: tcgen05.ld each K-block's partial,
 //            acc += (sP*sQ) * partial in FP32 registers (packed f32x2 FMAs),
 //            release the TMEM buffer, and at the end of a tile round to BF16
-//            and store it (TMA store, or direct stores in swap-AB mode).
+//            and store it straight from registers.
 // Split-K: a tile's K-blocks are divided among `splits` work items; each
 // writes an FP32 partial tile to a workspace, and the last to arrive (per-tile
 // counter) adds all partials in split order -- the same order every run -- and
@@ -57,8 +57,8 @@ constexpr int kTimeoutCode = 6;  // BSGEMM_ERR_DEVICE_TIMEOUT
 // setmaxnreg.inc can only be satisfied if the launch really had kLaunchRegs
 // per thread, so the host checks the compiled count before every launch.
 constexpr int kLaunchRegs = 168;
-constexpr int kProducerRegs = 72;
-constexpr int kPromoteRegs = 216;
+constexpr int kProducerRegs = 56;
+constexpr int kPromoteRegs = 224;
 static_assert(kProducerRegs * 128 + kPromoteRegs * 256 <= kLaunchRegs * kNumThreads,
               "register split exceeds the launch allocation");
 
@@ -97,7 +97,7 @@ struct Tiles {
 template <int BNQ, bool Q_MN, bool SWAP>
 struct StageCfg {
   static constexpr int kStageBytes = Tiles<BNQ, Q_MN>::kPBytes + Tiles<BNQ, Q_MN>::kQBytes;
-  static constexpr int kEpiBytes = SWAP ? 0 : kNumEpiWarps * 32 * 128;  // 4 KB per warp
+  static constexpr int kEpiBytes = 0;  // the epilogue stores straight from registers
   static constexpr int kBudget = 227 * 1024 - 1024 /*align slack*/ - 512 /*barriers*/;
   static constexpr int kStagesRaw = (kBudget - kEpiBytes) / kStageBytes;
   static constexpr int kStages = kStagesRaw > 8 ? 8 : kStagesRaw;
@@ -108,10 +108,9 @@ struct StageCfg {
 struct __align__(8) Barriers {
   uint64_t full[8];
   uint64_t empty[8];
-  uint64_t tmem_full[2];
-  uint64_t tmem_empty[2];
+  uint64_t tmem_full[8];
+  uint64_t tmem_empty[8];
   uint64_t mma_done;
-  uint64_t epi_sync;     // bounded rendezvous of the promotion warps (split-K)
   uint32_t tmem_base;
   int abort_flag;
   int split_last;
@@ -124,15 +123,20 @@ __device__ __forceinline__ void record_timeout(const Params& p, Barriers* bars, 
 }
 
 // Bounded mbarrier wait. Returns false on timeout or when another warp of the
-// CTA has raised the abort flag (unless ignore_abort).
+// CTA has raised the abort flag (unless ignore_abort).  Waiters that are not
+// on the critical path pass a backoff so that their polling does not crowd
+// the barrier unit that the critical hand-offs go through.
+template <int kBackoffNs = 0>
 __device__ __forceinline__ bool bounded_wait(uint32_t bar, uint32_t parity, const Params& p,
                                           Barriers* bars, int where, bool ignore_abort = false) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer_ns();
   while (true) {
 #pragma unroll 1
-    for (int i = 0; i < 32; ++i)
+    for (int i = 0; i < 32; ++i) {
       if (mbar_try_wait(bar, parity)) return true;
+      if constexpr (kBackoffNs > 0) __nanosleep(kBackoffNs);
+    }
     if (!ignore_abort && *reinterpret_cast<volatile int*>(&bars->abort_flag)) return false;
     if (globaltimer_ns() - t0 > p.timeout_ns) {
       if (!ignore_abort) record_timeout(p, bars, where);
@@ -141,27 +145,16 @@ __device__ __forceinline__ bool bounded_wait(uint32_t bar, uint32_t parity, cons
   }
 }
 
-// Warp-uniform bounded wait: lane 0 waits, every lane gets the same answer,
-// and the warp is converged afterwards (needed before .sync.aligned ops).
+// Warp-uniform bounded wait: lane 0 polls (one poller per warp keeps the
+// barrier traffic low), every lane gets the same answer, and the warp is
+// converged afterwards.
+template <int kBackoffNs = 0>
 __device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, const Params& p,
-                                          Barriers* bars, int where) {
+                                          Barriers* bars, int where, bool ignore_abort = false) {
   int ok = 0;
-  if (lane_id() == 0) ok = bounded_wait(bar, parity, p, bars, where) ? 1 : 0;
+  if (lane_id() == 0) ok = bounded_wait<kBackoffNs>(bar, parity, p, bars, where, ignore_abort) ? 1 : 0;
   ok = __shfl_sync(0xffffffffu, ok, 0);
-  __syncwarp();
   return ok != 0;
-}
-
-// Bounded rendezvous of the promotion warps (replaces an unbounded bar.sync,
-// which would hang if one warp had left on an abort). `uses` counts this
-// thread's previous rendezvous.
-__device__ __forceinline__ bool epi_rendezvous(uint32_t& uses, const Params& p, Barriers* bars) {
-  __syncwarp();
-  const uint32_t bar = smem_addr(&bars->epi_sync);
-  if (lane_id() == 0) mbar_arrive(bar);
-  const bool ok = warp_wait(bar, uses & 1, p, bars, 5);
-  ++uses;
-  return ok;
 }
 
 // Shared-memory matrix descriptor for tcgen05 (sm_100 format, version 1),
@@ -231,27 +224,30 @@ __device__ __forceinline__ void stage_range(const Params& p, const Work& w, int&
 template <int BNQ, int GRAN, bool SWAP, bool P_MN, bool Q_MN, bool SPLIT>
 __global__ void __launch_bounds__(kNumThreads, 1)
     bsgemm_kernel(const __grid_constant__ CUtensorMap tm_p, const __grid_constant__ CUtensorMap tm_q,
-                  const __grid_constant__ CUtensorMap tm_out, const Params p) {
+                  const Params p) {
   using TL = Tiles<BNQ, Q_MN>;
   using SC = StageCfg<BNQ, Q_MN, SWAP>;
   constexpr int STAGES = SC::kStages;
   constexpr int kHalf = BNQ / 2;                      // columns per promotion warp
   constexpr int kNumGroups = (kHalf > GRAN) ? kHalf / GRAN : 1;  // scale groups per warp
   constexpr int kGroupCols = kHalf / kNumGroups;
-  constexpr uint32_t kTmemCols = (2 * BNQ <= 32) ? 32 : (2 * BNQ <= 64) ? 64
-                                : (2 * BNQ <= 128) ? 128 : (2 * BNQ <= 256) ? 256 : 512;
+  // TMEM partial buffers: as many as fit (up to 8) so the MMA can run ahead of
+  // the promotion warps; 512 columns hold 2 x 256, 4 x 128 or 8 x 64.
+  constexpr int kBufs = (BNQ >= 256) ? 2 : (BNQ >= 128) ? 4 : 8;
+  constexpr uint32_t kTmemCols = (kBufs * BNQ <= 32) ? 32 : (kBufs * BNQ <= 64) ? 64
+                                : (kBufs * BNQ <= 128) ? 128 : (kBufs * BNQ <= 256) ? 256 : 512;
+  static_assert(kBufs * BNQ <= 512, "TMEM holds 512 columns");
   constexpr uint32_t kTxBytes = TL::kPBytes + TL::kQBytes;
   static_assert(BNQ % 16 == 0 && BNQ >= 16 && BNQ <= 256, "MMA N must be a multiple of 16 in [16, 256]");
   static_assert(GRAN == 64 || GRAN == 128 || GRAN == 256, "granularity");
   static_assert(kHalf % 8 == 0, "columns per warp");
-  static_assert(SWAP || kHalf % 64 == 0, "TMA-store epilogue writes 64-column boxes");
+  static_assert(SWAP || kHalf % 8 == 0, "the epilogue stores 8 BF16 columns at a time");
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* p_tiles = smem;
   uint8_t* q_tiles = smem + STAGES * TL::kPBytes;
-  uint8_t* epi_buf = q_tiles + STAGES * TL::kQBytes;
-  Barriers* bars = reinterpret_cast<Barriers*>(epi_buf + SC::kEpiBytes);
+  Barriers* bars = reinterpret_cast<Barriers*>(q_tiles + STAGES * TL::kQBytes);
 
   const int warp = threadIdx.x / 32;
   const uint32_t lane = lane_id();
@@ -262,12 +258,11 @@ __global__ void __launch_bounds__(kNumThreads, 1)
       mbar_init(smem_addr(&bars->full[s]), 1);
       mbar_init(smem_addr(&bars->empty[s]), 1);
     }
-    for (int b = 0; b < 2; ++b) {
+    for (int b = 0; b < kBufs; ++b) {
       mbar_init(smem_addr(&bars->tmem_full[b]), 1);
       mbar_init(smem_addr(&bars->tmem_empty[b]), kNumEpiWarps);
     }
     mbar_init(smem_addr(&bars->mma_done), 1);
-    mbar_init(smem_addr(&bars->epi_sync), kNumEpiWarps);
     bars->abort_flag = 0;
     bars->split_last = 0;
     fence_barrier_init();
@@ -275,7 +270,6 @@ __global__ void __launch_bounds__(kNumThreads, 1)
   if (warp == kProducerWarp && lane == 0) {
     tma_prefetch_desc(&tm_p);
     tma_prefetch_desc(&tm_q);
-    if (!SWAP) tma_prefetch_desc(&tm_out);
   }
   if (warp == kMmaWarp) {
     tmem_alloc(smem_addr(&bars->tmem_base), kTmemCols);
@@ -301,7 +295,7 @@ __global__ void __launch_bounds__(kNumThreads, 1)
         for (int st = st0; st < st1; ++st, ++it) {
           const int s = it % STAGES;
           const uint32_t ph = (it / STAGES) & 1;
-          if (!bounded_wait(smem_addr(&bars->empty[s]), ph ^ 1, p, bars, 1)) { ok = false; break; }
+          if (!bounded_wait<32>(smem_addr(&bars->empty[s]), ph ^ 1, p, bars, 1)) { ok = false; break; }
           const uint32_t fb = smem_addr(&bars->full[s]);
           mbar_arrive_expect_tx(fb, kTxBytes);
           const uint32_t pd = smem_addr(p_tiles + s * TL::kPBytes);
@@ -328,50 +322,72 @@ __global__ void __launch_bounds__(kNumThreads, 1)
     }
   } else if (warp == kMmaWarp) {
     // ============================================================ MMA issuer
+    // One thread issues: per K-block it claims a TMEM buffer, issues the
+    // block's MMAs (K = 32 each) stage by stage -- waiting for a stage at its
+    // first k-step, releasing it after its last -- and commits the buffer to
+    // the promotion warps as soon as the block's last MMA is issued (the
+    // promotion of block kb gates the MMAs of block kb + kBufs).  The issue
+    // path is straight-line code on one lane: per-MMA branching in a
+    // converged warp costs far more than the MMA issue itself.
     if (lane == 0) {
       constexpr uint32_t idesc = instr_desc<BNQ, P_MN, Q_MN>();
-      uint32_t it = 0;   // stage-slot uses so far
-      uint32_t pc = 0;   // K-blocks (TMEM partials) produced so far
+      // descriptor steps: per k-step of 32 (K-major +32 B, MN-major +32 rows
+      // of 128 B) and per pipeline stage, in the descriptor's 16-byte units
+      constexpr uint64_t kPStep = P_MN ? (kMmaK * 128) >> 4 : kMmaK >> 4;
+      constexpr uint64_t kQStep = Q_MN ? (kMmaK * 128) >> 4 : kMmaK >> 4;
+      constexpr uint64_t kPStage = TL::kPBytes >> 4, kQStage = TL::kQBytes >> 4;
+      const uint64_t ad0 = smem_desc_sw128(smem_addr(p_tiles), P_MN ? 128 * BK : 16);
+      const uint64_t bd0 = smem_desc_sw128(smem_addr(q_tiles), Q_MN ? 128 * BK : 16);
+      uint32_t s = 0, ph = 0;     // pipeline stage and its phase
+      uint32_t b = 0, bph = 0;    // TMEM buffer and its phase
       bool ok = true;
       for (int wi = blockIdx.x; wi < p.num_work && ok; wi += gridDim.x) {
         const Work w = decode_work(p, wi);
-        int st0, st1;
-        stage_range<GRAN>(p, w, st0, st1);
-        int cur_kb = -1;
-        uint32_t buf = 0, accum = 0;
-        for (int st = st0; st < st1 && ok; ++st, ++it) {
-          const int s = it % STAGES;
-          if (!bounded_wait(smem_addr(&bars->full[s]), (it / STAGES) & 1, p, bars, 2)) { ok = false; break; }
-          tc_fence_after();
-          const uint32_t pa = smem_addr(p_tiles + s * TL::kPBytes);
-          const uint32_t qa = smem_addr(q_tiles + s * TL::kQBytes);
+        for (int kb = w.kb0; kb < w.kb1; ++kb) {
+          // the promotion warps arrive only after tcgen05.wait::ld, so their
+          // reads of this buffer are complete before it is overwritten
+          if (!bounded_wait(smem_addr(&bars->tmem_empty[b]), bph ^ 1, p, bars, 3)) { ok = false; break; }
+          const uint32_t d_tmem = tmem_base + b * BNQ;
+          if constexpr (GRAN >= BK) {
+            // whole stages: GRAN / 128 of them, 4 k-steps each (fewer at the K tail)
 #pragma unroll
-          for (int kk = 0; kk < BK / kMmaK; ++kk) {
-            const int k = st * BK + kk * kMmaK;
-            const int kb = k / GRAN;
-            if (k >= p.K || kb >= w.kb1) break;
-            if (kb < w.kb0) continue;
-            if (kb != cur_kb) {
-              if (cur_kb >= 0) { mma_commit(smem_addr(&bars->tmem_full[buf])); ++pc; }
-              cur_kb = kb;
-              buf = pc & 1;
-              if (!bounded_wait(smem_addr(&bars->tmem_empty[buf]), ((pc >> 1) & 1) ^ 1, p, bars, 3)) {
-                ok = false;
-                break;
+            for (int j = 0; j < GRAN / BK; ++j) {
+              const int k0 = kb * GRAN + j * BK;
+              if (k0 >= p.K) break;
+              // TMA writes and MMA reads are async-proxy accesses ordered by this barrier
+              if (!bounded_wait(smem_addr(&bars->full[s]), ph, p, bars, 2)) { ok = false; break; }
+              const uint64_t ad = ad0 + s * kPStage, bd = bd0 + s * kQStage;
+              if (k0 + BK <= p.K) {
+#pragma unroll
+                for (int t = 0; t < BK / kMmaK; ++t)
+                  mma_f8f6f4(d_tmem, ad + t * kPStep, bd + t * kQStep, idesc, (j > 0 || t > 0) ? 1u : 0u);
+              } else {
+                const int nsteps = (p.K - k0 + kMmaK - 1) / kMmaK;
+                for (int t = 0; t < nsteps; ++t)
+                  mma_f8f6f4(d_tmem, ad + t * kPStep, bd + t * kQStep, idesc, (j > 0 || t > 0) ? 1u : 0u);
               }
-              tc_fence_after();
-              accum = 0;
+              mma_commit(smem_addr(&bars->empty[s]));  // stage free once these MMAs finish
+              if (++s == STAGES) { s = 0; ph ^= 1; }
             }
-            const uint64_t ad = P_MN ? smem_desc_sw128(pa + kk * kMmaK * 128, 128 * BK)
-                                     : smem_desc_sw128(pa + kk * kMmaK, 16);
-            const uint64_t bd = Q_MN ? smem_desc_sw128(qa + kk * kMmaK * 128, 128 * BK)
-                                     : smem_desc_sw128(qa + kk * kMmaK, 16);
-            mma_f8f6f4(tmem_base + buf * BNQ, ad, bd, idesc, accum);
-            accum = 1;
+            if (!ok) break;
+          } else {
+            // GRAN == 64: a K-block is half a stage; even blocks open the
+            // stage, odd blocks (or the K tail) release it
+            const int k0 = kb * GRAN;
+            const int t0 = (kb & 1) * 2;
+            if (t0 == 0 && !bounded_wait(smem_addr(&bars->full[s]), ph, p, bars, 2)) { ok = false; break; }
+            const uint64_t ad = ad0 + s * kPStage, bd = bd0 + s * kQStage;
+            const int nsteps = (p.K - k0 >= GRAN) ? 2 : (p.K - k0 + kMmaK - 1) / kMmaK;
+            for (int t = 0; t < nsteps; ++t)
+              mma_f8f6f4(d_tmem, ad + (t0 + t) * kPStep, bd + (t0 + t) * kQStep, idesc, t > 0 ? 1u : 0u);
+            if (t0 == 2 || k0 + GRAN >= p.K) {
+              mma_commit(smem_addr(&bars->empty[s]));
+              if (++s == STAGES) { s = 0; ph ^= 1; }
+            }
           }
-          mma_commit(smem_addr(&bars->empty[s]));  // stage free once these MMAs finish
+          mma_commit(smem_addr(&bars->tmem_full[b]));
+          if (++b == kBufs) { b = 0; bph ^= 1; }
         }
-        if (ok && cur_kb >= 0) { mma_commit(smem_addr(&bars->tmem_full[buf])); ++pc; }
       }
       // all MMAs issued by this thread complete before TMEM is freed
       mma_commit(smem_addr(&bars->mma_done));
@@ -387,7 +403,6 @@ __global__ void __launch_bounds__(kNumThreads, 1)
     const int row_in_tile = quad * 32 + static_cast<int>(lane);
     const uint32_t t_lane = static_cast<uint32_t>(quad * 32) << 16;
     uint32_t pc = 0;          // K-blocks consumed so far (TMEM buffer / phase)
-    uint32_t sync_uses = 0;   // epilogue rendezvous so far
     bool ok = true;
     float2 acc[kHalf / 2];    // this thread's row, columns [half*kHalf, (half+1)*kHalf)
 
@@ -434,39 +449,52 @@ __global__ void __launch_bounds__(kNumThreads, 1)
           s2[j] = make_float2(sv, sv);
         }
 
-        const uint32_t buf = pc & 1;
-        if (!warp_wait(smem_addr(&bars->tmem_full[buf]), (pc >> 1) & 1, p, bars, 4)) { ok = false; break; }
-        tc_fence_after();
+        const uint32_t buf = pc % kBufs;
+        // tcgen05.commit arrives only once the MMAs' TMEM writes are complete
+        if (!warp_wait(smem_addr(&bars->tmem_full[buf]), (pc / kBufs) & 1, p, bars, 4)) { ok = false; break; }
         const uint32_t taddr = tmem_base + t_lane + buf * BNQ + half * kHalf;
         {
-          // TMEM -> registers in chunks of CW columns, two chunks in flight;
-          // 128 accumulator columns per thread leave room for 2 x 8 only
-          constexpr int CW = (kHalf >= 128 || kHalf % 16 != 0) ? 8 : 16;
+          // TMEM -> registers in chunks of 32 columns; with up to 64
+          // accumulator columns per thread the next chunk's load is in flight
+          // while the current one is scaled (two chunks of staging), with 128
+          // there is room for one chunk only
+          constexpr int CW = kHalf < 32 ? kHalf : 32;
           constexpr int NC = kHalf / CW;
+          constexpr bool kDouble = kHalf <= 64;
           uint32_t ra[CW], rb[CW];
           auto fma_chunk = [&](const uint32_t (&r)[CW], int c) {
-            const float2 sv = s2[(c * CW) / kGroupCols];
 #pragma unroll
-            for (int i = 0; i < CW / 2; ++i)
+            for (int i = 0; i < CW / 2; ++i) {
+              const float2 sv = s2[(c * CW + 2 * i) / kGroupCols];
               acc[c * (CW / 2) + i] =
                   ffma2(make_float2(__uint_as_float(r[2 * i]), __uint_as_float(r[2 * i + 1])), sv,
                         acc[c * (CW / 2) + i]);
+            }
           };
-          tmem_ld(taddr, ra);
-          tmem_wait_ld(ra);
+          if constexpr (kDouble) {
+            tmem_ld(taddr, ra);
+            tmem_wait_ld(ra);
 #pragma unroll
-          for (int c = 0; c < NC; c += 2) {
-            if (c + 1 < NC) tmem_ld(taddr + (c + 1) * CW, rb);
-            fma_chunk(ra, c);
-            if (c + 1 < NC) {
-              tmem_wait_ld(rb);
-              if (c + 2 < NC) tmem_ld(taddr + (c + 2) * CW, ra);
-              fma_chunk(rb, c + 1);
-              if (c + 2 < NC) tmem_wait_ld(ra);
+            for (int c = 0; c < NC; c += 2) {
+              if (c + 1 < NC) tmem_ld(taddr + (c + 1) * CW, rb);
+              fma_chunk(ra, c);
+              if (c + 1 < NC) {
+                tmem_wait_ld(rb);
+                if (c + 2 < NC) tmem_ld(taddr + (c + 2) * CW, ra);
+                fma_chunk(rb, c + 1);
+                if (c + 2 < NC) tmem_wait_ld(ra);
+              }
+            }
+          } else {
+            (void)rb;
+#pragma unroll
+            for (int c = 0; c < NC; ++c) {
+              tmem_ld(taddr + c * CW, ra);
+              tmem_wait_ld(ra);
+              fma_chunk(ra, c);
             }
           }
         }
-        tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(smem_addr(&bars->tmem_empty[buf]));
       }
@@ -484,15 +512,15 @@ __global__ void __launch_bounds__(kNumThreads, 1)
           }
           __threadfence();
           // the partial now lives in the workspace; acc is dead until the sum below
-          if (!epi_rendezvous(sync_uses, p, bars)) { ok = false; break; }
+          named_barrier_sync(1, kNumEpiThreads);
           if (ew == 0 && lane == 0) {
             const int old = atomicAdd(p.counters + w.tile, 1);
             bars->split_last = (old == p.splits - 1) ? 1 : 0;
           }
-          if (!epi_rendezvous(sync_uses, p, bars)) { ok = false; break; }
+          named_barrier_sync(1, kNumEpiThreads);
           const bool last = *reinterpret_cast<volatile int*>(&bars->split_last) != 0;
-          // nobody may overwrite split_last before every warp has read it
-          if (!epi_rendezvous(sync_uses, p, bars)) { ok = false; break; }
+          // nobody may overwrite split_last before every thread has read it
+          named_barrier_sync(1, kNumEpiThreads);
           if (!last) continue;
           __threadfence();
           // fixed order: split 0, 1, ..., whoever arrived last
@@ -528,35 +556,26 @@ __global__ void __launch_bounds__(kNumThreads, 1)
           }
         }
       } else {
-        uint8_t* stage_buf = epi_buf + ew * (32 * 128);
-        const uint32_t sbase = smem_addr(stage_buf);
+        // this thread owns row m, columns [n0, n0 + kHalf): 16-byte stores of
+        // 8 BF16 values (N % 8 == 0, so a group is either all in or all out)
+        const int m = w.tp * BM + row_in_tile;
+        const int n0 = w.tq * BNQ + half * kHalf;
+        if (m < p.M) {
+          __nv_bfloat16* row = p.out + static_cast<size_t>(m) * p.N + n0;
 #pragma unroll
-        for (int box = 0; box < kHalf / 64; ++box) {
-          if (lane == 0) bulk_wait_group_read0();  // previous store done reading the buffer
-          __syncwarp();
-#pragma unroll
-          for (int c = 0; c < 8; ++c) {
-            const int i0 = box * 32 + c * 4;  // float2 index of column box*64 + c*8
-            const uint32_t x = pack_bf16x2(acc[i0].x, acc[i0].y);
-            const uint32_t y = pack_bf16x2(acc[i0 + 1].x, acc[i0 + 1].y);
-            const uint32_t z = pack_bf16x2(acc[i0 + 2].x, acc[i0 + 2].y);
-            const uint32_t q = pack_bf16x2(acc[i0 + 3].x, acc[i0 + 3].y);
-            // 128B swizzle: 16-byte chunk c of row `lane` lives at chunk c ^ (lane % 8)
-            const uint32_t off = lane * 128 + ((c ^ (lane & 7)) * 16);
-            asm volatile("st.shared.v4.b32 [%0], {%1,%2,%3,%4};" ::"r"(sbase + off), "r"(x), "r"(y),
-                         "r"(z), "r"(q)
-                         : "memory");
-          }
-          fence_proxy_async_smem();
-          __syncwarp();
-          if (lane == 0) {
-            tma_store_2d(&tm_out, sbase, w.tq * BNQ + half * kHalf + box * 64, w.tp * BM + quad * 32);
-            bulk_commit_group();
+          for (int c = 0; c < kHalf / 8; ++c) {
+            if (n0 + c * 8 < p.N) {
+              uint4 v;
+              v.x = pack_bf16x2(acc[c * 4].x, acc[c * 4].y);
+              v.y = pack_bf16x2(acc[c * 4 + 1].x, acc[c * 4 + 1].y);
+              v.z = pack_bf16x2(acc[c * 4 + 2].x, acc[c * 4 + 2].y);
+              v.w = pack_bf16x2(acc[c * 4 + 3].x, acc[c * 4 + 3].y);
+              *reinterpret_cast<uint4*>(row + c * 8) = v;
+            }
           }
         }
       }
     }
-    if (!SWAP && lane == 0) bulk_wait_group0();
   }
   __syncwarp();
 
