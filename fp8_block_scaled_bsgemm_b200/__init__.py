@@ -24,7 +24,8 @@ LIB_PATH = os.path.join(_HERE, "libbsgemm.so")
 LAYOUTS = {"nt": 0, "tn": 1, "nn": 2, "tt": 3}
 VARIANTS = {"auto": 0, "data_parallel": 1, "swap_ab": 2}
 STATUS = {0: "ok", 1: "invalid argument", 2: "unsupported granularity", 3: "misaligned",
-          4: "unsupported device", 5: "CUDA error", 6: "device wait timeout"}
+          4: "unsupported device", 5: "CUDA error", 6: "device wait timeout",
+          7: "needs more scratch than the allocation-free entry point holds"}
 
 _lock = threading.Lock()
 _lib = None
@@ -50,7 +51,8 @@ class Plan(ctypes.Structure):
 
 EXPORTS = ("bsgemm_fp8_nt", "bsgemm_fp8_tn", "bsgemm_fp8_nn", "bsgemm_fp8_tt", "bsgemm_fp8_gemm_ex",
            "bsgemm_make_plan", "bsgemm_status_string", "bsgemm_get_last_device_status",
-           "bsgemm_last_device_status_detail", "bsgemm_diag_wait_timeout", "bsgemm_version")
+           "bsgemm_last_device_status_detail", "bsgemm_diag_wait_timeout", "bsgemm_version",
+           "bsgemm_fp8_nt_noalloc")
 
 
 def lib():
@@ -64,7 +66,8 @@ def lib():
             L = ctypes.CDLL(LIB_PATH)
             p, i64, i32 = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int
             gemm_args = [p, p, p, p, p, i64, i64, i64, i32, p]
-            for name in ("bsgemm_fp8_nt", "bsgemm_fp8_tn", "bsgemm_fp8_nn", "bsgemm_fp8_tt"):
+            for name in ("bsgemm_fp8_nt", "bsgemm_fp8_tn", "bsgemm_fp8_nn", "bsgemm_fp8_tt",
+                         "bsgemm_fp8_nt_noalloc"):
                 getattr(L, name).argtypes = gemm_args
                 getattr(L, name).restype = i32
             L.bsgemm_fp8_gemm_ex.argtypes = [i32, p, p, p, p, p, i64, i64, i64, i32,

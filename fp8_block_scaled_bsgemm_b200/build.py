@@ -60,7 +60,8 @@ def _compile(src: str, obj: str, defines: list[str]) -> str:
 def build(force: bool = False, jobs: int | None = None, verbose: bool = False) -> str:
     os.makedirs(BUILD, exist_ok=True)
     newest = _newest_source()
-    units = [(os.path.join(CSRC, "bsgemm_api.cu"), os.path.join(BUILD, "bsgemm_api.o"), [])]
+    units = [(os.path.join(CSRC, "bsgemm_api.cu"), os.path.join(BUILD, "bsgemm_api.o"), []),
+             (os.path.join(CSRC, "bsgemm_noalloc.cu"), os.path.join(BUILD, "bsgemm_noalloc.o"), [])]
     for g in GRANS:
         for lay in LAYOUTS:
             units.append((os.path.join(CSRC, "bsgemm_inst.cu"),

@@ -125,6 +125,13 @@ unsigned long long wait_timeout_ns() {
   return t;
 }
 
+bsgemm_status device_status_address(int** out) {
+  void* p = nullptr;
+  if (cudaGetSymbolAddress(&p, g_device_status) != cudaSuccess || p == nullptr) return BSGEMM_ERR_CUDA;
+  *out = static_cast<int*>(p);
+  return BSGEMM_OK;
+}
+
 }  // namespace bsg_host
 
 namespace {
@@ -286,6 +293,7 @@ extern "C" const char* bsgemm_status_string(bsgemm_status s) {
     case BSGEMM_ERR_UNSUPPORTED_DEVICE: return "current device is not sm_100 (B200)";
     case BSGEMM_ERR_CUDA: return "CUDA runtime or driver call failed";
     case BSGEMM_ERR_DEVICE_TIMEOUT: return "a bounded device-side wait timed out";
+    case BSGEMM_ERR_SCRATCH_LIMIT: return "problem needs more split-K scratch than the allocation-free entry point holds";
   }
   return "unknown status";
 }

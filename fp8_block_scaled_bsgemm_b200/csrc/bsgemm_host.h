@@ -35,6 +35,10 @@ bsgemm_status get_workspace(cudaStream_t stream, size_t ws_bytes, size_t n_count
 // Limit of every bounded device-side wait, in nanoseconds.
 unsigned long long wait_timeout_ns();
 
+// Device address of the current device's status word (looked up on every
+// call; allocates nothing).
+bsgemm_status device_status_address(int** out);
+
 #define BSG_RUN_DECL(G, L)                                                                       \
   bsgemm_status run_g##G##_##L(const bsgemm_plan& plan, const void* a, const void* b,          \
                                const float* sa, const float* sb, void* out, int M, int N, int K, \

@@ -1,0 +1,193 @@
+// bsgemm_fp8_nt_noalloc: the NT block-scaled FP8 GEMM for callers that cannot
+// allocate device memory.
+//
+// Who needs it: code that runs where cudaMalloc is unavailable or forbidden --
+// inside a host allocator callback, under a framework that owns all device
+// memory and hands out nothing but the tensors it passes in, or in a process
+// that must not grow its device footprint after start-up.  The regular entry
+// points create a split-K workspace on first use with cudaMalloc; this one
+// never does.
+//
+// Instead, the split-K scratch (FP32 partial tiles plus one counter per output
+// tile) is a fixed array in the library's own device memory, declared below.
+// Every GPU that loads the library holds one copy of it until the process
+// exits.  Its size bounds what this entry point accepts: a problem whose plan
+// needs more scratch than the array holds is rejected with
+// BSGEMM_ERR_SCRATCH_LIMIT before anything is launched.
+//
+// All calls share the array, and it keeps whatever the last call left in it.
+// The tile counters must start at zero, so each call clears them
+// (cudaMemsetAsync on the caller's stream, which allocates nothing) before its
+// kernel.  Two calls whose kernels overlap on the GPU -- different streams, or
+// different host threads on one device -- race on the array and corrupt each
+// other's results; callers must serialise them.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <atomic>
+#include <cstdint>
+#include <cstring>
+
+#include "bsgemm.h"
+#include "bsgemm_host.h"
+#include "bsgemm_kernel.cuh"
+
+namespace {
+
+constexpr size_t kPartialBytes = BSGEMM_NOALLOC_SCRATCH_BYTES;
+constexpr int kMaxTiles = BSGEMM_NOALLOC_MAX_TILES;
+
+// The scratch: FP32 partial tiles first, then the tile counters.
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kPartialBytes + kMaxTiles * sizeof(int)];
+
+// Per-device set-up, done once by the first call on each device: the device
+// address of the array (in host code its name is only a host-side stand-in).
+// A fixed table, so the set-up itself allocates nothing either.
+constexpr int kMaxDevices = 64;
+struct DeviceScratch {
+  std::atomic<int> state{0};  // 0 not set up, 1 being set up, 2 ready
+  unsigned char* base = nullptr;
+  int num_sms = 0;
+  int* status = nullptr;
+};
+DeviceScratch g_scratch[kMaxDevices];
+
+bsgemm_status setup_current_device(DeviceScratch*& out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return BSGEMM_ERR_CUDA;
+  if (dev < 0 || dev >= kMaxDevices) return BSGEMM_ERR_UNSUPPORTED_DEVICE;
+  DeviceScratch& d = g_scratch[dev];
+  int st = d.state.load(std::memory_order_acquire);
+  while (st != 2) {
+    int expect = 0;
+    if (st == 0 && d.state.compare_exchange_strong(expect, 1)) {
+      int major = 0, minor = 0, sms = 0;
+      void* p = nullptr;
+      int* status = nullptr;
+      bool ok = cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) == cudaSuccess &&
+                cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) == cudaSuccess &&
+                cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess;
+      if (ok && !(major == 10 && minor == 0)) {
+        d.state.store(0, std::memory_order_release);
+        return BSGEMM_ERR_UNSUPPORTED_DEVICE;
+      }
+      ok = ok && cudaGetSymbolAddress(&p, g_noalloc_scratch) == cudaSuccess && p != nullptr;
+      ok = ok && bsg_host::device_status_address(&status) == BSGEMM_OK;
+      if (!ok) {
+        d.state.store(0, std::memory_order_release);
+        return BSGEMM_ERR_CUDA;
+      }
+      d.base = static_cast<unsigned char*>(p);
+      d.num_sms = sms;
+      d.status = status;
+      d.state.store(2, std::memory_order_release);
+    }
+    st = d.state.load(std::memory_order_acquire);
+  }
+  out = &d;
+  return BSGEMM_OK;
+}
+
+// Same kernel as the regular NT split-K path, launched on the fixed scratch.
+template <int BNQ, int GRAN, bool SWAP>
+bsgemm_status launch_fixed(const bsgemm_plan& plan, const void* a, const void* b, const float* sa,
+                           const float* sb, void* out, int M, int N, int K, cudaStream_t stream,
+                           const DeviceScratch& d) {
+  using SC = bsg::StageCfg<BNQ, false, SWAP>;
+  auto kern = bsg::bsgemm_kernel<BNQ, GRAN, SWAP, false, false, true>;
+  const void* p_ptr = SWAP ? b : a;
+  const void* q_ptr = SWAP ? a : b;
+  const int P = SWAP ? N : M;
+  const int Q = SWAP ? M : N;
+  CUtensorMap tm_p, tm_q;
+  if (!bsg_host::make_map_2d(&tm_p, p_ptr, CU_TENSOR_MAP_DATA_TYPE_UINT8, K, P, K, bsg::BK, bsg::BM) ||
+      !bsg_host::make_map_2d(&tm_q, q_ptr, CU_TENSOR_MAP_DATA_TYPE_UINT8, K, Q, K, bsg::BK, BNQ))
+    return BSGEMM_ERR_CUDA;
+
+  bsg::Params prm{};
+  prm.M = M; prm.N = N; prm.K = K;
+  prm.P = P; prm.Q = Q;
+  prm.Kb = (K + GRAN - 1) / GRAN;
+  prm.Pb = (P + GRAN - 1) / GRAN;
+  prm.Qb = (Q + GRAN - 1) / GRAN;
+  prm.tiles_p = plan.tiles_p;
+  prm.tiles_q = plan.tiles_q;
+  prm.num_tiles = plan.tiles_p * plan.tiles_q;
+  prm.splits = plan.splits;
+  prm.kb_per_split = plan.kb_per_split;
+  prm.num_work = prm.num_tiles * plan.splits;
+  prm.group_p = plan.group_p;
+  prm.sP = SWAP ? sb : sa;
+  prm.sQ = SWAP ? sa : sb;
+  prm.out = static_cast<__nv_bfloat16*>(out);
+  prm.status = d.status;
+  prm.timeout_ns = bsg_host::wait_timeout_ns();
+  if (plan.splits > 1) {
+    const size_t need = (size_t)prm.num_work * BNQ * bsg::BM * sizeof(float);
+    if (need > kPartialBytes || prm.num_tiles > kMaxTiles) return BSGEMM_ERR_SCRATCH_LIMIT;
+    prm.ws = reinterpret_cast<float*>(d.base);
+    prm.counters = reinterpret_cast<int*>(d.base + kPartialBytes);
+    // the counters must start at zero; the array keeps the previous call's contents
+    if (cudaMemsetAsync(prm.counters, 0, (size_t)prm.num_tiles * sizeof(int), stream) != cudaSuccess)
+      return BSGEMM_ERR_CUDA;
+  }
+  if (bsg::RegSplit<BNQ>::kEnabled) {
+    cudaFuncAttributes fa{};
+    if (cudaFuncGetAttributes(&fa, kern) != cudaSuccess || fa.numRegs != bsg::kLaunchRegs)
+      return BSGEMM_ERR_CUDA;
+  }
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SC::kSmemBytes) != cudaSuccess)
+    return BSGEMM_ERR_CUDA;
+  kern<<<plan.grid, bsg::kNumThreads, SC::kSmemBytes, stream>>>(tm_p, tm_q, prm);
+  return cudaGetLastError() == cudaSuccess ? BSGEMM_OK : BSGEMM_ERR_CUDA;
+}
+
+template <int GRAN>
+bsgemm_status dispatch_fixed(const bsgemm_plan& pl, const void* a, const void* b, const float* sa,
+                             const float* sb, void* out, int M, int N, int K, cudaStream_t s,
+                             const DeviceScratch& d) {
+  if (pl.swap_ab) {
+    switch (pl.bnq) {
+      case 16:  return launch_fixed<16, GRAN, true>(pl, a, b, sa, sb, out, M, N, K, s, d);
+      case 32:  return launch_fixed<32, GRAN, true>(pl, a, b, sa, sb, out, M, N, K, s, d);
+      case 64:  return launch_fixed<64, GRAN, true>(pl, a, b, sa, sb, out, M, N, K, s, d);
+      case 128: return launch_fixed<128, GRAN, true>(pl, a, b, sa, sb, out, M, N, K, s, d);
+      default:  return BSGEMM_ERR_INVALID_ARG;
+    }
+  }
+  switch (pl.bnq) {
+    case 128: return launch_fixed<128, GRAN, false>(pl, a, b, sa, sb, out, M, N, K, s, d);
+    case 256: return launch_fixed<256, GRAN, false>(pl, a, b, sa, sb, out, M, N, K, s, d);
+    default:  return BSGEMM_ERR_INVALID_ARG;
+  }
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+bool aligned4(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 3u) == 0; }
+
+}  // namespace
+
+extern "C" bsgemm_status bsgemm_fp8_nt_noalloc(const void* a, const void* b, const float* scale_a,
+                                               const float* scale_b, void* out, int64_t M, int64_t N,
+                                               int64_t K, int gran, bsgemm_stream_t stream) {
+  if (!a || !b || !scale_a || !scale_b || !out) return BSGEMM_ERR_INVALID_ARG;
+  if (M <= 0 || N <= 0 || K <= 0 || M > (1 << 30) || N > (1 << 30) || K > (1 << 30))
+    return BSGEMM_ERR_INVALID_ARG;
+  if (gran != 64 && gran != 128 && gran != 256) return BSGEMM_ERR_UNSUPPORTED_GRAN;
+  if (!aligned16(a) || !aligned16(b) || !aligned16(out) || !aligned4(scale_a) || !aligned4(scale_b))
+    return BSGEMM_ERR_MISALIGNED;
+  if (K % 16 || N % 8) return BSGEMM_ERR_MISALIGNED;
+  DeviceScratch* d = nullptr;
+  bsgemm_status st = setup_current_device(d);
+  if (st != BSGEMM_OK) return st;
+  bsgemm_plan pl;
+  st = bsgemm_make_plan(BSGEMM_LAYOUT_NT, M, N, K, gran, d->num_sms, nullptr, &pl);
+  if (st != BSGEMM_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const int m = static_cast<int>(M), n = static_cast<int>(N), k = static_cast<int>(K);
+  switch (gran) {
+    case 64:  return dispatch_fixed<64>(pl, a, b, scale_a, scale_b, out, m, n, k, s, *d);
+    case 128: return dispatch_fixed<128>(pl, a, b, scale_a, scale_b, out, m, n, k, s, *d);
+    default:  return dispatch_fixed<256>(pl, a, b, scale_a, scale_b, out, m, n, k, s, *d);
+  }
+}

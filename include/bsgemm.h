@@ -77,7 +77,9 @@ typedef enum {
     BSGEMM_ERR_MISALIGNED = 3,       /* a TMA alignment rule above is broken */
     BSGEMM_ERR_UNSUPPORTED_DEVICE = 4, /* current device is not sm_100 */
     BSGEMM_ERR_CUDA = 5,             /* a CUDA runtime/driver call failed */
-    BSGEMM_ERR_DEVICE_TIMEOUT = 6    /* a bounded device-side wait ran out */
+    BSGEMM_ERR_DEVICE_TIMEOUT = 6,   /* a bounded device-side wait ran out */
+    BSGEMM_ERR_SCRATCH_LIMIT = 7     /* bsgemm_fp8_nt_noalloc: the problem needs more
+                                        scratch than its fixed array holds */
 } bsgemm_status;
 
 /* NT: A [M,K], B [N,K] -- the native form (§3.3: fastest). */
@@ -165,6 +167,39 @@ int bsgemm_last_device_status_detail(void);
  * bsgemm_get_last_device_status. Exercises the bounded-wait path of the
  * GEMM kernels without hanging or faulting the GPU. */
 bsgemm_status bsgemm_diag_wait_timeout(unsigned long long timeout_ns, bsgemm_stream_t stream);
+
+/* ---- allocation-free variant --------------------------------------------
+ * The pages have no counterpart to this entry point; it serves callers that
+ * cannot allocate device memory: code running inside an allocator callback,
+ * under a framework that owns every byte of device memory and hands the
+ * library only the tensors of the call, or in a process that must not grow
+ * its device footprint after start-up.  The entry points above create their
+ * split-K workspace with cudaMalloc on first use; this one never allocates
+ * (no cudaMalloc, cudaFree or allocating library call, torch's included).
+ *
+ * It computes exactly what bsgemm_fp8_nt computes, with the same arguments,
+ * rules and errors, and with the same kernels and plan.  Its split-K scratch
+ * is a fixed array inside the library's device memory: each GPU that loads
+ * the library holds BSGEMM_NOALLOC_SCRATCH_BYTES of FP32 partial tiles plus
+ * BSGEMM_NOALLOC_MAX_TILES tile counters until the process exits.  A problem
+ * whose plan needs more -- (tiles x splits) x tile width x 128 x 4 bytes of
+ * partials, or more tiles than counters -- is rejected with
+ * BSGEMM_ERR_SCRATCH_LIMIT before anything is launched.  Problems whose plan
+ * does not split K use no scratch at all.
+ *
+ * The first call on each device looks up the array's device address (once,
+ * with that device current); make that first call before any stream capture.
+ * Every call shares the array, which keeps the previous call's contents:
+ * each call clears the tile counters on its stream before its kernel.  Calls
+ * whose kernels overlap on the GPU (other streams, other host threads on the
+ * same device) race on the array and corrupt each other's results, so the
+ * caller must serialise them. */
+#define BSGEMM_NOALLOC_SCRATCH_BYTES (16u << 20)
+#define BSGEMM_NOALLOC_MAX_TILES 4096
+
+bsgemm_status bsgemm_fp8_nt_noalloc(const void *a, const void *b, const float *scale_a,
+                                    const float *scale_b, void *out, int64_t M, int64_t N,
+                                    int64_t K, int gran, bsgemm_stream_t stream);
 
 /* Library version as major*10000 + minor*100 + patch. */
 int bsgemm_version(void);
