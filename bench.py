@@ -96,6 +96,42 @@ def algorithmic_bytes(p: workloads.Problem) -> int:
     return p.M * p.K + p.N * p.K + 2 * p.M * p.N + 4 * (-(-p.M // p.gran) + -(-p.N // p.gran)) * kb
 
 
+KERNEL_FILES = ("bsgemm_inst.cu", "bsgemm_kernel.cuh", "ptx.cuh")
+
+
+def kernel_source_hash() -> str:
+    """Short hash of the files that define the GEMM kernel (ties ncu figures to a kernel version)."""
+    import hashlib
+    h = hashlib.sha256()
+    for f in KERNEL_FILES:
+        path = os.path.join(ROOT, "fp8_block_scaled_bsgemm_b200", "csrc", f)
+        h.update(f.encode())
+        with open(path, "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic(workload: str):
+    """DRAM bytes per launch from a committed ncu summary of this workload, if it
+    was taken on the current kernel sources; otherwise None."""
+    import glob
+    want = kernel_source_hash()
+    for path in sorted(glob.glob(os.path.join(ROOT, "profiles", "*.md"))):
+        fields = {}
+        with open(path) as fh:
+            for ln in fh:
+                if ":" in ln and ln.split(":")[0] in ("kernel_source_sha256", "bench_workload",
+                                                      "traffic_bytes_per_launch"):
+                    k, v = ln.split(":", 1)
+                    fields[k.strip()] = v.strip()
+        if fields.get("bench_workload") == workload and fields.get("kernel_source_sha256") == want:
+            try:
+                return int(fields["traffic_bytes_per_launch"])
+            except (KeyError, ValueError):
+                return None
+    return None
+
+
 def measured_peaks() -> dict:
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(path):
@@ -317,7 +353,7 @@ def run_ours(args):
         peak = peaks["bf16_tflops"] * 2.0
         achieved = p.flops / (ms * 1e-3) / 1e12
         roof = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
-                "frac": achieved / peak, "traffic": None,
+                "frac": achieved / peak, "traffic": profiled_traffic(args.workload),
                 "peak_source": f"{peaks['source']} bf16 burst x 2 (FP8/BF16 nominal ratio)",
                 "frac_of_nominal_4500": achieved / 4500.0}
     else:
@@ -325,7 +361,7 @@ def run_ours(args):
         peak = peaks["hbm_gbs"]
         achieved = bytes_ / (ms * 1e-3) / 1e9
         roof = {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
-                "frac": achieved / peak, "traffic": None, "peak_source": f"{peaks['source']} hbm copy",
+                "frac": achieved / peak, "traffic": profiled_traffic(args.workload), "peak_source": f"{peaks['source']} hbm copy",
                 "algorithmic_bytes_per_launch": bytes_}
     line = {
         "metric": METRIC, "value": world * p.flops / (ms_max * 1e-3) / 1e12, "unit": "TFLOP/s",
