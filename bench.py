@@ -63,6 +63,8 @@ def parse_args(argv=None):
                     help="override the plan's variant (default: library heuristic)")
     ap.add_argument("--bnq", type=int, default=0, help="override the tile width on the MMA N side")
     ap.add_argument("--splits", type=int, default=0, help="override the K splits per tile")
+    ap.add_argument("--stream-k", type=int, default=0, choices=[-1, 0, 1],
+                    help="stream-K for a ragged last wave: -1 never, 0 library heuristic, 1 always")
     return ap.parse_args(argv)
 
 
@@ -275,8 +277,8 @@ def run_ours(args):
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
     num_sms = torch.cuda.get_device_properties(dev).multi_processor_count
     tuning = None
-    if args.variant != "auto" or args.bnq or args.splits:
-        tuning = {"variant": args.variant, "bnq": args.bnq, "splits": args.splits}
+    if args.variant != "auto" or args.bnq or args.splits or args.stream_k:
+        tuning = {"variant": args.variant, "bnq": args.bnq, "splits": args.splits, "stream_k": args.stream_k}
     plan = bsg.make_plan(p.M, p.N, p.K, p.gran, p.layout, num_sms, tuning)
 
     def gemm():

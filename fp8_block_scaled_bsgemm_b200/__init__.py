@@ -38,12 +38,14 @@ class BsgemmError(RuntimeError):
 
 
 class Tuning(ctypes.Structure):
-    _fields_ = [("variant", ctypes.c_int), ("bnq", ctypes.c_int), ("splits", ctypes.c_int)]
+    _fields_ = [("variant", ctypes.c_int), ("bnq", ctypes.c_int), ("splits", ctypes.c_int),
+                ("stream_k", ctypes.c_int)]
 
 
 class Plan(ctypes.Structure):
     _fields_ = [(n, ctypes.c_int) for n in ("layout", "gran", "swap_ab", "bnq", "tiles_p", "tiles_q",
-                                            "splits", "kb_per_split", "grid", "group_p", "kernels")]
+                                            "splits", "kb_per_split", "grid", "group_p", "kernels",
+                                            "sk_first_tile", "sk_units_per_tile", "sk_ctas", "sk_units")]
 
     def as_dict(self):
         return {n: getattr(self, n) for n, _ in self._fields_}
@@ -106,7 +108,7 @@ def _tuning(tuning):
     if isinstance(tuning, Tuning):
         return ctypes.byref(tuning)
     t = Tuning(VARIANTS[tuning.get("variant", "auto")], int(tuning.get("bnq", 0)),
-               int(tuning.get("splits", 0)))
+               int(tuning.get("splits", 0)), int(tuning.get("stream_k", 0)))
     return ctypes.byref(t)
 
 
@@ -165,6 +167,16 @@ def bsgemm_fp8_nn(a, b, scale_a, scale_b, out=None, gran=128, stream=None):
 
 def bsgemm_fp8_tt(a, b, scale_a, scale_b, out=None, gran=128, stream=None):
     return gemm(a, b, scale_a, scale_b, out, "tt", gran, None, stream)
+
+
+def scratch_bytes(plan: dict) -> int:
+    """Split-K / stream-K workspace bytes (FP32 partial tiles) a plan uses."""
+    tile = plan["bnq"] * 128 * 4
+    if plan["sk_ctas"] > 0:
+        return 2 * plan["sk_ctas"] * tile
+    if plan["splits"] > 1:
+        return plan["tiles_p"] * plan["tiles_q"] * plan["splits"] * tile
+    return 0
 
 
 def make_plan(M, N, K, gran=128, layout="nt", num_sms=148, tuning=None) -> dict:

@@ -190,19 +190,55 @@ extern "C" bsgemm_status bsgemm_make_plan(int layout, int64_t M, int64_t N, int6
   pl.tiles_q = static_cast<int>((Q + bnq - 1) / bnq);
   const int64_t tiles = static_cast<int64_t>(pl.tiles_p) * pl.tiles_q;
   if (tiles > (1 << 30)) return BSGEMM_ERR_INVALID_ARG;
-  // split-K only when the tiles alone cannot fill the SMs; among the split
-  // counts, take the one with the least estimated time:
-  //   waves(tiles * splits) * (K-blocks per split + per-item overhead),
-  // the overhead standing for the FP32 partial tile written and re-read
+  // K is handed out in units of one 128-deep stage (two K-blocks when g = 64)
+  const int unit_kb = (gran == 64) ? 2 : 1;
+  const int U = (Kb + unit_kb - 1) / unit_kb;
   auto split_fix = [&](int s, int& per) {
     per = (Kb + s - 1) / s;
     if (gran == 64 && (per & 1)) ++per;  // a split starts on a 128-element stage
     return (Kb + per - 1) / per;
   };
-  int splits = t ? t->splits : 0;
-  if (splits <= 0) {
-    splits = 1;
-    if (tiles < num_sms) {
+  const int splits_req = t ? t->splits : 0;
+  const int sk_req = t ? t->stream_k : 0;
+  int splits = 1;
+  pl.sk_first_tile = 0;
+  pl.sk_units_per_tile = U;
+  pl.sk_ctas = 0;
+  pl.sk_units = 0;
+  if (splits_req > 0) {
+    splits = splits_req;
+  } else {
+    // Stream-K when whole tiles would leave a ragged last wave: the full
+    // waves stay whole tiles and the remaining tiles' units are shared out
+    // evenly. Compared on the busiest CTA's units, with a partial tile written
+    // and re-read counted as (1 + width/128) units.  Measured on B200, the
+    // ranges only pay off when a tile has many units (K >= 64 K-blocks of
+    // 128) or, with fewer tiles than SMs, when the tiles are at least 64
+    // wide; below that whole tiles (or split-K) win, so the heuristic keeps
+    // to those cases.  stream_k = 1 forces it wherever a wave is ragged.
+    const int64_t full = (tiles / num_sms) * num_sms;
+    const int64_t rem = tiles - full;
+    const bool sk_pays = tiles < num_sms ? bnq >= 64 : U * unit_kb * gran >= 64 * 128;
+    bool use_sk = false;
+    if (rem > 0 && sk_req >= 0 && (sk_req > 0 || sk_pays)) {
+      const int64_t R = rem * U;
+      int64_t gp = R / 4;  // at least ~4 units per CTA
+      if (gp > num_sms) gp = num_sms;
+      if (gp < 1) gp = 1;
+      const double piece_cost = 1.0 + bnq / 128.0;
+      const double cost_dp = static_cast<double>((tiles + num_sms - 1) / num_sms) * U;
+      const double cost_sk = static_cast<double>(full / num_sms) * U +
+                             static_cast<double>((R + gp - 1) / gp) + 2.0 * piece_cost;
+      if (R < (int64_t(1) << 31) && (sk_req > 0 || cost_sk < cost_dp)) {
+        use_sk = true;
+        pl.sk_first_tile = static_cast<int>(full);
+        pl.sk_ctas = static_cast<int>(gp);
+        pl.sk_units = static_cast<int>(R);
+      }
+    }
+    if (!use_sk && tiles < num_sms) {
+      // no stream-K: split-K fills the SMs; among the split counts take the
+      // least estimated time, waves(tiles * splits) * (K-blocks per split + overhead)
       const double overhead = 1.0 + bnq / 64.0;
       double best = 1e30;
       for (int s = 1; s <= Kb && s <= 64; ++s) {
@@ -218,7 +254,9 @@ extern "C" bsgemm_status bsgemm_make_plan(int layout, int64_t M, int64_t N, int6
   int per = 0;
   pl.splits = split_fix(splits, per);
   pl.kb_per_split = per;
-  const int64_t work = tiles * pl.splits;
+  const int64_t whole = pl.sk_ctas > 0 ? pl.sk_first_tile : tiles;
+  int64_t work = whole * pl.splits;
+  if (work < pl.sk_ctas) work = pl.sk_ctas;
   pl.grid = static_cast<int>(work < num_sms ? work : num_sms);
   pl.group_p = 16;
   pl.layout = layout;

@@ -48,26 +48,32 @@ bsgemm_status launch(const bsgemm_plan& plan, const void* a, const void* b, cons
 
   bsg::Params prm{};
   prm.M = M; prm.N = N; prm.K = K;
-  prm.P = P; prm.Q = Q;
   prm.Kb = (K + GRAN - 1) / GRAN;
   prm.Pb = (P + GRAN - 1) / GRAN;
   prm.Qb = (Q + GRAN - 1) / GRAN;
   prm.tiles_p = plan.tiles_p;
   prm.tiles_q = plan.tiles_q;
-  prm.num_tiles = plan.tiles_p * plan.tiles_q;
+  const int num_tiles = plan.tiles_p * plan.tiles_q;
   prm.splits = plan.splits;
   prm.kb_per_split = plan.kb_per_split;
-  prm.num_work = prm.num_tiles * plan.splits;
+  prm.num_work = (plan.sk_ctas > 0 ? plan.sk_first_tile : num_tiles) * plan.splits;
+  prm.sk_first_tile = plan.sk_first_tile;
+  prm.sk_units_per_tile = plan.sk_units_per_tile;
+  prm.sk_ctas = plan.sk_ctas;
+  prm.sk_q = plan.sk_ctas > 0 ? plan.sk_units / plan.sk_ctas : 0;
+  prm.sk_r = plan.sk_ctas > 0 ? plan.sk_units % plan.sk_ctas : 0;
   prm.group_p = plan.group_p;
   prm.sP = SWAP ? sb : sa;
   prm.sQ = SWAP ? sa : sb;
   prm.out = static_cast<__nv_bfloat16*>(out);
   prm.status = dev.status;
   prm.timeout_ns = wait_timeout_ns();
-  if (SPLIT && plan.splits > 1) {
+  if (SPLIT && (plan.splits > 1 || plan.sk_ctas > 0)) {
+    // split-K: one partial tile per piece; stream-K: two per CTA (its first and last tile)
+    const size_t partials = plan.sk_ctas > 0 ? 2 * (size_t)plan.sk_ctas : (size_t)prm.num_work;
+    const size_t counters = plan.sk_ctas > 0 ? (size_t)(num_tiles - plan.sk_first_tile) : (size_t)num_tiles;
     Workspace w;
-    bsgemm_status st = get_workspace(stream, (size_t)prm.num_work * BNQ * bsg::BM * sizeof(float),
-                                     (size_t)prm.num_tiles, w);
+    bsgemm_status st = get_workspace(stream, partials * BNQ * bsg::BM * sizeof(float), counters, w);
     if (st != BSGEMM_OK) return st;
     prm.ws = w.ws;
     prm.counters = w.counters;
@@ -105,7 +111,7 @@ bsgemm_status BSG_RUN_NAME(BSG_GRAN, BSG_LAYOUT)(const bsgemm_plan& pl, const vo
       default:  return BSGEMM_ERR_INVALID_ARG;
     }
   }
-  const bool split = pl.splits > 1;
+  const bool split = pl.splits > 1 || pl.sk_ctas > 0;
   switch (pl.bnq) {
     case 128:
       return split ? launch<128, G, false, kAMn, kBMn, true>(pl, a, b, sa, sb, out, M, N, K, s, d)

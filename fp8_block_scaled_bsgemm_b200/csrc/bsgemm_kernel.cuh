@@ -22,9 +22,15 @@
 //            acc += (sP*sQ) * partial in FP32 registers (packed f32x2 FMAs),
 //            release the TMEM buffer, and at the end of a tile round to BF16
 //            and store it straight from registers.
-// Split-K: a tile's K-blocks are divided among `splits` work items; each
-// writes an FP32 partial tile to a workspace, and the last to arrive (per-tile
-// counter) adds all partials in split order -- the same order every run -- and
+// Work is split three ways:
+//   whole tiles (data-parallel), walked by the persistent CTAs in raster order;
+//   split-K: every tile's K-blocks cut into `splits` equal pieces;
+//   stream-K: after the full waves of whole tiles, the remaining tiles'
+//     K-blocks, laid end to end, are cut into equal contiguous ranges, one
+//     per CTA, so no SM idles in a ragged last wave.
+// A piece that is not a whole tile writes its FP32 partial tile to a
+// workspace slot; the last piece of a tile to arrive (per-tile counter) adds
+// all the tile's partials in K order -- the same order every run -- and
 // stores the BF16 tile.
 //
 // Every mbarrier wait is bounded by a %globaltimer deadline.  When one runs
@@ -69,20 +75,24 @@ struct RegSplit {
 
 struct Params {
   int M, N, K;           // logical GEMM sizes
-  int P, Q;              // rows of the P operand and of the Q operand
   int Kb;                // ceil(K / gran)
   int Pb, Qb;            // ceil(P / gran), ceil(Q / gran)
   int tiles_p, tiles_q;  // tiles along P (128 rows) and along Q (BNQ rows)
-  int num_tiles;
   int splits;            // K splits per tile (1 = none)
   int kb_per_split;      // K-blocks per split (even when gran == 64)
-  int num_work;          // num_tiles * splits
+  int num_work;          // whole-tile or split-K work items: tiles before sk_first_tile, times splits
+  int sk_first_tile;     // stream-K: first tile handled by stream-K (tiles before it are whole)
+  int sk_units_per_tile; // stream-K: units (K-blocks; pairs of K-blocks when gran == 64) per tile
+  int sk_ctas;           // stream-K: CTAs sharing the stream-K units (0 = no stream-K)
+  int sk_q, sk_r;        // stream-K: the stream-K units number sk_q * sk_ctas + sk_r; the first
+                         // sk_r CTAs take sk_q + 1 of them, the others sk_q
   int group_p;           // raster group height in P tiles (L2 locality)
   const float* sP;       // [Pb][Kb]
   const float* sQ;       // [Qb][Kb]
   __nv_bfloat16* out;    // [M][N] row-major (direct stores in swap mode)
-  float* ws;             // split partials: [num_tiles][splits][BNQ][BM]
-  int* counters;         // [num_tiles], zero between launches
+  float* ws;             // partial tiles [slot][BNQ][BM]: split-K slot tile*splits+split,
+                         // stream-K slot 2*cta + (0: the CTA's first tile, 1: its last)
+  int* counters;         // one per split or stream-K tile, zero between launches
   int* status;           // device status word
   unsigned long long timeout_ns;
 };
@@ -114,7 +124,11 @@ struct __align__(8) Barriers {
   uint32_t tmem_base;
   int abort_flag;
   int split_last;
+  // per promotion warp: the current work item's Pieces (pieces, slot,
+  // counter, slot0, slot_base, slot_step), parked here for the K-loop
+  int pieces[kNumEpiWarps][6];
 };
+static_assert(sizeof(Barriers) <= 512, "barrier block is 512 bytes");
 
 // ---------------------------------------------------------------- helpers
 __device__ __forceinline__ void record_timeout(const Params& p, Barriers* bars, int where) {
@@ -183,26 +197,130 @@ __device__ __forceinline__ constexpr uint32_t instr_desc() {
 }
 
 struct Work {
-  int tile, split, tp, tq, kb0, kb1;
+  int tile, tp, tq, kb0, kb1;  // output tile and its K-blocks [kb0, kb1)
 };
 
-__device__ __forceinline__ Work decode_work(const Params& p, int w) {
-  Work x;
-  x.tile = w / p.splits;
-  x.split = w - x.tile * p.splits;
-  // grouped raster: walk group_p P-tiles down, then across Q
+// Tile index -> (P tile, Q tile) in grouped raster order: group_p P-tiles
+// down, then across Q, so concurrently running CTAs share operand tiles in L2.
+__device__ __forceinline__ void tile_coords(const Params& p, int tile, int& tp, int& tq) {
   const int per_group = p.group_p * p.tiles_q;
-  const int grp = x.tile / per_group;
+  const int grp = tile / per_group;
   const int first_p = grp * p.group_p;
   int rows = p.tiles_p - first_p;
   rows = rows < p.group_p ? rows : p.group_p;
-  const int local = x.tile - grp * per_group;
-  x.tp = first_p + local % rows;
-  x.tq = local / rows;
-  x.kb0 = x.split * p.kb_per_split;
-  x.kb1 = x.kb0 + p.kb_per_split;
-  if (x.kb1 > p.Kb) x.kb1 = p.Kb;
-  return x;
+  const int local = tile - grp * per_group;
+  tp = first_p + local % rows;
+  tq = local / rows;
+}
+
+// Stream-K: CTA c owns units [sk_start(c), sk_start(c + 1)); the first sk_r
+// CTAs take sk_q + 1 units, the others sk_q (32-bit arithmetic throughout).
+// A unit is one K-block, or two (one 128-deep stage) when gran == 64.
+__device__ __forceinline__ int sk_start(const Params& p, int c) {
+  return c * p.sk_q + min(c, p.sk_r);
+}
+// The CTA whose range holds unit u.
+__device__ __forceinline__ int sk_owner(const Params& p, int u) {
+  const int split = p.sk_r * (p.sk_q + 1);  // units held by the CTAs with one extra unit
+  return u < split ? u / (p.sk_q + 1) : p.sk_r + (u - split) / p.sk_q;
+}
+
+// Every role of a CTA walks the same sequence of work items: first its whole
+// tiles or split-K pieces (blockIdx.x, +gridDim.x, ...), then the segments of
+// its stream-K range, one per tile the range touches.
+struct WorkIter {
+  int wi;  // next whole-tile / split-K item
+  int u;   // next stream-K unit
+};
+
+template <bool SPLIT>
+__device__ __forceinline__ void work_begin(const Params& p, WorkIter& it) {
+  it.wi = blockIdx.x;
+  it.u = 0;
+  if (SPLIT && static_cast<int>(blockIdx.x) < p.sk_ctas) it.u = sk_start(p, blockIdx.x);
+}
+
+// Instances without the partial-tile fix-up (SPLIT false) never get a
+// stream-K range, so their walk is the whole-tile loop alone.
+template <int GRAN, bool SPLIT>
+__device__ __forceinline__ bool work_next(const Params& p, WorkIter& it, Work& w) {
+  if (it.wi < p.num_work) {
+    w.tile = it.wi / p.splits;
+    const int split = it.wi - w.tile * p.splits;
+    tile_coords(p, w.tile, w.tp, w.tq);
+    w.kb0 = split * p.kb_per_split;
+    w.kb1 = min(p.Kb, w.kb0 + p.kb_per_split);
+    it.wi += gridDim.x;
+    return true;
+  }
+  if constexpr (SPLIT) {
+    const int bid = static_cast<int>(blockIdx.x);
+    const int u_end = bid < p.sk_ctas ? sk_start(p, bid + 1) : 0;
+    if (it.u < u_end) {
+      constexpr int kUnitKb = GRAN == 64 ? 2 : 1;
+      const int U = p.sk_units_per_tile;
+      const int t_local = it.u / U;
+      const int tile_u0 = t_local * U;
+      const int seg_end = min(u_end, tile_u0 + U);
+      w.tile = p.sk_first_tile + t_local;
+      tile_coords(p, w.tile, w.tp, w.tq);
+      w.kb0 = (it.u - tile_u0) * kUnitKb;
+      w.kb1 = min(p.Kb, (seg_end - tile_u0) * kUnitKb);
+      it.u = seg_end;
+      return true;
+    }
+  }
+  return false;
+}
+
+// Where a work item's partial goes and where its tile's other pieces are,
+// from the item alone.
+struct Pieces {
+  int pieces;   // pieces the tile is cut into (1: the item is the whole tile)
+  int slot;     // workspace slot of this item's partial
+  int counter;  // arrival counter of the tile
+  // slots of the tile's pieces in K order: piece 0 in slot0, piece j > 0 in
+  // slot_base + j * slot_step
+  int slot0, slot_base, slot_step;
+};
+
+template <int GRAN>
+__device__ __forceinline__ Pieces pieces_of(const Params& p, const Work& w) {
+  Pieces r;
+  if (p.sk_ctas == 0 || w.tile < p.sk_first_tile) {
+    // whole tile or split-K piece
+    r.pieces = p.splits;
+    r.counter = w.tile;
+    r.slot0 = r.slot_base = w.tile * p.splits;
+    r.slot_step = 1;
+    r.slot = r.slot_base + w.kb0 / p.kb_per_split;
+    return r;
+  }
+  // stream-K segment.  A CTA's partial pieces are the first and the last
+  // segment of its range: slot 2c for its first, 2c + 1 for its last.  Piece
+  // j > 0 of a tile starts its CTA's range (slot 2c); piece 0 is its CTA's
+  // first segment only if that CTA's range starts at the tile's first unit.
+  constexpr int kUnitKb = GRAN == 64 ? 2 : 1;
+  const int U = p.sk_units_per_tile;
+  const int t_local = w.tile - p.sk_first_tile;
+  const int tile_u0 = t_local * U;
+  const int bid = static_cast<int>(blockIdx.x);
+  r.counter = t_local;
+  r.pieces = 1;
+  r.slot = r.slot0 = r.slot_base = 0;
+  r.slot_step = 2;
+  if (w.kb0 != 0 || w.kb1 != p.Kb) {
+    const int first_cta = sk_owner(p, tile_u0);
+    r.pieces = sk_owner(p, tile_u0 + U - 1) - first_cta + 1;
+    r.slot = 2 * bid + (tile_u0 + w.kb0 / kUnitKb == sk_start(p, bid) ? 0 : 1);
+    r.slot_base = 2 * first_cta;
+    r.slot0 = r.slot_base + (sk_start(p, first_cta) < tile_u0 ? 1 : 0);
+  }
+  return r;
+}
+
+__device__ __forceinline__ int piece_slot(const Pieces& pc, int j) {
+  return j == 0 ? pc.slot0 : pc.slot_base + j * pc.slot_step;
 }
 
 // Pipeline stages [st0, st1) of 128 K-elements that K-blocks [kb0, kb1) cover.
@@ -288,8 +406,9 @@ __global__ void __launch_bounds__(kNumThreads, 1)
     if (lane == 0) {
       uint32_t it = 0;  // stage-slot uses so far
       bool ok = true;
-      for (int wi = blockIdx.x; wi < p.num_work && ok; wi += gridDim.x) {
-        const Work w = decode_work(p, wi);
+      WorkIter wit;
+      work_begin<SPLIT>(p, wit);
+      for (Work w; ok && work_next<GRAN, SPLIT>(p, wit, w);) {
         int st0, st1;
         stage_range<GRAN>(p, w, st0, st1);
         for (int st = st0; st < st1; ++st, ++it) {
@@ -327,8 +446,9 @@ __global__ void __launch_bounds__(kNumThreads, 1)
     // first k-step, releasing it after its last -- and commits the buffer to
     // the promotion warps as soon as the block's last MMA is issued (the
     // promotion of block kb gates the MMAs of block kb + kBufs).  The issue
-    // path is straight-line code on one lane: per-MMA branching in a
-    // converged warp costs far more than the MMA issue itself.
+    // path is straight-line code on one lane: measured in this kernel, both a
+    // converged warp that branches per MMA and a converged warp whose lanes
+    // all wait (one lane issuing) are slower.
     if (lane == 0) {
       constexpr uint32_t idesc = instr_desc<BNQ, P_MN, Q_MN>();
       // descriptor steps: per k-step of 32 (K-major +32 B, MN-major +32 rows
@@ -341,12 +461,17 @@ __global__ void __launch_bounds__(kNumThreads, 1)
       uint32_t s = 0, ph = 0;     // pipeline stage and its phase
       uint32_t b = 0, bph = 0;    // TMEM buffer and its phase
       bool ok = true;
-      for (int wi = blockIdx.x; wi < p.num_work && ok; wi += gridDim.x) {
-        const Work w = decode_work(p, wi);
+      WorkIter wit;
+      work_begin<SPLIT>(p, wit);
+      for (Work w; ok && work_next<GRAN, SPLIT>(p, wit, w);) {
         for (int kb = w.kb0; kb < w.kb1; ++kb) {
-          // the promotion warps arrive only after tcgen05.wait::ld, so their
-          // reads of this buffer are complete before it is overwritten
-          if (!bounded_wait(smem_addr(&bars->tmem_empty[b]), bph ^ 1, p, bars, 3)) { ok = false; break; }
+          // Order of the waits: the stage's operands first (normally already
+          // loaded, so that wait is cheap and happens while the tensor pipe
+          // still works on the previous block), then the TMEM buffer, which
+          // gates the MMAs; the promotion warps arrive on tmem_empty only
+          // after tcgen05.wait::ld, so their reads of the buffer are complete
+          // before it is overwritten.  Commits: tmem_full first (the
+          // promotion warps wait on it), then the stage release.
           const uint32_t d_tmem = tmem_base + b * BNQ;
           if constexpr (GRAN >= BK) {
             // whole stages: GRAN / 128 of them, 4 k-steps each (fewer at the K tail)
@@ -356,6 +481,10 @@ __global__ void __launch_bounds__(kNumThreads, 1)
               if (k0 >= p.K) break;
               // TMA writes and MMA reads are async-proxy accesses ordered by this barrier
               if (!bounded_wait(smem_addr(&bars->full[s]), ph, p, bars, 2)) { ok = false; break; }
+              if (j == 0 && !bounded_wait(smem_addr(&bars->tmem_empty[b]), bph ^ 1, p, bars, 3)) {
+                ok = false;
+                break;
+              }
               const uint64_t ad = ad0 + s * kPStage, bd = bd0 + s * kQStage;
               if (k0 + BK <= p.K) {
 #pragma unroll
@@ -366,6 +495,7 @@ __global__ void __launch_bounds__(kNumThreads, 1)
                 for (int t = 0; t < nsteps; ++t)
                   mma_f8f6f4(d_tmem, ad + t * kPStep, bd + t * kQStep, idesc, (j > 0 || t > 0) ? 1u : 0u);
               }
+              if (j == GRAN / BK - 1 || k0 + BK >= p.K) mma_commit(smem_addr(&bars->tmem_full[b]));
               mma_commit(smem_addr(&bars->empty[s]));  // stage free once these MMAs finish
               if (++s == STAGES) { s = 0; ph ^= 1; }
             }
@@ -376,16 +506,17 @@ __global__ void __launch_bounds__(kNumThreads, 1)
             const int k0 = kb * GRAN;
             const int t0 = (kb & 1) * 2;
             if (t0 == 0 && !bounded_wait(smem_addr(&bars->full[s]), ph, p, bars, 2)) { ok = false; break; }
+            if (!bounded_wait(smem_addr(&bars->tmem_empty[b]), bph ^ 1, p, bars, 3)) { ok = false; break; }
             const uint64_t ad = ad0 + s * kPStage, bd = bd0 + s * kQStage;
             const int nsteps = (p.K - k0 >= GRAN) ? 2 : (p.K - k0 + kMmaK - 1) / kMmaK;
             for (int t = 0; t < nsteps; ++t)
               mma_f8f6f4(d_tmem, ad + (t0 + t) * kPStep, bd + (t0 + t) * kQStep, idesc, t > 0 ? 1u : 0u);
+            mma_commit(smem_addr(&bars->tmem_full[b]));
             if (t0 == 2 || k0 + GRAN >= p.K) {
               mma_commit(smem_addr(&bars->empty[s]));
               if (++s == STAGES) { s = 0; ph ^= 1; }
             }
           }
-          mma_commit(smem_addr(&bars->tmem_full[b]));
           if (++b == kBufs) { b = 0; bph ^= 1; }
         }
       }
@@ -406,8 +537,22 @@ __global__ void __launch_bounds__(kNumThreads, 1)
     bool ok = true;
     float2 acc[kHalf / 2];    // this thread's row, columns [half*kHalf, (half+1)*kHalf)
 
-    for (int wi = blockIdx.x; wi < p.num_work && ok; wi += gridDim.x) {
-      const Work w = decode_work(p, wi);
+    WorkIter wit;
+    work_begin<SPLIT>(p, wit);
+    for (Work w; ok && work_next<GRAN, SPLIT>(p, wit, w);) {
+      if constexpr (SPLIT) {
+        // where this item's partial goes: worked out while the accumulator
+        // is dead and parked in shared memory (registers are short during
+        // the K-loop); each warp has its own copy
+        const Pieces pq = pieces_of<GRAN>(p, w);
+        __syncwarp();
+        if (lane == 0) {
+          volatile int* d = bars->pieces[ew];
+          d[0] = pq.pieces; d[1] = pq.slot; d[2] = pq.counter;
+          d[3] = pq.slot0; d[4] = pq.slot_base; d[5] = pq.slot_step;
+        }
+        __syncwarp();
+      }
 #pragma unroll
       for (int i = 0; i < kHalf / 2; ++i) acc[i] = make_float2(0.f, 0.f);
 
@@ -454,15 +599,20 @@ __global__ void __launch_bounds__(kNumThreads, 1)
         if (!warp_wait(smem_addr(&bars->tmem_full[buf]), (pc / kBufs) & 1, p, bars, 4)) { ok = false; break; }
         const uint32_t taddr = tmem_base + t_lane + buf * BNQ + half * kHalf;
         {
-          // TMEM -> registers in chunks of 32 columns; with up to 64
-          // accumulator columns per thread the next chunk's load is in flight
-          // while the current one is scaled (two chunks of staging), with 128
-          // there is room for one chunk only
-          constexpr int CW = kHalf < 32 ? kHalf : 32;
+          // TMEM -> registers in chunks of up to 64 columns.  The buffer is
+          // released as soon as the last chunk is in registers, before that
+          // chunk is scaled, so the MMA can start refilling it sooner.
+          constexpr int CW = kHalf < 64 ? kHalf : 64;
           constexpr int NC = kHalf / CW;
-          constexpr bool kDouble = kHalf <= 64;
-          uint32_t ra[CW], rb[CW];
-          auto fma_chunk = [&](const uint32_t (&r)[CW], int c) {
+          uint32_t r[CW];
+#pragma unroll
+          for (int c = 0; c < NC; ++c) {
+            tmem_ld(taddr + c * CW, r);
+            tmem_wait_ld(r);
+            if (c == NC - 1) {
+              __syncwarp();
+              if (lane == 0) mbar_arrive(smem_addr(&bars->tmem_empty[buf]));
+            }
 #pragma unroll
             for (int i = 0; i < CW / 2; ++i) {
               const float2 sv = s2[(c * CW + 2 * i) / kGroupCols];
@@ -470,41 +620,22 @@ __global__ void __launch_bounds__(kNumThreads, 1)
                   ffma2(make_float2(__uint_as_float(r[2 * i]), __uint_as_float(r[2 * i + 1])), sv,
                         acc[c * (CW / 2) + i]);
             }
-          };
-          if constexpr (kDouble) {
-            tmem_ld(taddr, ra);
-            tmem_wait_ld(ra);
-#pragma unroll
-            for (int c = 0; c < NC; c += 2) {
-              if (c + 1 < NC) tmem_ld(taddr + (c + 1) * CW, rb);
-              fma_chunk(ra, c);
-              if (c + 1 < NC) {
-                tmem_wait_ld(rb);
-                if (c + 2 < NC) tmem_ld(taddr + (c + 2) * CW, ra);
-                fma_chunk(rb, c + 1);
-                if (c + 2 < NC) tmem_wait_ld(ra);
-              }
-            }
-          } else {
-            (void)rb;
-#pragma unroll
-            for (int c = 0; c < NC; ++c) {
-              tmem_ld(taddr + c * CW, ra);
-              tmem_wait_ld(ra);
-              fma_chunk(ra, c);
-            }
           }
         }
-        __syncwarp();
-        if (lane == 0) mbar_arrive(smem_addr(&bars->tmem_empty[buf]));
       }
       if (!ok) break;
 
-      // ---------------------------------------------------------- split-K fix-up
+      // ---------------------------------------------------------- partial-tile fix-up
       if constexpr (SPLIT) {
-        if (p.splits > 1) {
+        Pieces pcs;
+        {
+          const volatile int* d = bars->pieces[ew];
+          pcs.pieces = d[0]; pcs.slot = d[1]; pcs.counter = d[2];
+          pcs.slot0 = d[3]; pcs.slot_base = d[4]; pcs.slot_step = d[5];
+        }
+        if (pcs.pieces > 1) {
           // partial tile, column-major [BNQ][BM]: a warp writes 128 contiguous bytes per column
-          float* my_ws = p.ws + (static_cast<size_t>(w.tile) * p.splits + w.split) * (BNQ * BM);
+          float* my_ws = p.ws + static_cast<size_t>(pcs.slot) * (BNQ * BM);
 #pragma unroll
           for (int i = 0; i < kHalf / 2; ++i) {
             __stcg(my_ws + (half * kHalf + 2 * i) * BM + row_in_tile, acc[i].x);
@@ -514,8 +645,8 @@ __global__ void __launch_bounds__(kNumThreads, 1)
           // the partial now lives in the workspace; acc is dead until the sum below
           named_barrier_sync(1, kNumEpiThreads);
           if (ew == 0 && lane == 0) {
-            const int old = atomicAdd(p.counters + w.tile, 1);
-            bars->split_last = (old == p.splits - 1) ? 1 : 0;
+            const int old = atomicAdd(p.counters + pcs.counter, 1);
+            bars->split_last = (old == pcs.pieces - 1) ? 1 : 0;
           }
           named_barrier_sync(1, kNumEpiThreads);
           const bool last = *reinterpret_cast<volatile int*>(&bars->split_last) != 0;
@@ -523,23 +654,25 @@ __global__ void __launch_bounds__(kNumThreads, 1)
           named_barrier_sync(1, kNumEpiThreads);
           if (!last) continue;
           __threadfence();
-          // fixed order: split 0, 1, ..., whoever arrived last
-          const float* tile_ws = p.ws + static_cast<size_t>(w.tile) * p.splits * (BNQ * BM) +
-                                 (half * kHalf) * BM + row_in_tile;
+          // fixed order: the tile's pieces in K order, whoever arrived last
+          const size_t col_off = static_cast<size_t>(half * kHalf) * BM + row_in_tile;
+          {
+            const float* src = p.ws + static_cast<size_t>(piece_slot(pcs, 0)) * (BNQ * BM) + col_off;
 #pragma unroll
-          for (int i = 0; i < kHalf / 2; ++i) {
-            acc[i].x = __ldcg(tile_ws + (2 * i) * BM);
-            acc[i].y = __ldcg(tile_ws + (2 * i + 1) * BM);
+            for (int i = 0; i < kHalf / 2; ++i) {
+              acc[i].x = __ldcg(src + (2 * i) * BM);
+              acc[i].y = __ldcg(src + (2 * i + 1) * BM);
+            }
           }
-          for (int sidx = 1; sidx < p.splits; ++sidx) {
-            const float* src = tile_ws + static_cast<size_t>(sidx) * (BNQ * BM);
+          for (int j = 1; j < pcs.pieces; ++j) {
+            const float* src = p.ws + static_cast<size_t>(piece_slot(pcs, j)) * (BNQ * BM) + col_off;
 #pragma unroll
             for (int i = 0; i < kHalf / 2; ++i) {
               acc[i].x += __ldcg(src + (2 * i) * BM);
               acc[i].y += __ldcg(src + (2 * i + 1) * BM);
             }
           }
-          if (ew == 0 && lane == 0) p.counters[w.tile] = 0;  // ready for the next launch
+          if (ew == 0 && lane == 0) p.counters[pcs.counter] = 0;  // ready for the next launch
         }
       }
 

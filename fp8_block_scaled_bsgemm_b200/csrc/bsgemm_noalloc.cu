@@ -5,11 +5,12 @@
 // inside a host allocator callback, under a framework that owns all device
 // memory and hands out nothing but the tensors it passes in, or in a process
 // that must not grow its device footprint after start-up.  The regular entry
-// points create a split-K workspace on first use with cudaMalloc; this one
-// never does.
+// points create a split-K / stream-K workspace on first use with cudaMalloc;
+// this one never does.
 //
-// Instead, the split-K scratch (FP32 partial tiles plus one counter per output
-// tile) is a fixed array in the library's own device memory, declared below.
+// Instead, that scratch (FP32 partial tiles plus one counter per output tile
+// that is cut into pieces) is a fixed array in the library's own device
+// memory, declared below.
 // Every GPU that loads the library holds one copy of it until the process
 // exits.  Its size bounds what this entry point accepts: a problem whose plan
 // needs more scratch than the array holds is rejected with
@@ -88,7 +89,29 @@ bsgemm_status setup_current_device(DeviceScratch*& out) {
   return BSGEMM_OK;
 }
 
-// Same kernel as the regular NT split-K path, launched on the fixed scratch.
+// Partial tiles and tile counters a plan needs: split-K one partial per piece
+// and one counter per tile; stream-K two partials per CTA and one counter per
+// stream-K tile; none without either.
+void scratch_need(const bsgemm_plan& pl, size_t& partials, size_t& counters) {
+  const size_t tiles = (size_t)pl.tiles_p * pl.tiles_q;
+  if (pl.sk_ctas > 0) {
+    partials = 2 * (size_t)pl.sk_ctas;
+    counters = tiles - pl.sk_first_tile;
+  } else if (pl.splits > 1) {
+    partials = tiles * pl.splits;
+    counters = tiles;
+  } else {
+    partials = counters = 0;
+  }
+}
+
+bool fits(const bsgemm_plan& pl) {
+  size_t partials = 0, counters = 0;
+  scratch_need(pl, partials, counters);
+  return partials * pl.bnq * bsg::BM * sizeof(float) <= kPartialBytes && counters <= (size_t)kMaxTiles;
+}
+
+// Same kernel as the regular NT split-K / stream-K path, launched on the fixed scratch.
 template <int BNQ, int GRAN, bool SWAP>
 bsgemm_status launch_fixed(const bsgemm_plan& plan, const void* a, const void* b, const float* sa,
                            const float* sb, void* out, int M, int N, int K, cudaStream_t stream,
@@ -106,29 +129,35 @@ bsgemm_status launch_fixed(const bsgemm_plan& plan, const void* a, const void* b
 
   bsg::Params prm{};
   prm.M = M; prm.N = N; prm.K = K;
-  prm.P = P; prm.Q = Q;
   prm.Kb = (K + GRAN - 1) / GRAN;
   prm.Pb = (P + GRAN - 1) / GRAN;
   prm.Qb = (Q + GRAN - 1) / GRAN;
   prm.tiles_p = plan.tiles_p;
   prm.tiles_q = plan.tiles_q;
-  prm.num_tiles = plan.tiles_p * plan.tiles_q;
+  const int num_tiles = plan.tiles_p * plan.tiles_q;
   prm.splits = plan.splits;
   prm.kb_per_split = plan.kb_per_split;
-  prm.num_work = prm.num_tiles * plan.splits;
+  prm.num_work = (plan.sk_ctas > 0 ? plan.sk_first_tile : num_tiles) * plan.splits;
+  prm.sk_first_tile = plan.sk_first_tile;
+  prm.sk_units_per_tile = plan.sk_units_per_tile;
+  prm.sk_ctas = plan.sk_ctas;
+  prm.sk_q = plan.sk_ctas > 0 ? plan.sk_units / plan.sk_ctas : 0;
+  prm.sk_r = plan.sk_ctas > 0 ? plan.sk_units % plan.sk_ctas : 0;
   prm.group_p = plan.group_p;
   prm.sP = SWAP ? sb : sa;
   prm.sQ = SWAP ? sa : sb;
   prm.out = static_cast<__nv_bfloat16*>(out);
   prm.status = d.status;
   prm.timeout_ns = bsg_host::wait_timeout_ns();
-  if (plan.splits > 1) {
-    const size_t need = (size_t)prm.num_work * BNQ * bsg::BM * sizeof(float);
-    if (need > kPartialBytes || prm.num_tiles > kMaxTiles) return BSGEMM_ERR_SCRATCH_LIMIT;
+  if (plan.splits > 1 || plan.sk_ctas > 0) {
+    size_t partials = 0, counters = 0;
+    scratch_need(plan, partials, counters);
+    if (partials * BNQ * bsg::BM * sizeof(float) > kPartialBytes || counters > (size_t)kMaxTiles)
+      return BSGEMM_ERR_SCRATCH_LIMIT;
     prm.ws = reinterpret_cast<float*>(d.base);
     prm.counters = reinterpret_cast<int*>(d.base + kPartialBytes);
     // the counters must start at zero; the array keeps the previous call's contents
-    if (cudaMemsetAsync(prm.counters, 0, (size_t)prm.num_tiles * sizeof(int), stream) != cudaSuccess)
+    if (cudaMemsetAsync(prm.counters, 0, counters * sizeof(int), stream) != cudaSuccess)
       return BSGEMM_ERR_CUDA;
   }
   if (bsg::RegSplit<BNQ>::kEnabled) {
@@ -180,9 +209,16 @@ extern "C" bsgemm_status bsgemm_fp8_nt_noalloc(const void* a, const void* b, con
   DeviceScratch* d = nullptr;
   bsgemm_status st = setup_current_device(d);
   if (st != BSGEMM_OK) return st;
+  // the regular plan when its scratch fits; otherwise the plan without stream-K
   bsgemm_plan pl;
   st = bsgemm_make_plan(BSGEMM_LAYOUT_NT, M, N, K, gran, d->num_sms, nullptr, &pl);
   if (st != BSGEMM_OK) return st;
+  if (!fits(pl)) {
+    const bsgemm_tuning no_sk = {0, 0, 0, -1};
+    st = bsgemm_make_plan(BSGEMM_LAYOUT_NT, M, N, K, gran, d->num_sms, &no_sk, &pl);
+    if (st != BSGEMM_OK) return st;
+    if (!fits(pl)) return BSGEMM_ERR_SCRATCH_LIMIT;
+  }
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const int m = static_cast<int>(M), n = static_cast<int>(N), k = static_cast<int>(K);
   switch (gran) {

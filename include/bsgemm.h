@@ -119,9 +119,10 @@ typedef enum {
 
 /* Optional overrides of the plan; 0 in any field means "choose". */
 typedef struct {
-    int variant; /* bsgemm_variant */
-    int bnq;     /* tile width on the MMA N side: 128/256 (data-parallel), 16..128 (swap-AB) */
-    int splits;  /* K splits per output tile (split-K) */
+    int variant;  /* bsgemm_variant */
+    int bnq;      /* tile width on the MMA N side: 128/256 (data-parallel), 16..128 (swap-AB) */
+    int splits;   /* K splits per output tile (split-K); > 0 turns stream-K off */
+    int stream_k; /* 0 choose, 1 use stream-K whenever tiles would leave SMs idle, -1 never */
 } bsgemm_tuning;
 
 /* What one call will launch (filled by bsgemm_make_plan). */
@@ -135,6 +136,10 @@ typedef struct {
     int grid;           /* persistent CTAs launched (<= number of SMs) */
     int group_p;        /* raster group height in tiles */
     int kernels;        /* kernel launches per call */
+    int sk_first_tile;  /* stream-K: tiles before this one are computed whole, in full waves */
+    int sk_units_per_tile; /* stream-K: units per tile (a unit is one K block; two when gran = 64) */
+    int sk_ctas;        /* stream-K: CTAs sharing the remaining tiles' units (0: no stream-K) */
+    int sk_units;       /* stream-K: units of all stream-K tiles together */
 } bsgemm_plan;
 
 /* The operation above with the layout as an argument and optional tuning
@@ -178,14 +183,17 @@ bsgemm_status bsgemm_diag_wait_timeout(unsigned long long timeout_ns, bsgemm_str
  * (no cudaMalloc, cudaFree or allocating library call, torch's included).
  *
  * It computes exactly what bsgemm_fp8_nt computes, with the same arguments,
- * rules and errors, and with the same kernels and plan.  Its split-K scratch
- * is a fixed array inside the library's device memory: each GPU that loads
+ * rules and errors, and with the same kernels.  It takes the same plan when
+ * that plan's scratch fits the array, otherwise the plan without stream-K.
+ * Its split-K / stream-K scratch is a fixed array inside the library's device
+ * memory: each GPU that loads
  * the library holds BSGEMM_NOALLOC_SCRATCH_BYTES of FP32 partial tiles plus
  * BSGEMM_NOALLOC_MAX_TILES tile counters until the process exits.  A problem
- * whose plan needs more -- (tiles x splits) x tile width x 128 x 4 bytes of
- * partials, or more tiles than counters -- is rejected with
+ * whose plan needs more -- split-K: tiles x splits partial tiles; stream-K:
+ * 2 x sk_ctas partial tiles; a partial tile is tile width x 128 x 4 bytes --
+ * or more tile counters than it holds, even without stream-K, is rejected with
  * BSGEMM_ERR_SCRATCH_LIMIT before anything is launched.  Problems whose plan
- * does not split K use no scratch at all.
+ * neither splits K nor uses stream-K need no scratch at all.
  *
  * The first call on each device looks up the array's device address (once,
  * with that device current); make that first call before any stream capture.

@@ -49,13 +49,83 @@ def test_plan_is_consistent(M, N, K, gran, want_swap):
     assert pl["splits"] * pl["kb_per_split"] >= Kb > (pl["splits"] - 1) * pl["kb_per_split"]
     if gran == 64:
         assert pl["kb_per_split"] % 2 == 0 or pl["splits"] == 1
+    tiles = pl["tiles_p"] * pl["tiles_q"]
+    U = -(-Kb // (2 if gran == 64 else 1))
+    assert pl["sk_units_per_tile"] == U
     assert 1 <= pl["grid"] <= 148
-    assert pl["grid"] == min(148, pl["tiles_p"] * pl["tiles_q"] * pl["splits"])
+    if pl["sk_ctas"] > 0:
+        # whole tiles in full waves, then the rest shared out by stream-K
+        assert pl["splits"] == 1 and pl["sk_first_tile"] % 148 == 0
+        assert pl["sk_units"] == (tiles - pl["sk_first_tile"]) * U
+        assert 1 <= pl["sk_ctas"] <= min(148, pl["sk_units"])
+        assert pl["grid"] == min(148, max(pl["sk_first_tile"], pl["sk_ctas"]))
+    else:
+        assert pl["grid"] == min(148, tiles * pl["splits"])
 
 
 def test_plan_fills_the_machine_for_small_m():
     pl = bsg.make_plan(1, 7168, 7168, 128, "nt", 148)
-    assert pl["tiles_p"] * pl["splits"] >= 100
+    assert max(pl["tiles_p"] * pl["splits"], pl["sk_ctas"]) >= 100
+
+
+def test_plan_uses_stream_k_for_a_ragged_last_wave():
+    # long K: 256 tiles = 1 wave + 108, whose units are shared out
+    pl = bsg.make_plan(2048, 4096, 32768, 128, "nt", 148)
+    assert pl["sk_first_tile"] == 148 and pl["sk_ctas"] == 148
+    assert bsg.make_plan(2048, 4096, 32768, 128, "nt", 148, {"stream_k": -1})["sk_ctas"] == 0
+    assert bsg.make_plan(2048, 4096, 32768, 128, "nt", 148, {"splits": 2})["sk_ctas"] == 0
+    # short K (32 K-blocks): whole tiles unless forced
+    assert bsg.make_plan(4096, 4096, 4096, 128, "nt", 148)["sk_ctas"] == 0
+    forced = bsg.make_plan(4096, 4096, 4096, 128, "nt", 148, {"stream_k": 1})
+    assert forced["sk_first_tile"] == 444 and forced["sk_ctas"] == 148
+    # fewer tiles than SMs: stream-K for tiles at least 64 wide, split-K below
+    assert bsg.make_plan(128, 7168, 7168, 128, "nt", 148)["sk_ctas"] == 148
+    small = bsg.make_plan(16, 7168, 7168, 128, "nt", 148)
+    assert small["sk_ctas"] == 0 and small["splits"] > 1
+    # an exact number of full waves needs no stream-K
+    assert bsg.make_plan(128 * 148, 256, 1024, 128, "nt", 148, {"stream_k": 1})["sk_ctas"] == 0
+
+
+def _sk_partition(tiles_sk, U, G):
+    """Mirror of the kernel's stream-K walk (sk_start, sk_owner, piece slots)."""
+    R = tiles_sk * U
+    q, r = divmod(R, G)
+    start = lambda c: c * q + min(c, r)
+    owner = lambda u: u // (q + 1) if u < r * (q + 1) else r + (u - r * (q + 1)) // q
+    assert start(G) == R and all(owner(u) == max(c for c in range(G) if start(c) <= u) for u in range(R))
+    pieces = {}
+    for c in range(G):
+        u, ue = start(c), start(c + 1)
+        while u < ue:
+            t = u // U
+            t0 = t * U
+            se = min(ue, t0 + U)
+            slot = 2 * c + (0 if start(c) // U == t else 1)
+            pieces.setdefault(t, []).append((c, u - t0, se - t0, slot, owner(t0), owner(t0 + U - 1)))
+            u = se
+    return pieces, start
+
+
+@pytest.mark.parametrize("tiles_sk,U,G", [(68, 32, 148), (56, 56, 148), (108, 256, 148), (1, 2, 1),
+                                          (3, 5, 7), (32, 32, 148), (5, 3, 4), (16, 64, 148)])
+def test_stream_k_partition_covers_each_tile_once_in_k_order(tiles_sk, U, G):
+    pieces, start = _sk_partition(tiles_sk, U, G)
+    assert sorted(pieces) == list(range(tiles_sk))
+    used = set()
+    for t, ps in pieces.items():
+        # contiguous cover of [0, U) by CTAs in increasing order
+        assert ps[0][1] == 0 and ps[-1][2] == U
+        for a, b in zip(ps, ps[1:]):
+            assert a[2] == b[1] and b[0] == a[0] + 1
+        first, last = ps[0][4], ps[0][5]
+        assert [p[0] for p in ps] == list(range(first, last + 1))
+        if len(ps) > 1:
+            for j, p in enumerate(ps):
+                # the slot the reducer computes for piece j is the one the piece wrote
+                c = first + j
+                assert p[3] == 2 * c + (0 if start(c) // U == t else 1)
+                assert p[3] not in used
+                used.add(p[3])
 
 
 def test_plan_rejects_bad_tuning():

@@ -62,6 +62,18 @@ def test_split_k_each_granularity_and_layout(gran, layout):
         full_parity(p, tuning={"variant": v, "bnq": bnq, "splits": 5}, what=f"{layout} g={gran} {v}")
 
 
+@pytest.mark.parametrize("gran", [64, 128, 256])
+@pytest.mark.parametrize("layout", ["nt", "tn"])
+@pytest.mark.parametrize("M,N,K", [(2048, 1536, 1040), (96, 2048, 3072)])
+def test_stream_k(gran, layout, M, N, K):
+    """Stream-K forced: whole tiles plus shared-out K ranges, pieces summed in K order."""
+    p = workloads.make_problem(M, N, K, gran, layout, seed=gran + M)
+    plan = bsg.make_plan(M, N, K, gran, layout, torch.cuda.get_device_properties(0).multi_processor_count,
+                         {"stream_k": 1})
+    assert plan["sk_ctas"] > 0
+    full_parity(p, tuning={"stream_k": 1}, what=f"stream-K {layout} {M}x{N}x{K} g={gran}")
+
+
 # ---------------------------------------------------------------- small M (decode-style)
 @pytest.mark.parametrize("M", [1, 8, 32, 64, 128])
 def test_small_m_reduced_k(M):
@@ -87,7 +99,8 @@ def _integer_problem(M, N, K, gran, layout, seed):
 
 @pytest.mark.parametrize("layout", ["nt", "tn", "nn", "tt"])
 @pytest.mark.parametrize("tuning", [None, {"variant": "swap_ab", "bnq": 32, "splits": 2},
-                                    {"variant": "data_parallel", "bnq": 256, "splits": 3}])
+                                    {"variant": "data_parallel", "bnq": 256, "splits": 3},
+                                    {"variant": "data_parallel", "bnq": 128, "stream_k": 1}])
 def test_integer_exact_bit_for_bit(layout, tuning):
     p = _integer_problem(272, 304, 1024, 128, layout, seed=5)
     ref, want = oracle.bsgemm(p.layout, p.a, p.b, p.sa, p.sb, p.M, p.N, p.K, p.gran)
@@ -126,7 +139,8 @@ def test_layouts_agree_bit_for_bit():
         assert torch.equal(o, outs[0])
 
 
-@pytest.mark.parametrize("tuning", [None, {"variant": "swap_ab", "bnq": 16, "splits": 6}])
+@pytest.mark.parametrize("tuning", [None, {"variant": "swap_ab", "bnq": 16, "splits": 6},
+                                    {"variant": "data_parallel", "bnq": 128, "stream_k": 1}])
 def test_deterministic_repeats(tuning):
     p = workloads.make_problem(64, 2048, 4096, 128, "nt", seed=11)
     a, b, sa, sb = to_device(p)

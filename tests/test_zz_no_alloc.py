@@ -31,10 +31,13 @@ def _num_sms():
     return torch.cuda.get_device_properties(torch.cuda.current_device()).multi_processor_count
 
 
-def _scratch_bytes(plan):
-    if plan["splits"] <= 1:
-        return 0
-    return plan["tiles_p"] * plan["tiles_q"] * plan["splits"] * plan["bnq"] * 128 * 4
+def _fixed_plan(M, N, K, g):
+    """The plan the allocation-free entry point takes: the regular one when its
+    scratch fits the fixed array, otherwise the one without stream-K."""
+    plan = bsg.make_plan(M, N, K, g, "nt", _num_sms())
+    if bsg.scratch_bytes(plan) > LIMIT_BYTES:
+        plan = bsg.make_plan(M, N, K, g, "nt", _num_sms(), {"stream_k": -1})
+    return plan
 
 
 def _call(fn, a, b, sa, sb, out, M, N, K, g):
@@ -44,8 +47,8 @@ def _call(fn, a, b, sa, sb, out, M, N, K, g):
 
 @pytest.mark.parametrize("M,N,K,g", [(8, 7168, 7168, 128), (256, 7168, 2048, 128), (100, 1024, 4096, 64)])
 def test_no_alloc_matches_regular_entry_point_twice(M, N, K, g):
-    plan = bsg.make_plan(M, N, K, g, "nt", _num_sms())
-    assert plan["splits"] > 1 and 0 < _scratch_bytes(plan) <= LIMIT_BYTES, plan
+    plan = _fixed_plan(M, N, K, g)
+    assert 0 < bsg.scratch_bytes(plan) <= LIMIT_BYTES, plan   # the plan uses the scratch
     p = workloads.make_problem(M, N, K, g, "nt", seed=31)
     a, b, sa, sb = to_device(p)
     L = bsg.lib()
@@ -62,9 +65,9 @@ def test_no_alloc_matches_regular_entry_point_twice(M, N, K, g):
 
 
 def test_no_alloc_rejects_problems_beyond_its_scratch():
-    # find a problem whose plan needs more split-K scratch than the fixed array holds
+    # find a problem whose plan needs more scratch than the fixed array holds
     M, N, K, g = next((m, n, k, 128) for m, n, k in [(256, 4096, 7168), (256, 2048, 16384), (384, 4096, 8192)]
-                      if _scratch_bytes(bsg.make_plan(m, n, k, 128, "nt", _num_sms())) > LIMIT_BYTES)
+                      if bsg.scratch_bytes(_fixed_plan(m, n, k, 128)) > LIMIT_BYTES)
     a = torch.zeros((M, K), dtype=torch.uint8, device="cuda")
     b = torch.zeros((N, K), dtype=torch.uint8, device="cuda")
     sa = torch.ones((-(-M // g), -(-K // g)), dtype=torch.float32, device="cuda")
