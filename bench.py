@@ -59,7 +59,7 @@ def parse_args(argv=None):
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="target CPU seconds of the oracle sample")
-    ap.add_argument("--variant", default="auto", choices=["auto", "data_parallel", "swap_ab"],
+    ap.add_argument("--variant", default="auto", choices=["auto", "data_parallel", "swap_ab", "cta_pair"],
                     help="override the plan's variant (default: library heuristic)")
     ap.add_argument("--bnq", type=int, default=0, help="override the tile width on the MMA N side")
     ap.add_argument("--splits", type=int, default=0, help="override the K splits per tile")

@@ -22,7 +22,7 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libbsgemm.so")
 
 LAYOUTS = {"nt": 0, "tn": 1, "nn": 2, "tt": 3}
-VARIANTS = {"auto": 0, "data_parallel": 1, "swap_ab": 2}
+VARIANTS = {"auto": 0, "data_parallel": 1, "swap_ab": 2, "cta_pair": 3}
 STATUS = {0: "ok", 1: "invalid argument", 2: "unsupported granularity", 3: "misaligned",
           4: "unsupported device", 5: "CUDA error", 6: "device wait timeout",
           7: "needs more scratch than the allocation-free entry point holds"}
@@ -45,7 +45,8 @@ class Tuning(ctypes.Structure):
 class Plan(ctypes.Structure):
     _fields_ = [(n, ctypes.c_int) for n in ("layout", "gran", "swap_ab", "bnq", "tiles_p", "tiles_q",
                                             "splits", "kb_per_split", "grid", "group_p", "kernels",
-                                            "sk_first_tile", "sk_units_per_tile", "sk_ctas", "sk_units")]
+                                            "sk_first_tile", "sk_units_per_tile", "sk_ctas", "sk_units",
+                                            "cta_pair")]
 
     def as_dict(self):
         return {n: getattr(self, n) for n, _ in self._fields_}

@@ -177,6 +177,29 @@ extern "C" bsgemm_status bsgemm_make_plan(int layout, int64_t M, int64_t N, int6
   const int Kb = static_cast<int>((K + gran - 1) / gran);
   int variant = t ? t->variant : BSGEMM_VARIANT_AUTO;
   if (variant == BSGEMM_VARIANT_AUTO) variant = (M <= 128) ? BSGEMM_VARIANT_SWAP_AB : BSGEMM_VARIANT_DATA_PARALLEL;
+  if (variant == BSGEMM_VARIANT_CTA_PAIR) {
+    // 256 x 256 tiles on CTA pairs, whole tiles walked by persistent pairs
+    if ((t && t->bnq != 0 && t->bnq != 256) || (t && t->splits > 1) || (t && t->stream_k > 0))
+      return BSGEMM_ERR_INVALID_ARG;
+    if (num_sms < 2) return BSGEMM_ERR_INVALID_ARG;
+    pl.cta_pair = 1;
+    pl.bnq = 256;
+    pl.tiles_p = static_cast<int>((M + 255) / 256);
+    pl.tiles_q = static_cast<int>((N + 255) / 256);
+    const int64_t pair_tiles = static_cast<int64_t>(pl.tiles_p) * pl.tiles_q;
+    if (pair_tiles > (1 << 30)) return BSGEMM_ERR_INVALID_ARG;
+    const int64_t pairs = pair_tiles < num_sms / 2 ? pair_tiles : num_sms / 2;
+    pl.grid = static_cast<int>(2 * pairs);
+    pl.splits = 1;
+    pl.kb_per_split = Kb;
+    pl.sk_units_per_tile = (Kb + (gran == 64 ? 1 : 0)) / (gran == 64 ? 2 : 1);
+    pl.group_p = 8;
+    pl.layout = layout;
+    pl.gran = gran;
+    pl.kernels = 1;
+    *plan = pl;
+    return BSGEMM_OK;
+  }
   if (variant != BSGEMM_VARIANT_SWAP_AB && variant != BSGEMM_VARIANT_DATA_PARALLEL) return BSGEMM_ERR_INVALID_ARG;
   pl.swap_ab = (variant == BSGEMM_VARIANT_SWAP_AB);
   const int64_t P = pl.swap_ab ? N : M;

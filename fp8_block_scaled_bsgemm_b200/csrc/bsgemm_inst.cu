@@ -5,6 +5,7 @@
 
 #include "bsgemm_host.h"
 #include "bsgemm_kernel.cuh"
+#include "bsgemm_pair.cuh"
 
 #ifndef BSG_GRAN
 #error "compile with -DBSG_GRAN=64|128|256"
@@ -95,12 +96,79 @@ bsgemm_status launch(const bsgemm_plan& plan, const void* a, const void* b, cons
   return cudaGetLastError() == cudaSuccess ? BSGEMM_OK : BSGEMM_ERR_CUDA;
 }
 
+// 256 x 256 tiles on CTA pairs (cluster of 2); whole tiles only.
+template <int GRAN, bool P_MN, bool Q_MN>
+bsgemm_status launch_pair(const bsgemm_plan& plan, const void* a, const void* b, const float* sa,
+                          const float* sb, void* out, int M, int N, int K, cudaStream_t stream,
+                          const DeviceInfo& dev) {
+  using PC = bsg::PairCfg;
+  auto kern = bsg::bsgemm_pair_kernel<GRAN, P_MN, Q_MN>;
+  CUtensorMap tm_p, tm_q;
+  bool ok = true;
+  if (P_MN) ok &= make_map_2d(&tm_p, a, CU_TENSOR_MAP_DATA_TYPE_UINT8, M, K, M, 128, bsg::BK);
+  else      ok &= make_map_2d(&tm_p, a, CU_TENSOR_MAP_DATA_TYPE_UINT8, K, M, K, bsg::BK, bsg::BM);
+  if (Q_MN) ok &= make_map_2d(&tm_q, b, CU_TENSOR_MAP_DATA_TYPE_UINT8, N, K, N, 128, bsg::BK);
+  else      ok &= make_map_2d(&tm_q, b, CU_TENSOR_MAP_DATA_TYPE_UINT8, K, N, K, bsg::BK, bsg::kPairQRows);
+  if (!ok) return BSGEMM_ERR_CUDA;
+
+  bsg::Params prm{};
+  prm.M = M; prm.N = N; prm.K = K;
+  prm.Kb = (K + GRAN - 1) / GRAN;
+  prm.Pb = (M + GRAN - 1) / GRAN;
+  prm.Qb = (N + GRAN - 1) / GRAN;
+  prm.tiles_p = plan.tiles_p;
+  prm.tiles_q = plan.tiles_q;
+  prm.splits = 1;
+  prm.kb_per_split = prm.Kb;
+  prm.num_work = plan.tiles_p * plan.tiles_q;
+  prm.group_p = plan.group_p;
+  prm.sP = sa;
+  prm.sQ = sb;
+  prm.out = static_cast<__nv_bfloat16*>(out);
+  prm.status = dev.status;
+  prm.timeout_ns = wait_timeout_ns();
+
+  cudaLaunchConfig_t cfg{};
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.blockDim = dim3(bsg::kNumThreads, 1, 1);
+  cfg.dynamicSmemBytes = PC::kSmemBytes;
+  cfg.stream = stream;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+
+  static int max_pairs = 0;  // co-resident CTA pairs, once per instance
+  if (max_pairs == 0) {
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, PC::kSmemBytes) != cudaSuccess)
+      return BSGEMM_ERR_CUDA;
+    // the setmaxnreg split is only safe with exactly the planned launch registers
+    cudaFuncAttributes fa{};
+    if (cudaFuncGetAttributes(&fa, kern) != cudaSuccess || fa.numRegs != bsg::kLaunchRegs)
+      return BSGEMM_ERR_CUDA;
+    cfg.gridDim = dim3(plan.grid, 1, 1);
+    int n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) != cudaSuccess || n < 1) return BSGEMM_ERR_CUDA;
+    max_pairs = n;
+  }
+  // a persistent grid no larger than the pairs that can be resident at once
+  int pairs = plan.grid / 2;
+  if (pairs > max_pairs) pairs = max_pairs;
+  if (pairs < 1) return BSGEMM_ERR_INVALID_ARG;
+  cfg.gridDim = dim3(2 * pairs, 1, 1);
+  if (cudaLaunchKernelEx(&cfg, kern, tm_p, tm_q, prm) != cudaSuccess) return BSGEMM_ERR_CUDA;
+  return cudaGetLastError() == cudaSuccess ? BSGEMM_OK : BSGEMM_ERR_CUDA;
+}
+
 }  // namespace
 
 bsgemm_status BSG_RUN_NAME(BSG_GRAN, BSG_LAYOUT)(const bsgemm_plan& pl, const void* a, const void* b,
                                                  const float* sa, const float* sb, void* out, int M,
                                                  int N, int K, cudaStream_t s, const DeviceInfo& d) {
   constexpr int G = BSG_GRAN;
+  if (pl.cta_pair) return launch_pair<G, kAMn, kBMn>(pl, a, b, sa, sb, out, M, N, K, s, d);
   if (pl.swap_ab) {
     // P = B, Q = A
     switch (pl.bnq) {

@@ -114,13 +114,16 @@ typedef enum {
 typedef enum {
     BSGEMM_VARIANT_AUTO = 0,          /* library heuristic */
     BSGEMM_VARIANT_DATA_PARALLEL = 1, /* 128 rows of A per tile on the MMA M side */
-    BSGEMM_VARIANT_SWAP_AB = 2        /* 128 rows of B per tile on the MMA M side (small M) */
+    BSGEMM_VARIANT_SWAP_AB = 2,       /* 128 rows of B per tile on the MMA M side (small M) */
+    BSGEMM_VARIANT_CTA_PAIR = 3       /* 256 x 256 tiles, each computed by a pair of CTAs
+                                         (tcgen05 cta_group::2); whole tiles only */
 } bsgemm_variant;
 
 /* Optional overrides of the plan; 0 in any field means "choose". */
 typedef struct {
     int variant;  /* bsgemm_variant */
-    int bnq;      /* tile width on the MMA N side: 128/256 (data-parallel), 16..128 (swap-AB) */
+    int bnq;      /* tile width on the MMA N side: 128/256 (data-parallel), 16..128 (swap-AB);
+                     256 for CTA pairs */
     int splits;   /* K splits per output tile (split-K); > 0 turns stream-K off */
     int stream_k; /* 0 choose, 1 use stream-K whenever tiles would leave SMs idle, -1 never */
 } bsgemm_tuning;
@@ -140,6 +143,8 @@ typedef struct {
     int sk_units_per_tile; /* stream-K: units per tile (a unit is one K block; two when gran = 64) */
     int sk_ctas;        /* stream-K: CTAs sharing the remaining tiles' units (0: no stream-K) */
     int sk_units;       /* stream-K: units of all stream-K tiles together */
+    int cta_pair;       /* 1: 256 x 256 tiles on CTA pairs (tiles_p, tiles_q count those;
+                           grid counts CTAs, two per pair) */
 } bsgemm_plan;
 
 /* The operation above with the layout as an argument and optional tuning

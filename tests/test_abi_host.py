@@ -86,6 +86,19 @@ def test_plan_uses_stream_k_for_a_ragged_last_wave():
     assert bsg.make_plan(128 * 148, 256, 1024, 128, "nt", 148, {"stream_k": 1})["sk_ctas"] == 0
 
 
+def test_plan_for_cta_pairs():
+    pl = bsg.make_plan(4096, 4096, 4096, 128, "nt", 148, {"variant": "cta_pair"})
+    assert pl["cta_pair"] == 1 and pl["bnq"] == 256 and pl["splits"] == 1 and pl["sk_ctas"] == 0
+    assert (pl["tiles_p"], pl["tiles_q"]) == (16, 16) and pl["grid"] == 148
+    small = bsg.make_plan(300, 200, 64, 64, "tn", 148, {"variant": "cta_pair"})
+    assert (small["tiles_p"], small["tiles_q"], small["grid"]) == (2, 1, 4)
+    for bad in ({"variant": "cta_pair", "bnq": 128}, {"variant": "cta_pair", "splits": 2},
+                {"variant": "cta_pair", "stream_k": 1}):
+        with pytest.raises(bsg.BsgemmError):
+            bsg.make_plan(4096, 4096, 4096, 128, "nt", 148, bad)
+    assert bsg.make_plan(4096, 4096, 4096, 128, "nt", 148)["cta_pair"] == 0
+
+
 def _sk_partition(tiles_sk, U, G):
     """Mirror of the kernel's stream-K walk (sk_start, sk_owner, piece slots)."""
     R = tiles_sk * U

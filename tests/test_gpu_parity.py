@@ -12,7 +12,7 @@ import oracle
 import workloads
 import fp8_block_scaled_bsgemm_b200 as bsg
 
-from gpu_util import check_close, full_parity, gpu_as_f64, run_gpu, to_device
+from gpu_util import check_close, full_parity, gpu_as_f64, run_gpu, sampled_parity, to_device
 
 pytestmark = pytest.mark.gpu
 
@@ -74,6 +74,36 @@ def test_stream_k(gran, layout, M, N, K):
     full_parity(p, tuning={"stream_k": 1}, what=f"stream-K {layout} {M}x{N}x{K} g={gran}")
 
 
+# ---------------------------------------------------------------- CTA pairs (cta_group::2)
+@pytest.mark.parametrize("gran", [64, 128, 256])
+@pytest.mark.parametrize("layout", ["nt", "tn", "nn", "tt"])
+def test_cta_pair_each_granularity_and_layout(gran, layout):
+    """256 x 256 tiles on CTA pairs; ragged M, N and K tails (odd CTA's rows partly past M)."""
+    p = workloads.make_problem(656, 784, 1008, gran, layout, seed=11 + gran)
+    full_parity(p, tuning={"variant": "cta_pair"}, what=f"pair {layout} g={gran}")
+
+
+@pytest.mark.parametrize("M,N,K", [(2560, 2304, 512), (384, 4096, 2176), (130, 264, 96)])
+def test_cta_pair_shapes(M, N, K):
+    """More pair tiles than resident pairs (several waves), a single row of tiles, tiny."""
+    p = workloads.make_problem(M, N, K, 128, "nt", seed=M)
+    if M * N * K > 1 << 31:
+        sampled_parity(p, count=4000, tuning={"variant": "cta_pair"}, what=f"pair {M}x{N}x{K}")
+    else:
+        full_parity(p, tuning={"variant": "cta_pair"}, what=f"pair {M}x{N}x{K}")
+
+
+def test_cta_pair_agrees_with_single_cta():
+    """Same K-block order and promotion arithmetic; the tensor core's FP32 sums
+    inside a K-block round differently between the pair and the single-CTA
+    instruction shapes (measured: up to 3 BF16 ulps on near-cancelling
+    elements), so the two agree to the parity tolerance, not bit for bit."""
+    p = workloads.make_problem(1024, 1280, 1536, 128, "nt", seed=5)
+    one = gpu_as_f64(run_gpu(p, tuning={"variant": "data_parallel", "bnq": 256, "stream_k": -1}))
+    two = gpu_as_f64(run_gpu(p, tuning={"variant": "cta_pair"}))
+    check_close(two, one, "pair vs single CTA")
+
+
 # ---------------------------------------------------------------- small M (decode-style)
 @pytest.mark.parametrize("M", [1, 8, 32, 64, 128])
 def test_small_m_reduced_k(M):
@@ -100,7 +130,8 @@ def _integer_problem(M, N, K, gran, layout, seed):
 @pytest.mark.parametrize("layout", ["nt", "tn", "nn", "tt"])
 @pytest.mark.parametrize("tuning", [None, {"variant": "swap_ab", "bnq": 32, "splits": 2},
                                     {"variant": "data_parallel", "bnq": 256, "splits": 3},
-                                    {"variant": "data_parallel", "bnq": 128, "stream_k": 1}])
+                                    {"variant": "data_parallel", "bnq": 128, "stream_k": 1},
+                                    {"variant": "cta_pair"}])
 def test_integer_exact_bit_for_bit(layout, tuning):
     p = _integer_problem(272, 304, 1024, 128, layout, seed=5)
     ref, want = oracle.bsgemm(p.layout, p.a, p.b, p.sa, p.sb, p.M, p.N, p.K, p.gran)
@@ -140,7 +171,8 @@ def test_layouts_agree_bit_for_bit():
 
 
 @pytest.mark.parametrize("tuning", [None, {"variant": "swap_ab", "bnq": 16, "splits": 6},
-                                    {"variant": "data_parallel", "bnq": 128, "stream_k": 1}])
+                                    {"variant": "data_parallel", "bnq": 128, "stream_k": 1},
+                                    {"variant": "cta_pair"}])
 def test_deterministic_repeats(tuning):
     p = workloads.make_problem(64, 2048, 4096, 128, "nt", seed=11)
     a, b, sa, sb = to_device(p)
