@@ -22,6 +22,7 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libbsgemm.so")
 
 LAYOUTS = {"nt": 0, "tn": 1, "nn": 2, "tt": 3}
+FORMATS = {"e4m3": 0, "e5m2": 1}
 VARIANTS = {"auto": 0, "data_parallel": 1, "swap_ab": 2, "cta_pair": 3}
 STATUS = {0: "ok", 1: "invalid argument", 2: "unsupported granularity", 3: "misaligned",
           4: "unsupported device", 5: "CUDA error", 6: "device wait timeout",
@@ -53,9 +54,10 @@ class Plan(ctypes.Structure):
 
 
 EXPORTS = ("bsgemm_fp8_nt", "bsgemm_fp8_tn", "bsgemm_fp8_nn", "bsgemm_fp8_tt", "bsgemm_fp8_gemm_ex",
+           "bsgemm_fp8_gemm_fmt",
            "bsgemm_make_plan", "bsgemm_status_string", "bsgemm_get_last_device_status",
            "bsgemm_last_device_status_detail", "bsgemm_diag_wait_timeout", "bsgemm_version",
-           "bsgemm_fp8_nt_noalloc")
+           "bsgemm_fp8_nt_noalloc", "bsgemm_quantize_fp8")
 
 
 def lib():
@@ -70,12 +72,15 @@ def lib():
             p, i64, i32 = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int
             gemm_args = [p, p, p, p, p, i64, i64, i64, i32, p]
             for name in ("bsgemm_fp8_nt", "bsgemm_fp8_tn", "bsgemm_fp8_nn", "bsgemm_fp8_tt",
-                         "bsgemm_fp8_nt_noalloc"):
+                         "bsgemm_fp8_nt_noalloc", "bsgemm_quantize_fp8"):
                 getattr(L, name).argtypes = gemm_args
                 getattr(L, name).restype = i32
             L.bsgemm_fp8_gemm_ex.argtypes = [i32, p, p, p, p, p, i64, i64, i64, i32,
                                              ctypes.POINTER(Tuning), p]
             L.bsgemm_fp8_gemm_ex.restype = i32
+            L.bsgemm_fp8_gemm_fmt.argtypes = [i32, i32, i32, p, p, p, p, p, i64, i64, i64, i32,
+                                              ctypes.POINTER(Tuning), p]
+            L.bsgemm_fp8_gemm_fmt.restype = i32
             L.bsgemm_make_plan.argtypes = [i32, i64, i64, i64, i32, i32, ctypes.POINTER(Tuning),
                                            ctypes.POINTER(Plan)]
             L.bsgemm_make_plan.restype = i32
@@ -87,6 +92,8 @@ def lib():
             L.bsgemm_last_device_status_detail.restype = i32
             L.bsgemm_diag_wait_timeout.argtypes = [ctypes.c_ulonglong, p]
             L.bsgemm_diag_wait_timeout.restype = i32
+            L.bsgemm_quantize_fp8.argtypes = [i32, i32, p, i64, i64, i32, p, p, p]
+            L.bsgemm_quantize_fp8.restype = i32
             L.bsgemm_version.argtypes = []
             L.bsgemm_version.restype = i32
             _lib = L
@@ -114,8 +121,8 @@ def _tuning(tuning):
 
 
 def _as_bytes(x: torch.Tensor, name: str) -> torch.Tensor:
-    if x.dtype not in (torch.float8_e4m3fn, torch.uint8):
-        raise TypeError(f"{name} must be float8_e4m3fn or uint8 codes, got {x.dtype}")
+    if x.dtype not in (torch.float8_e4m3fn, torch.float8_e5m2, torch.uint8):
+        raise TypeError(f"{name} must be float8_e4m3fn, float8_e5m2 or uint8 codes, got {x.dtype}")
     if not x.is_cuda or not x.is_contiguous():
         raise ValueError(f"{name} must be a contiguous CUDA tensor")
     return x
@@ -132,10 +139,27 @@ def shapes(layout: str, a: torch.Tensor, b: torch.Tensor):
     return int(M), int(N), int(Ka)
 
 
-def gemm(a, b, scale_a, scale_b, out=None, layout="nt", gran=128, tuning=None, stream=None):
-    """out[M,N] (BF16) of the block-scaled FP8 GEMM; see ``include/bsgemm.h``."""
+def _format(x: torch.Tensor, given, name: str) -> int:
+    """FP8 format of an operand: from its dtype, or ``given`` for uint8 codes."""
+    from_dtype = {torch.float8_e4m3fn: "e4m3", torch.float8_e5m2: "e5m2"}.get(x.dtype)
+    fmt = given if given is not None else (from_dtype or "e4m3")
+    if fmt not in FORMATS:
+        raise ValueError(f"{name}: format must be one of {sorted(FORMATS)}")
+    if from_dtype is not None and fmt != from_dtype:
+        raise ValueError(f"{name}: dtype {x.dtype} does not match format {fmt}")
+    return FORMATS[fmt]
+
+
+def gemm(a, b, scale_a, scale_b, out=None, layout="nt", gran=128, tuning=None, stream=None,
+         a_format=None, b_format=None):
+    """out[M,N] (BF16) of the block-scaled FP8 GEMM; see ``include/bsgemm.h``.
+
+    ``a_format`` / ``b_format``: "e4m3" or "e5m2"; taken from the tensor's
+    dtype when it is a float8 type, E4M3 for uint8 codes unless given."""
     if layout not in LAYOUTS:
         raise ValueError(f"layout must be one of {sorted(LAYOUTS)}")
+    fa = _format(a, a_format, "a")
+    fb = _format(b, b_format, "b")
     a = _as_bytes(a, "a")
     b = _as_bytes(b, "b")
     M, N, K = shapes(layout, a, b)
@@ -146,9 +170,9 @@ def gemm(a, b, scale_a, scale_b, out=None, layout="nt", gran=128, tuning=None, s
         out = torch.empty((M, N), dtype=torch.bfloat16, device=a.device)
     if out.dtype != torch.bfloat16 or tuple(out.shape) != (M, N) or not out.is_contiguous():
         raise ValueError("out must be a contiguous bfloat16 [M, N] tensor")
-    st = lib().bsgemm_fp8_gemm_ex(LAYOUTS[layout], a.data_ptr(), b.data_ptr(), scale_a.data_ptr(),
-                                  scale_b.data_ptr(), out.data_ptr(), M, N, K, int(gran),
-                                  _tuning(tuning), _stream_handle(stream))
+    st = lib().bsgemm_fp8_gemm_fmt(LAYOUTS[layout], fa, fb, a.data_ptr(), b.data_ptr(),
+                                   scale_a.data_ptr(), scale_b.data_ptr(), out.data_ptr(), M, N, K,
+                                   int(gran), _tuning(tuning), _stream_handle(stream))
     if st != 0:
         raise BsgemmError(st, f"bsgemm {layout} M={M} N={N} K={K} g={gran}")
     return out
@@ -168,6 +192,30 @@ def bsgemm_fp8_nn(a, b, scale_a, scale_b, out=None, gran=128, stream=None):
 
 def bsgemm_fp8_tt(a, b, scale_a, scale_b, out=None, gran=128, stream=None):
     return gemm(a, b, scale_a, scale_b, out, "tt", gran, None, stream)
+
+
+def quantize(x: torch.Tensor, gran: int = 128, fmt: str = "e4m3", q=None, scales=None, stream=None):
+    """Per-block FP8 quantisation of a row-major FP32/BF16 CUDA matrix [rows, cols].
+
+    Returns (q uint8 [rows, cols], scales float32 [ceil(rows/g), ceil(cols/g)]):
+    the GEMM's operand and scale tensors. See ``bsgemm_quantize_fp8``."""
+    if x.dim() != 2 or not x.is_cuda or not x.is_contiguous():
+        raise ValueError("x must be a contiguous 2-D CUDA tensor")
+    src = {torch.float32: 0, torch.bfloat16: 1}.get(x.dtype)
+    if src is None:
+        raise TypeError(f"x must be float32 or bfloat16, got {x.dtype}")
+    if fmt not in FORMATS:
+        raise ValueError(f"fmt must be one of {sorted(FORMATS)}")
+    rows, cols = x.shape
+    if q is None:
+        q = torch.empty((rows, cols), dtype=torch.uint8, device=x.device)
+    if scales is None:
+        scales = torch.empty((-(-rows // gran), -(-cols // gran)), dtype=torch.float32, device=x.device)
+    st = lib().bsgemm_quantize_fp8(src, FORMATS[fmt], x.data_ptr(), rows, cols, int(gran), q.data_ptr(),
+                                   scales.data_ptr(), _stream_handle(stream))
+    if st != 0:
+        raise BsgemmError(st, f"bsgemm_quantize_fp8 {rows}x{cols} g={gran}")
+    return q, scales
 
 
 def scratch_bytes(plan: dict) -> int:

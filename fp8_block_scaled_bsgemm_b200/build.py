@@ -1,6 +1,8 @@
 """Build ``libbsgemm.so`` in-tree for sm_100a with nvcc.
 
-The C ABI unit (``csrc/bsgemm_api.cu``) and one kernel-instance unit per
+The C ABI unit (``csrc/bsgemm_api.cu``), the allocation-free entry point
+(``csrc/bsgemm_noalloc.cu``), the quantiser (``csrc/bsgemm_quant.cu``) and
+one kernel-instance unit per
 (granularity, layout) pair (``csrc/bsgemm_inst.cu`` compiled twelve times with
 -DBSG_GRAN / -DBSG_LAYOUT) are compiled in parallel and linked into one shared
 library next to this file.  Objects are rebuilt only when a source under
@@ -61,7 +63,8 @@ def build(force: bool = False, jobs: int | None = None, verbose: bool = False) -
     os.makedirs(BUILD, exist_ok=True)
     newest = _newest_source()
     units = [(os.path.join(CSRC, "bsgemm_api.cu"), os.path.join(BUILD, "bsgemm_api.o"), []),
-             (os.path.join(CSRC, "bsgemm_noalloc.cu"), os.path.join(BUILD, "bsgemm_noalloc.o"), [])]
+             (os.path.join(CSRC, "bsgemm_noalloc.cu"), os.path.join(BUILD, "bsgemm_noalloc.o"), []),
+             (os.path.join(CSRC, "bsgemm_quant.cu"), os.path.join(BUILD, "bsgemm_quant.o"), [])]
     for g in GRANS:
         for lay in LAYOUTS:
             units.append((os.path.join(CSRC, "bsgemm_inst.cu"),

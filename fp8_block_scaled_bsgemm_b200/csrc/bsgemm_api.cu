@@ -290,10 +290,13 @@ extern "C" bsgemm_status bsgemm_make_plan(int layout, int64_t M, int64_t N, int6
 }
 
 // ------------------------------------------------------------------ entry points
-extern "C" bsgemm_status bsgemm_fp8_gemm_ex(int layout, const void* a, const void* b,
-                                            const float* scale_a, const float* scale_b, void* out,
-                                            int64_t M, int64_t N, int64_t K, int gran,
-                                            const bsgemm_tuning* tuning, bsgemm_stream_t stream) {
+extern "C" bsgemm_status bsgemm_fp8_gemm_fmt(int layout, int a_format, int b_format, const void* a,
+                                             const void* b, const float* scale_a, const float* scale_b,
+                                             void* out, int64_t M, int64_t N, int64_t K, int gran,
+                                             const bsgemm_tuning* tuning, bsgemm_stream_t stream) {
+  if ((a_format != BSGEMM_FP8_E4M3 && a_format != BSGEMM_FP8_E5M2) ||
+      (b_format != BSGEMM_FP8_E4M3 && b_format != BSGEMM_FP8_E5M2))
+    return BSGEMM_ERR_INVALID_ARG;
   bsgemm_status st = check_args(layout, a, b, scale_a, scale_b, out, M, N, K, gran);
   if (st != BSGEMM_OK) return st;
   DeviceInfo dev;
@@ -304,7 +307,8 @@ extern "C" bsgemm_status bsgemm_fp8_gemm_ex(int layout, const void* a, const voi
   if (st != BSGEMM_OK) return st;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const int m = static_cast<int>(M), n = static_cast<int>(N), k = static_cast<int>(K);
-#define BSG_RUN(G, L) bsg_host::run_g##G##_##L(pl, a, b, scale_a, scale_b, out, m, n, k, s, dev)
+#define BSG_RUN(G, L) \
+  bsg_host::run_g##G##_##L(pl, a, b, scale_a, scale_b, out, m, n, k, a_format, b_format, s, dev)
 #define BSG_RUN_LAYOUTS(G)                              \
   switch (layout) {                                     \
     case BSGEMM_LAYOUT_NT: return BSG_RUN(G, nt);       \
@@ -319,6 +323,14 @@ extern "C" bsgemm_status bsgemm_fp8_gemm_ex(int layout, const void* a, const voi
   }
 #undef BSG_RUN_LAYOUTS
 #undef BSG_RUN
+}
+
+extern "C" bsgemm_status bsgemm_fp8_gemm_ex(int layout, const void* a, const void* b,
+                                            const float* scale_a, const float* scale_b, void* out,
+                                            int64_t M, int64_t N, int64_t K, int gran,
+                                            const bsgemm_tuning* tuning, bsgemm_stream_t stream) {
+  return bsgemm_fp8_gemm_fmt(layout, BSGEMM_FP8_E4M3, BSGEMM_FP8_E4M3, a, b, scale_a, scale_b, out,
+                             M, N, K, gran, tuning, stream);
 }
 
 extern "C" bsgemm_status bsgemm_fp8_nt(const void* a, const void* b, const float* sa, const float* sb,

@@ -39,10 +39,11 @@ unsigned long long wait_timeout_ns();
 // call; allocates nothing).
 bsgemm_status device_status_address(int** out);
 
+// a_fmt, b_fmt: bsgemm_fp8_format of the logical A and B operands.
 #define BSG_RUN_DECL(G, L)                                                                       \
   bsgemm_status run_g##G##_##L(const bsgemm_plan& plan, const void* a, const void* b,          \
                                const float* sa, const float* sb, void* out, int M, int N, int K, \
-                               cudaStream_t stream, const DeviceInfo& dev);
+                               int a_fmt, int b_fmt, cudaStream_t stream, const DeviceInfo& dev);
 BSG_RUN_DECL(64, nt) BSG_RUN_DECL(64, tn) BSG_RUN_DECL(64, nn) BSG_RUN_DECL(64, tt)
 BSG_RUN_DECL(128, nt) BSG_RUN_DECL(128, tn) BSG_RUN_DECL(128, nn) BSG_RUN_DECL(128, tt)
 BSG_RUN_DECL(256, nt) BSG_RUN_DECL(256, tn) BSG_RUN_DECL(256, nn) BSG_RUN_DECL(256, tt)

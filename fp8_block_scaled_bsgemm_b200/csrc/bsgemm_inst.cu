@@ -27,10 +27,16 @@ constexpr const char* kLayout = BSG_STR(BSG_LAYOUT);
 constexpr bool kAMn = kLayout[0] == 't';
 constexpr bool kBMn = kLayout[1] == 'n';
 
+// Format fields of the instruction descriptor for operands P (MMA A side)
+// and Q (MMA B side).
+inline uint32_t fmt_bits(int p_fmt, int q_fmt) {
+  return (static_cast<uint32_t>(p_fmt) << 7) | (static_cast<uint32_t>(q_fmt) << 10);
+}
+
 template <int BNQ, int GRAN, bool SWAP, bool P_MN, bool Q_MN, bool SPLIT>
 bsgemm_status launch(const bsgemm_plan& plan, const void* a, const void* b, const float* sa,
-                     const float* sb, void* out, int M, int N, int K, cudaStream_t stream,
-                     const DeviceInfo& dev) {
+                     const float* sb, void* out, int M, int N, int K, int a_fmt, int b_fmt,
+                     cudaStream_t stream, const DeviceInfo& dev) {
   using SC = bsg::StageCfg<BNQ, Q_MN, SWAP>;
   auto kern = bsg::bsgemm_kernel<BNQ, GRAN, SWAP, P_MN, Q_MN, SPLIT>;
 
@@ -64,6 +70,7 @@ bsgemm_status launch(const bsgemm_plan& plan, const void* a, const void* b, cons
   prm.sk_q = plan.sk_ctas > 0 ? plan.sk_units / plan.sk_ctas : 0;
   prm.sk_r = plan.sk_ctas > 0 ? plan.sk_units % plan.sk_ctas : 0;
   prm.group_p = plan.group_p;
+  prm.fmt_bits = SWAP ? fmt_bits(b_fmt, a_fmt) : fmt_bits(a_fmt, b_fmt);
   prm.sP = SWAP ? sb : sa;
   prm.sQ = SWAP ? sa : sb;
   prm.out = static_cast<__nv_bfloat16*>(out);
@@ -99,8 +106,8 @@ bsgemm_status launch(const bsgemm_plan& plan, const void* a, const void* b, cons
 // 256 x 256 tiles on CTA pairs (cluster of 2); whole tiles only.
 template <int GRAN, bool P_MN, bool Q_MN>
 bsgemm_status launch_pair(const bsgemm_plan& plan, const void* a, const void* b, const float* sa,
-                          const float* sb, void* out, int M, int N, int K, cudaStream_t stream,
-                          const DeviceInfo& dev) {
+                          const float* sb, void* out, int M, int N, int K, int a_fmt, int b_fmt,
+                          cudaStream_t stream, const DeviceInfo& dev) {
   using PC = bsg::PairCfg;
   auto kern = bsg::bsgemm_pair_kernel<GRAN, P_MN, Q_MN>;
   CUtensorMap tm_p, tm_q;
@@ -122,6 +129,7 @@ bsgemm_status launch_pair(const bsgemm_plan& plan, const void* a, const void* b,
   prm.kb_per_split = prm.Kb;
   prm.num_work = plan.tiles_p * plan.tiles_q;
   prm.group_p = plan.group_p;
+  prm.fmt_bits = fmt_bits(a_fmt, b_fmt);
   prm.sP = sa;
   prm.sQ = sb;
   prm.out = static_cast<__nv_bfloat16*>(out);
@@ -166,27 +174,28 @@ bsgemm_status launch_pair(const bsgemm_plan& plan, const void* a, const void* b,
 
 bsgemm_status BSG_RUN_NAME(BSG_GRAN, BSG_LAYOUT)(const bsgemm_plan& pl, const void* a, const void* b,
                                                  const float* sa, const float* sb, void* out, int M,
-                                                 int N, int K, cudaStream_t s, const DeviceInfo& d) {
+                                                 int N, int K, int fa, int fb, cudaStream_t s,
+                                                 const DeviceInfo& d) {
   constexpr int G = BSG_GRAN;
-  if (pl.cta_pair) return launch_pair<G, kAMn, kBMn>(pl, a, b, sa, sb, out, M, N, K, s, d);
+  if (pl.cta_pair) return launch_pair<G, kAMn, kBMn>(pl, a, b, sa, sb, out, M, N, K, fa, fb, s, d);
   if (pl.swap_ab) {
     // P = B, Q = A
     switch (pl.bnq) {
-      case 16:  return launch<16, G, true, kBMn, kAMn, true>(pl, a, b, sa, sb, out, M, N, K, s, d);
-      case 32:  return launch<32, G, true, kBMn, kAMn, true>(pl, a, b, sa, sb, out, M, N, K, s, d);
-      case 64:  return launch<64, G, true, kBMn, kAMn, true>(pl, a, b, sa, sb, out, M, N, K, s, d);
-      case 128: return launch<128, G, true, kBMn, kAMn, true>(pl, a, b, sa, sb, out, M, N, K, s, d);
+      case 16:  return launch<16, G, true, kBMn, kAMn, true>(pl, a, b, sa, sb, out, M, N, K, fa, fb, s, d);
+      case 32:  return launch<32, G, true, kBMn, kAMn, true>(pl, a, b, sa, sb, out, M, N, K, fa, fb, s, d);
+      case 64:  return launch<64, G, true, kBMn, kAMn, true>(pl, a, b, sa, sb, out, M, N, K, fa, fb, s, d);
+      case 128: return launch<128, G, true, kBMn, kAMn, true>(pl, a, b, sa, sb, out, M, N, K, fa, fb, s, d);
       default:  return BSGEMM_ERR_INVALID_ARG;
     }
   }
   const bool split = pl.splits > 1 || pl.sk_ctas > 0;
   switch (pl.bnq) {
     case 128:
-      return split ? launch<128, G, false, kAMn, kBMn, true>(pl, a, b, sa, sb, out, M, N, K, s, d)
-                   : launch<128, G, false, kAMn, kBMn, false>(pl, a, b, sa, sb, out, M, N, K, s, d);
+      return split ? launch<128, G, false, kAMn, kBMn, true>(pl, a, b, sa, sb, out, M, N, K, fa, fb, s, d)
+                   : launch<128, G, false, kAMn, kBMn, false>(pl, a, b, sa, sb, out, M, N, K, fa, fb, s, d);
     case 256:
-      return split ? launch<256, G, false, kAMn, kBMn, true>(pl, a, b, sa, sb, out, M, N, K, s, d)
-                   : launch<256, G, false, kAMn, kBMn, false>(pl, a, b, sa, sb, out, M, N, K, s, d);
+      return split ? launch<256, G, false, kAMn, kBMn, true>(pl, a, b, sa, sb, out, M, N, K, fa, fb, s, d)
+                   : launch<256, G, false, kAMn, kBMn, false>(pl, a, b, sa, sb, out, M, N, K, fa, fb, s, d);
     default:
       return BSGEMM_ERR_INVALID_ARG;
   }

@@ -87,6 +87,7 @@ struct Params {
   int sk_q, sk_r;        // stream-K: the stream-K units number sk_q * sk_ctas + sk_r; the first
                          // sk_r CTAs take sk_q + 1 of them, the others sk_q
   int group_p;           // raster group height in P tiles (L2 locality)
+  uint32_t fmt_bits;     // instruction-descriptor format fields of P and Q (E4M3 0, E5M2 1)
   const float* sP;       // [Pb][Kb]
   const float* sQ;       // [Qb][Kb]
   __nv_bfloat16* out;    // [M][N] row-major (direct stores in swap mode)
@@ -185,11 +186,12 @@ __device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t addr, uint32_t lbo)
   return d;
 }
 
-// Instruction descriptor: kind::f8f6f4, A = B = E4M3, D = F32, M = 128, N = BNQ.
+// Instruction descriptor: kind::f8f6f4, D = F32, M = 128, N = BNQ; the A and B
+// format fields (bits 7-9, 10-12: E4M3 0, E5M2 1) come from Params.fmt_bits.
 template <int BNQ, bool P_MN, bool Q_MN>
 __device__ __forceinline__ constexpr uint32_t instr_desc() {
   return (1u << 4)                               // D format: F32
-         | (0u << 7) | (0u << 10)                // A, B format: E4M3
+         | (0u << 7) | (0u << 10)                // A, B format: or-ed in at run time
          | ((P_MN ? 1u : 0u) << 15)              // A major (0 = K)
          | ((Q_MN ? 1u : 0u) << 16)              // B major
          | (static_cast<uint32_t>(BNQ >> 3) << 17)
@@ -450,7 +452,7 @@ __global__ void __launch_bounds__(kNumThreads, 1)
     // converged warp that branches per MMA and a converged warp whose lanes
     // all wait (one lane issuing) are slower.
     if (lane == 0) {
-      constexpr uint32_t idesc = instr_desc<BNQ, P_MN, Q_MN>();
+      const uint32_t idesc = instr_desc<BNQ, P_MN, Q_MN>() | p.fmt_bits;
       // descriptor steps: per k-step of 32 (K-major +32 B, MN-major +32 rows
       // of 128 B) and per pipeline stage, in the descriptor's 16-byte units
       constexpr uint64_t kPStep = P_MN ? (kMmaK * 128) >> 4 : kMmaK >> 4;

@@ -45,7 +45,7 @@ struct PairCfg {
 template <bool P_MN, bool Q_MN>
 __device__ __forceinline__ constexpr uint32_t instr_desc_pair() {
   return (1u << 4)                                        // D format: F32
-         | (0u << 7) | (0u << 10)                         // A, B format: E4M3
+         | (0u << 7) | (0u << 10)                         // A, B format: or-ed in at run time
          | ((P_MN ? 1u : 0u) << 15) | ((Q_MN ? 1u : 0u) << 16)
          | (static_cast<uint32_t>(kPairN >> 3) << 17)
          | (static_cast<uint32_t>(kPairM >> 4) << 24);
@@ -156,7 +156,7 @@ __global__ void __launch_bounds__(kNumThreads, 1)
   } else if (warp == kMmaWarp) {
     // ============================================================ MMA issuer (even CTA)
     if (rank == 0 && lane == 0) {
-      constexpr uint32_t idesc = instr_desc_pair<P_MN, Q_MN>();
+      const uint32_t idesc = instr_desc_pair<P_MN, Q_MN>() | p.fmt_bits;
       constexpr uint64_t kPStep = P_MN ? (kMmaK * 128) >> 4 : kMmaK >> 4;
       constexpr uint64_t kQStep = Q_MN ? (kMmaK * 128) >> 4 : kMmaK >> 4;
       constexpr uint64_t kPStage = PC::kPBytes >> 4, kQStage = PC::kQBytes >> 4;

@@ -1,0 +1,161 @@
+// Per-block FP8 quantiser: the step the pages put in front of the GEMM
+// (hncyxsy.com/news/191052 §4.4: the quantisation granularity must match the
+// GEMM's; §5.2: quantisation divides by the scale, dequantisation multiplies).
+//
+// For each g x g block of a row-major [rows, cols] FP32 or BF16 matrix:
+//   amax = max |x| over the block's elements;
+//   s    = amax / FMAX in FP32, correctly rounded (FMAX = 448 for E4M3,
+//          57344 for E5M2), or 1 when amax is 0;
+//   q    = FP8 code of x / s (FP32 division, correctly rounded), rounded to
+//          nearest with ties to even and saturated to +-FMAX.
+// The codes go to q [rows, cols] (row-major, one byte each) and the scales
+// to scales [ceil(rows/g), ceil(cols/g)] (row-major FP32): exactly the
+// operand and scale tensors the GEMM takes.
+//
+// One CTA of 256 threads per block. The block is read twice (amax, then
+// encode); the second read comes from L2. Each thread handles runs of 8
+// consecutive columns: 32-byte (FP32) or 16-byte (BF16) loads, 8-byte stores
+// of 8 codes. This is HBM-bound work: no tensor cores.
+#include <cuda_bf16.h>
+#include <cuda_fp8.h>
+#include <cuda_runtime.h>
+
+#include <cstdint>
+
+#include "bsgemm.h"
+
+namespace bsgq {
+
+constexpr int kThreads = 256;
+constexpr int kVec = 8;  // columns per run
+
+template <bool BF16_IN>
+__device__ __forceinline__ void load8(const void* x, int64_t off, float (&v)[kVec]) {
+  if constexpr (BF16_IN) {
+    const uint4 u = __ldg(reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(x) + off));
+    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      v[2 * i] = __uint_as_float(w[i] << 16);
+      v[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
+    }
+  } else {
+    const float4* p = reinterpret_cast<const float4*>(static_cast<const float*>(x) + off);
+    const float4 a = __ldg(p), b = __ldg(p + 1);
+    v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
+    v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+  }
+}
+
+template <int FMT>
+__device__ __forceinline__ uint32_t encode(float v) {
+  // round to nearest even, saturating to the largest finite value
+  return static_cast<uint32_t>(
+      __nv_cvt_float_to_fp8(v, __NV_SATFINITE, FMT == BSGEMM_FP8_E5M2 ? __NV_E5M2 : __NV_E4M3));
+}
+
+template <int G, bool BF16_IN, int FMT>
+__global__ void __launch_bounds__(kThreads)
+    quant_kernel(const void* __restrict__ x, int64_t rows, int64_t cols, int64_t col_blocks,
+                 uint8_t* __restrict__ q, float* __restrict__ scales) {
+  constexpr int kRuns = G * G / kVec;   // runs of 8 columns in a full block
+  constexpr int kRunsPerRow = G / kVec;
+  constexpr float kFmax = FMT == BSGEMM_FP8_E5M2 ? 57344.0f : 448.0f;
+  __shared__ float warp_max[kThreads / 32];
+  __shared__ float block_scale;
+
+  const int64_t blk = blockIdx.x;
+  const int64_t r0 = (blk / col_blocks) * G;
+  const int64_t c0 = (blk % col_blocks) * G;
+
+  // ---- pass 1: amax over the block (elements outside the matrix are skipped)
+  float amax = 0.f;
+  for (int run = threadIdx.x; run < kRuns; run += kThreads) {
+    const int64_t r = r0 + run / kRunsPerRow;
+    const int64_t c = c0 + (run % kRunsPerRow) * kVec;
+    if (r < rows && c < cols) {  // cols % 8 == 0: a run is wholly in or out
+      float v[kVec];
+      load8<BF16_IN>(x, r * cols + c, v);
+#pragma unroll
+      for (int i = 0; i < kVec; ++i) amax = fmaxf(amax, fabsf(v[i]));
+    }
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+  if ((threadIdx.x & 31) == 0) warp_max[threadIdx.x >> 5] = amax;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    float m = warp_max[0];
+#pragma unroll
+    for (int w = 1; w < kThreads / 32; ++w) m = fmaxf(m, warp_max[w]);
+    const float s = m > 0.f ? __fdiv_rn(m, kFmax) : 1.0f;
+    block_scale = s;
+    scales[blk] = s;
+  }
+  __syncthreads();
+  const float s = block_scale;
+
+  // ---- pass 2: encode
+  for (int run = threadIdx.x; run < kRuns; run += kThreads) {
+    const int64_t r = r0 + run / kRunsPerRow;
+    const int64_t c = c0 + (run % kRunsPerRow) * kVec;
+    if (r < rows && c < cols) {
+      float v[kVec];
+      load8<BF16_IN>(x, r * cols + c, v);
+      uint32_t lo = 0, hi = 0;
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        lo |= encode<FMT>(__fdiv_rn(v[i], s)) << (8 * i);
+        hi |= encode<FMT>(__fdiv_rn(v[4 + i], s)) << (8 * i);
+      }
+      *reinterpret_cast<uint2*>(q + r * cols + c) = make_uint2(lo, hi);
+    }
+  }
+}
+
+template <int G, bool BF16_IN, int FMT>
+bsgemm_status launch(const void* x, int64_t rows, int64_t cols, uint8_t* q, float* scales,
+                     cudaStream_t stream) {
+  const int64_t rb = (rows + G - 1) / G, cb = (cols + G - 1) / G;
+  const int64_t blocks = rb * cb;
+  if (blocks > 0x7FFFFFFFll) return BSGEMM_ERR_INVALID_ARG;
+  quant_kernel<G, BF16_IN, FMT><<<static_cast<unsigned>(blocks), kThreads, 0, stream>>>(
+      x, rows, cols, cb, q, scales);
+  return cudaGetLastError() == cudaSuccess ? BSGEMM_OK : BSGEMM_ERR_CUDA;
+}
+
+template <int G>
+bsgemm_status dispatch_g(int src, int fmt, const void* x, int64_t rows, int64_t cols, uint8_t* q,
+                         float* s, cudaStream_t st) {
+  if (src == BSGEMM_SRC_BF16)
+    return fmt == BSGEMM_FP8_E5M2 ? launch<G, true, BSGEMM_FP8_E5M2>(x, rows, cols, q, s, st)
+                                  : launch<G, true, BSGEMM_FP8_E4M3>(x, rows, cols, q, s, st);
+  return fmt == BSGEMM_FP8_E5M2 ? launch<G, false, BSGEMM_FP8_E5M2>(x, rows, cols, q, s, st)
+                                : launch<G, false, BSGEMM_FP8_E4M3>(x, rows, cols, q, s, st);
+}
+
+}  // namespace bsgq
+
+extern "C" bsgemm_status bsgemm_quantize_fp8(int src_dtype, int fp8_format, const void* x,
+                                             int64_t rows, int64_t cols, int gran, void* q,
+                                             float* scales, bsgemm_stream_t stream) {
+  if (!x || !q || !scales || rows <= 0 || cols <= 0) return BSGEMM_ERR_INVALID_ARG;
+  if (src_dtype != BSGEMM_SRC_F32 && src_dtype != BSGEMM_SRC_BF16) return BSGEMM_ERR_INVALID_ARG;
+  if (fp8_format != BSGEMM_FP8_E4M3 && fp8_format != BSGEMM_FP8_E5M2) return BSGEMM_ERR_INVALID_ARG;
+  if (gran != 64 && gran != 128 && gran != 256) return BSGEMM_ERR_UNSUPPORTED_GRAN;
+  if (cols % 16 != 0 || (reinterpret_cast<uintptr_t>(x) & 15) != 0 ||
+      (reinterpret_cast<uintptr_t>(q) & 15) != 0 || (reinterpret_cast<uintptr_t>(scales) & 3) != 0)
+    return BSGEMM_ERR_MISALIGNED;
+  int dev = 0, major = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess)
+    return BSGEMM_ERR_CUDA;
+  if (major != 10) return BSGEMM_ERR_UNSUPPORTED_DEVICE;
+  auto* qq = static_cast<uint8_t*>(q);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  switch (gran) {
+    case 64:  return bsgq::dispatch_g<64>(src_dtype, fp8_format, x, rows, cols, qq, scales, s);
+    case 128: return bsgq::dispatch_g<128>(src_dtype, fp8_format, x, rows, cols, qq, scales, s);
+    default:  return bsgq::dispatch_g<256>(src_dtype, fp8_format, x, rows, cols, qq, scales, s);
+  }
+}

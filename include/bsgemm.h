@@ -147,11 +147,60 @@ typedef struct {
                            grid counts CTAs, two per pair) */
 } bsgemm_plan;
 
+/* FP8 formats of the operands (hncyxsy.com/news/191052 §2.2 names both).
+ * E4M3: the OCP "fn" variant, 1 sign, 4 exponent (bias 7), 3 mantissa bits,
+ * largest finite 448, no infinities, NaN 0x7F/0xFF.
+ * E5M2: 1 sign, 5 exponent (bias 15), 2 mantissa bits, largest finite 57344,
+ * +-Inf 0x7C/0xFC, NaN 0x7D-0x7F/0xFD-0xFF.
+ * Operands must hold finite codes only; the result for NaN or Inf inputs is
+ * unspecified (the call still completes and writes out). */
+typedef enum {
+    BSGEMM_FP8_E4M3 = 0,
+    BSGEMM_FP8_E5M2 = 1
+} bsgemm_fp8_format;
+
 /* The operation above with the layout as an argument and optional tuning
  * (NULL = heuristic). Same argument rules and errors as bsgemm_fp8_nt. */
 bsgemm_status bsgemm_fp8_gemm_ex(int layout, const void *a, const void *b, const float *scale_a,
                                  const float *scale_b, void *out, int64_t M, int64_t N, int64_t K,
                                  int gran, const bsgemm_tuning *tuning, bsgemm_stream_t stream);
+
+/* The operation with each operand's FP8 format given: a_format, b_format are
+ * bsgemm_fp8_format values (any combination; the tensor core decodes both,
+ * the products and block sums are the same FP32 path as E4M3 x E4M3).
+ * Everything else as bsgemm_fp8_gemm_ex; BSGEMM_ERR_INVALID_ARG for an
+ * unknown format. bsgemm_fp8_gemm_ex is this call with E4M3 x E4M3. */
+bsgemm_status bsgemm_fp8_gemm_fmt(int layout, int a_format, int b_format, const void *a,
+                                  const void *b, const float *scale_a, const float *scale_b,
+                                  void *out, int64_t M, int64_t N, int64_t K, int gran,
+                                  const bsgemm_tuning *tuning, bsgemm_stream_t stream);
+
+/* ---- per-block FP8 quantiser ---------------------------------------------
+ * The caller-side step the GEMM's scales come from (§4.4: the quantisation
+ * granularity must match the GEMM's; §5.2: quantising divides by the scale,
+ * dequantising multiplies). For each g x g block of the row-major
+ * [rows, cols] source x (FP32, or BF16 bits):
+ *   amax = max |x| over the block's elements (fewer in a partial block);
+ *   s    = amax / FMAX in FP32 (FMAX = 448 E4M3, 57344 E5M2), 1 if amax == 0;
+ *   q    = FP8 code of x / s (FP32 division, correctly rounded), nearest with
+ *          ties to even, saturated to +-FMAX.
+ * Outputs: q [rows, cols] row-major codes (the GEMM's A or B operand with
+ * K = cols) and scales [ceil(rows/g), ceil(cols/g)] row-major FP32 (its
+ * scale_a / scale_b). All pointers are device pointers owned by the caller;
+ * asynchronous on `stream`.
+ * Errors (before any launch, nothing written): NULL pointers or rows/cols
+ * <= 0 or unknown src_dtype / fp8_format -> BSGEMM_ERR_INVALID_ARG; gran not
+ * 64/128/256 -> BSGEMM_ERR_UNSUPPORTED_GRAN; cols % 16 != 0, x or q not
+ * 16-byte aligned, scales not 4-byte aligned -> BSGEMM_ERR_MISALIGNED; not an
+ * sm_100 device -> BSGEMM_ERR_UNSUPPORTED_DEVICE. Inputs must be finite. */
+typedef enum {
+    BSGEMM_SRC_F32 = 0,
+    BSGEMM_SRC_BF16 = 1
+} bsgemm_src_dtype;
+
+bsgemm_status bsgemm_quantize_fp8(int src_dtype, int fp8_format, const void *x, int64_t rows,
+                                  int64_t cols, int gran, void *q, float *scales,
+                                  bsgemm_stream_t stream);
 
 /* Host-only: the plan a call with these sizes would use on a device with
  * `num_sms` SMs. Touches no device. */

@@ -28,6 +28,7 @@ _lock = threading.Lock()
 _lib = None
 
 LAYOUTS = {"nt": 0, "tn": 1, "nn": 2, "tt": 3}
+FORMATS = {"e4m3": 0, "e5m2": 1}
 
 
 def build(force: bool = False) -> str:
@@ -57,6 +58,18 @@ def _load():
             lib.oracle_bsgemm_at.restype = ctypes.c_int
             lib.oracle_bsgemm_at.argtypes = [ctypes.c_int, p, p, p, p, i64, i64, i64, i64, i64,
                                              p, p, p, p]
+            lib.oracle_fp8_value.restype = ctypes.c_double
+            lib.oracle_fp8_value.argtypes = [ctypes.c_int, ctypes.c_uint8]
+            i32 = ctypes.c_int
+            lib.oracle_bsgemm_fmt.restype = ctypes.c_int
+            lib.oracle_bsgemm_fmt.argtypes = [i32, i32, i32, p, p, p, p, i64, i64, i64, i64, p, p]
+            lib.oracle_bsgemm_at_fmt.restype = ctypes.c_int
+            lib.oracle_bsgemm_at_fmt.argtypes = [i32, i32, i32, p, p, p, p, i64, i64, i64, i64, i64,
+                                                 p, p, p, p]
+            lib.oracle_fp8_encode.restype = ctypes.c_uint8
+            lib.oracle_fp8_encode.argtypes = [i32, ctypes.c_float]
+            lib.oracle_quantize_blocks.restype = ctypes.c_int
+            lib.oracle_quantize_blocks.argtypes = [i32, p, i64, i64, i64, p, p]
             lib.oracle_num_threads.restype = ctypes.c_int
             lib.oracle_num_threads.argtypes = []
             _lib = lib
@@ -75,6 +88,16 @@ def e4m3_value(code: int) -> float:
 def e4m3_table() -> np.ndarray:
     """All 256 E4M3 codes decoded to float64."""
     return np.array([e4m3_value(c) for c in range(256)], dtype=np.float64)
+
+
+def fp8_value(fmt: str, code: int) -> float:
+    """Exact value of one code of format ``fmt`` ("e4m3" or "e5m2")."""
+    return _load().oracle_fp8_value(FORMATS[fmt], int(code))
+
+
+def fp8_table(fmt: str) -> np.ndarray:
+    """All 256 codes of ``fmt`` decoded to float64 (E5M2: +-Inf and NaN codes included)."""
+    return np.array([fp8_value(fmt, c) for c in range(256)], dtype=np.float64)
 
 
 def bf16_rne(x: float) -> int:
@@ -101,19 +124,20 @@ def _check_inputs(layout, a, b, sa, sb, M, N, K, gran):
     return a, b, sa, sb
 
 
-def bsgemm(layout: str, a, b, sa, sb, M: int, N: int, K: int, gran: int):
+def bsgemm(layout: str, a, b, sa, sb, M: int, N: int, K: int, gran: int, a_fmt="e4m3", b_fmt="e4m3"):
     """Full oracle product. Returns (ref float64 [M,N], out bf16 bits uint16 [M,N])."""
     a, b, sa, sb = _check_inputs(layout, a, b, sa, sb, M, N, K, gran)
     ref = np.empty((M, N), dtype=np.float64)
     out = np.empty((M, N), dtype=np.uint16)
-    rc = _load().oracle_bsgemm(LAYOUTS[layout], _ptr(a), _ptr(b), _ptr(sa), _ptr(sb),
-                               M, N, K, gran, _ptr(ref), _ptr(out))
+    rc = _load().oracle_bsgemm_fmt(LAYOUTS[layout], FORMATS[a_fmt], FORMATS[b_fmt], _ptr(a), _ptr(b),
+                                   _ptr(sa), _ptr(sb), M, N, K, gran, _ptr(ref), _ptr(out))
     if rc != 0:
         raise RuntimeError(f"oracle_bsgemm failed with code {rc}")
     return ref, out
 
 
-def bsgemm_at(layout: str, a, b, sa, sb, M: int, N: int, K: int, gran: int, mi, ni):
+def bsgemm_at(layout: str, a, b, sa, sb, M: int, N: int, K: int, gran: int, mi, ni,
+              a_fmt="e4m3", b_fmt="e4m3"):
     """Oracle outputs at (mi[i], ni[i]) only. Returns (ref float64, out uint16)."""
     a, b, sa, sb = _check_inputs(layout, a, b, sa, sb, M, N, K, gran)
     mi = np.ascontiguousarray(mi, dtype=np.int64)
@@ -122,8 +146,30 @@ def bsgemm_at(layout: str, a, b, sa, sb, M: int, N: int, K: int, gran: int, mi, 
         raise ValueError("mi and ni must have the same shape")
     ref = np.empty(mi.shape, dtype=np.float64)
     out = np.empty(mi.shape, dtype=np.uint16)
-    rc = _load().oracle_bsgemm_at(LAYOUTS[layout], _ptr(a), _ptr(b), _ptr(sa), _ptr(sb),
-                                  M, N, K, gran, mi.size, _ptr(mi), _ptr(ni), _ptr(ref), _ptr(out))
+    rc = _load().oracle_bsgemm_at_fmt(LAYOUTS[layout], FORMATS[a_fmt], FORMATS[b_fmt], _ptr(a), _ptr(b),
+                                      _ptr(sa), _ptr(sb), M, N, K, gran, mi.size, _ptr(mi), _ptr(ni),
+                                      _ptr(ref), _ptr(out))
     if rc != 0:
         raise RuntimeError(f"oracle_bsgemm_at failed with code {rc}")
     return ref, out
+
+
+def fp8_encode(fmt: str, v: float) -> int:
+    """Nearest code of ``fmt`` to the FP32 value ``v``: ties to an even mantissa, saturating."""
+    return int(_load().oracle_fp8_encode(FORMATS[fmt], float(np.float32(v))))
+
+
+def quantize_blocks(x, gran: int, fmt: str = "e4m3"):
+    """Per-block FP8 quantisation of a row-major FP32 [rows, cols] matrix.
+
+    Returns (codes uint8 [rows, cols], scales float32 [ceil(rows/g), ceil(cols/g)]):
+    s = amax / FMAX per block (1 for an all-zero block), code = nearest(x / s)
+    with both divisions in FP32."""
+    x = np.ascontiguousarray(x, dtype=np.float32)
+    rows, cols = x.shape
+    q = np.empty((rows, cols), dtype=np.uint8)
+    s = np.empty((-(-rows // gran), -(-cols // gran)), dtype=np.float32)
+    rc = _load().oracle_quantize_blocks(FORMATS[fmt], _ptr(x), rows, cols, gran, _ptr(q), _ptr(s))
+    if rc != 0:
+        raise RuntimeError(f"oracle_quantize_blocks failed with code {rc}")
+    return q, s

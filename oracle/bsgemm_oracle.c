@@ -23,14 +23,21 @@
  *                                * sum_{k in block kb} dec(A[m,k]) * dec(B[n,k])
  *   out[m,n] = bf16_rne(ref[m,n])          (one rounding, straight from FP64)
  *
- * Arithmetic, chosen so that every step is either exact or one FP64 rounding:
- *   - dec(code) is an integer count of 2^-9 (every E4M3 value is a multiple
- *     of 2^-9, the smallest subnormal, and |value| <= 448 = 229376 * 2^-9);
- *   - the inner block sum is an exact int64 count of 2^-18 (|product| < 2^36,
- *     at most 256 terms, so |sum| < 2^44);
+ * The pages name two FP8 formats, E4M3 and E5M2 (§2.2); either operand may
+ * use either one (the _fmt entry points; the plain ones are E4M3 x E4M3).
+ *
+ * Arithmetic, chosen so that every step is exact or one FP64 rounding:
+ *   - dec(code) is an integer count of the format's smallest subnormal:
+ *     2^-9 for E4M3 (|value| <= 448 = 229376 * 2^-9), 2^-16 for E5M2
+ *     (|value| <= 57344 = 7 * 2^29 * 2^-16);
+ *   - the inner block sum is an exact 128-bit integer count of
+ *     2^-(qa + qb) (qa, qb = 9 or 16): |product| < 2^64, at most 256 terms;
+ *   - the block sum is converted to FP64: exact for E4M3 x E4M3 (|sum| <
+ *     2^44), otherwise exact whenever it has at most 53 significant bits and
+ *     else one rounding of relative size <= 2^-53;
  *   - sA*sB is exact in FP64 (24 + 24 significant bits <= 53);
- *   - term = blocksum * 2^-18 * (sA*sB) is one FP64 rounding, and the terms
- *     are added in ascending kb in FP64.
+ *   - term = blocksum * 2^-(qa+qb) * (sA*sB) is one FP64 rounding, and the
+ *     terms are added in ascending kb in FP64.
  *
  * Readings of points the pages leave open (each one is also listed in the
  * design notes): both operands use g x g blocks; the scale tensors are
@@ -79,6 +86,43 @@ static int e4m3_units(uint8_t code, int64_t *units)
     return 1;
 }
 
+/* ---- E5M2 (IEEE-like: infinities and NaNs) decode ---------------------------
+ * Bit layout: s eeeee mm, exponent bias 15.
+ *   eeeee == 0      : subnormal, value = (-1)^s * m/4 * 2^-14 = m * 2^-16
+ *   eeeee == 11111  : +-Inf (mm == 0) or NaN (mm != 0)
+ *   otherwise       : value = (-1)^s * (1 + m/4) * 2^(e-15)
+ *                           = (-1)^s * (4 + m) * 2^(e-1) * 2^-16
+ * The result is the value as a signed integer count of 2^-16.              */
+static int e5m2_units(uint8_t code, int64_t *units)
+{
+    int s = code >> 7;
+    int e = (code >> 2) & 0x1F;
+    int m = code & 0x3;
+    int64_t mag;
+    if (e == 0x1F)
+        return 0; /* Inf or NaN: not a finite input */
+    if (e == 0)
+        mag = m;
+    else
+        mag = (int64_t)(4 + m) << (e - 1);
+    *units = s ? -mag : mag;
+    return 1;
+}
+
+#define OR_FMT_E4M3 0
+#define OR_FMT_E5M2 1
+
+/* Decode one code of format fmt: units of 2^-quantum_log2(fmt). */
+static inline int fp8_units(int fmt, uint8_t code, int64_t *units)
+{
+    return fmt == OR_FMT_E5M2 ? e5m2_units(code, units) : e4m3_units(code, units);
+}
+
+static inline int quantum_log2(int fmt)
+{
+    return fmt == OR_FMT_E5M2 ? 16 : 9;
+}
+
 /* Value of one E4M3 code as a double (NaN for the NaN codes). */
 double oracle_e4m3_value(uint8_t code)
 {
@@ -86,6 +130,20 @@ double oracle_e4m3_value(uint8_t code)
     if (!e4m3_units(code, &u))
         return NAN;
     return ldexp((double)u, -9);
+}
+
+/* Value of one code of format fmt (0 E4M3, 1 E5M2) as a double. E5M2's
+ * infinities decode to +-Inf and its NaN codes to NaN.                     */
+double oracle_fp8_value(int fmt, uint8_t code)
+{
+    int64_t u = 0;
+    if (fmt == OR_FMT_E5M2) {
+        if (((code >> 2) & 0x1F) == 0x1F)
+            return (code & 0x3) ? NAN : ((code >> 7) ? -INFINITY : INFINITY);
+        e5m2_units(code, &u);
+        return ldexp((double)u, -16);
+    }
+    return oracle_e4m3_value(code);
 }
 
 /* ---- FP64 -> BF16, round to nearest, ties to even --------------------------
@@ -138,28 +196,29 @@ static inline uint8_t elem_b(int layout, const uint8_t *b, int64_t N, int64_t K,
 }
 
 /* One output element: the definition above, term by term.
- * Returns 0 on success, OR_ERR_NAN_INPUT if a NaN code was met.          */
-static int one_element(int layout, const uint8_t *a, const uint8_t *b, const float *sa,
-                       const float *sb, int64_t M, int64_t N, int64_t K, int64_t g,
-                       int64_t m, int64_t n, double *ref)
+ * Returns 0 on success, OR_ERR_NAN_INPUT if a non-finite code was met.   */
+static int one_element(int layout, int fa, int fb, const uint8_t *a, const uint8_t *b,
+                       const float *sa, const float *sb, int64_t M, int64_t N, int64_t K,
+                       int64_t g, int64_t m, int64_t n, double *ref)
 {
     int64_t Kb = (K + g - 1) / g;
+    int shift = quantum_log2(fa) + quantum_log2(fb);
     double acc = 0.0;
     for (int64_t kb = 0; kb < Kb; ++kb) {
         int64_t k0 = kb * g;
         int64_t k1 = k0 + g < K ? k0 + g : K;
-        int64_t blocksum = 0; /* exact, units of 2^-18 */
+        __int128 blocksum = 0; /* exact, units of 2^-shift */
         for (int64_t k = k0; k < k1; ++k) {
             int64_t ua, ub;
-            if (!e4m3_units(elem_a(layout, a, M, K, m, k), &ua) ||
-                !e4m3_units(elem_b(layout, b, N, K, n, k), &ub)) {
+            if (!fp8_units(fa, elem_a(layout, a, M, K, m, k), &ua) ||
+                !fp8_units(fb, elem_b(layout, b, N, K, n, k), &ub)) {
                 *ref = NAN;
                 return OR_ERR_NAN_INPUT;
             }
-            blocksum += ua * ub;
+            blocksum += (__int128)ua * ub;
         }
         double scale = (double)sa[(m / g) * Kb + kb] * (double)sb[(n / g) * Kb + kb]; /* exact */
-        acc += ldexp((double)blocksum, -18) * scale;
+        acc += ldexp((double)blocksum, -shift) * scale;
     }
     *ref = acc;
     return OR_OK;
@@ -178,18 +237,21 @@ static int check_args(int layout, const void *a, const void *b, const float *sa,
 /* Full output. ref: FP64 [M*N] (may be NULL); out: BF16 bits [M*N] (may be NULL).
  * Parallel over rows with OpenMP when compiled with it; each element is
  * computed independently, so the result does not depend on the thread count. */
-int oracle_bsgemm(int layout, const uint8_t *a, const uint8_t *b, const float *sa, const float *sb,
-                  int64_t M, int64_t N, int64_t K, int64_t g, double *ref, uint16_t *out)
+int oracle_bsgemm_fmt(int layout, int fa, int fb, const uint8_t *a, const uint8_t *b,
+                      const float *sa, const float *sb, int64_t M, int64_t N, int64_t K, int64_t g,
+                      double *ref, uint16_t *out)
 {
     int rc = check_args(layout, a, b, sa, sb, M, N, K, g);
     int bad = 0;
     if (rc)
         return rc;
+    if ((fa != OR_FMT_E4M3 && fa != OR_FMT_E5M2) || (fb != OR_FMT_E4M3 && fb != OR_FMT_E5M2))
+        return OR_ERR_ARG;
 #pragma omp parallel for schedule(dynamic, 1) reduction(| : bad)
     for (int64_t m = 0; m < M; ++m) {
         for (int64_t n = 0; n < N; ++n) {
             double r;
-            bad |= one_element(layout, a, b, sa, sb, M, N, K, g, m, n, &r);
+            bad |= one_element(layout, fa, fb, a, b, sa, sb, M, N, K, g, m, n, &r);
             if (ref)
                 ref[m * N + n] = r;
             if (out)
@@ -201,14 +263,17 @@ int oracle_bsgemm(int layout, const uint8_t *a, const uint8_t *b, const float *s
 
 /* Selected outputs only: element i is (mi[i], ni[i]). For parity checks at
  * sizes where the full product would take the oracle too long.            */
-int oracle_bsgemm_at(int layout, const uint8_t *a, const uint8_t *b, const float *sa,
-                     const float *sb, int64_t M, int64_t N, int64_t K, int64_t g, int64_t count,
-                     const int64_t *mi, const int64_t *ni, double *ref, uint16_t *out)
+int oracle_bsgemm_at_fmt(int layout, int fa, int fb, const uint8_t *a, const uint8_t *b,
+                         const float *sa, const float *sb, int64_t M, int64_t N, int64_t K,
+                         int64_t g, int64_t count, const int64_t *mi, const int64_t *ni,
+                         double *ref, uint16_t *out)
 {
     int rc = check_args(layout, a, b, sa, sb, M, N, K, g);
     int bad = 0;
     if (rc)
         return rc;
+    if ((fa != OR_FMT_E4M3 && fa != OR_FMT_E5M2) || (fb != OR_FMT_E4M3 && fb != OR_FMT_E5M2))
+        return OR_ERR_ARG;
     if (count < 0 || (count > 0 && (!mi || !ni)))
         return OR_ERR_ARG;
     for (int64_t i = 0; i < count; ++i)
@@ -217,13 +282,28 @@ int oracle_bsgemm_at(int layout, const uint8_t *a, const uint8_t *b, const float
 #pragma omp parallel for schedule(dynamic, 16) reduction(| : bad)
     for (int64_t i = 0; i < count; ++i) {
         double r;
-        bad |= one_element(layout, a, b, sa, sb, M, N, K, g, mi[i], ni[i], &r);
+        bad |= one_element(layout, fa, fb, a, b, sa, sb, M, N, K, g, mi[i], ni[i], &r);
         if (ref)
             ref[i] = r;
         if (out)
             out[i] = oracle_bf16_rne(r);
     }
     return bad ? OR_ERR_NAN_INPUT : OR_OK;
+}
+
+/* E4M3 x E4M3 forms of the two entry points above. */
+int oracle_bsgemm(int layout, const uint8_t *a, const uint8_t *b, const float *sa, const float *sb,
+                  int64_t M, int64_t N, int64_t K, int64_t g, double *ref, uint16_t *out)
+{
+    return oracle_bsgemm_fmt(layout, OR_FMT_E4M3, OR_FMT_E4M3, a, b, sa, sb, M, N, K, g, ref, out);
+}
+
+int oracle_bsgemm_at(int layout, const uint8_t *a, const uint8_t *b, const float *sa,
+                     const float *sb, int64_t M, int64_t N, int64_t K, int64_t g, int64_t count,
+                     const int64_t *mi, const int64_t *ni, double *ref, uint16_t *out)
+{
+    return oracle_bsgemm_at_fmt(layout, OR_FMT_E4M3, OR_FMT_E4M3, a, b, sa, sb, M, N, K, g, count,
+                                mi, ni, ref, out);
 }
 
 /* Number of OpenMP threads the oracle would use (1 without OpenMP). */
@@ -235,4 +315,77 @@ int oracle_num_threads(void)
 #else
     return 1;
 #endif
+}
+
+/* ---- per-block FP8 quantisation (§4.4 granularity must match, §5.2
+ * "quantise divides, dequantise multiplies") ------------------------------
+ * For each g x g block of a row-major [rows, cols] FP32 matrix x:
+ *   amax  = max |x| over the block's elements (partial blocks: the elements
+ *           that exist);
+ *   s     = amax / FMAX in FP32 (FMAX = 448 for E4M3, 57344 for E5M2), or
+ *           1.0 when amax is 0;
+ *   q     = the format's code nearest to the FP32 quotient x / s, ties to the
+ *           code with an even mantissa, saturating to +-FMAX.
+ * FP32 arithmetic is used for s and x / s because that is where the decision
+ * of each integer code is taken; it is IEEE division, correctly rounded.   */
+/* Nearest finite code to v (finite FP32), ties to even mantissa, saturating. */
+uint8_t oracle_fp8_encode(int fmt, float v)
+{
+    double fmax = fmt == OR_FMT_E5M2 ? 57344.0 : 448.0;
+    double x = (double)v; /* exact */
+    int neg = signbit(x) ? 1 : 0;
+    double ax = fabs(x);
+    int best = -1;
+    double best_err = 0.0;
+    if (ax >= fmax)
+        ax = fmax;
+    /* non-negative codes 0x00..0x7F: finite ones, increasing in value */
+    for (int c = 0; c < 0x80; ++c) {
+        double cv = oracle_fp8_value(fmt, (uint8_t)c);
+        double err;
+        if (!isfinite(cv))
+            continue;
+        err = fabs(cv - ax);
+        /* a tie is between two neighbouring codes; the even one (mantissa
+         * LSB = code LSB = 0) wins */
+        if (best < 0 || err < best_err || (err == best_err && (c & 1) == 0)) {
+            best = c;
+            best_err = err;
+        }
+    }
+    if (neg)
+        best |= 0x80; /* the sign is kept, zero included */
+    return (uint8_t)best;
+}
+
+int oracle_quantize_blocks(int fmt, const float *x, int64_t rows, int64_t cols, int64_t g,
+                           uint8_t *q, float *scales)
+{
+    int64_t Rb, Cb;
+    float fmax;
+    if ((fmt != OR_FMT_E4M3 && fmt != OR_FMT_E5M2) || !x || !q || !scales || rows <= 0 ||
+        cols <= 0 || g <= 0)
+        return OR_ERR_ARG;
+    Rb = (rows + g - 1) / g;
+    Cb = (cols + g - 1) / g;
+    fmax = fmt == OR_FMT_E5M2 ? 57344.0f : 448.0f;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int64_t blk = 0; blk < Rb * Cb; ++blk) {
+        int64_t rb = blk / Cb, cb = blk % Cb;
+        int64_t r0 = rb * g, r1 = r0 + g < rows ? r0 + g : rows;
+        int64_t c0 = cb * g, c1 = c0 + g < cols ? c0 + g : cols;
+        float amax = 0.0f, s;
+        for (int64_t r = r0; r < r1; ++r)
+            for (int64_t c = c0; c < c1; ++c) {
+                float a = fabsf(x[r * cols + c]);
+                if (a > amax)
+                    amax = a;
+            }
+        s = amax > 0.0f ? amax / fmax : 1.0f;
+        scales[rb * Cb + cb] = s;
+        for (int64_t r = r0; r < r1; ++r)
+            for (int64_t c = c0; c < c1; ++c)
+                q[r * cols + c] = oracle_fp8_encode(fmt, x[r * cols + c] / s);
+    }
+    return OR_OK;
 }

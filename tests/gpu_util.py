@@ -25,7 +25,8 @@ def to_device(p: workloads.Problem, device="cuda"):
 
 def run_gpu(p: workloads.Problem, tuning=None, out=None):
     a, b, sa, sb = to_device(p)
-    out = bsg.gemm(a, b, sa, sb, out=out, layout=p.layout, gran=p.gran, tuning=tuning)
+    out = bsg.gemm(a, b, sa, sb, out=out, layout=p.layout, gran=p.gran, tuning=tuning,
+                   a_format=p.a_fmt, b_format=p.b_fmt)
     torch.cuda.synchronize()
     return out
 
@@ -57,13 +58,14 @@ def check_close(got: np.ndarray, ref: np.ndarray, what=""):
 
 def full_parity(p: workloads.Problem, tuning=None, what=""):
     out = run_gpu(p, tuning)
-    ref, _ = oracle.bsgemm(p.layout, p.a, p.b, p.sa, p.sb, p.M, p.N, p.K, p.gran)
+    ref, _ = oracle.bsgemm(p.layout, p.a, p.b, p.sa, p.sb, p.M, p.N, p.K, p.gran, p.a_fmt, p.b_fmt)
     return check_close(gpu_as_f64(out), ref, what or p.name), out
 
 
 def sampled_parity(p: workloads.Problem, count=3000, tuning=None, seed=0, what=""):
     out = run_gpu(p, tuning)
     mi, ni = workloads.sample_indices(p.M, p.N, count, seed=seed)
-    ref, _ = oracle.bsgemm_at(p.layout, p.a, p.b, p.sa, p.sb, p.M, p.N, p.K, p.gran, mi, ni)
+    ref, _ = oracle.bsgemm_at(p.layout, p.a, p.b, p.sa, p.sb, p.M, p.N, p.K, p.gran, mi, ni,
+                              p.a_fmt, p.b_fmt)
     got = gpu_as_f64(out[torch.from_numpy(mi).cuda(), torch.from_numpy(ni).cuda()])
     return check_close(got, ref, what or p.name), out

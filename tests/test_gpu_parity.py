@@ -104,6 +104,53 @@ def test_cta_pair_agrees_with_single_cta():
     check_close(two, one, "pair vs single CTA")
 
 
+# ---------------------------------------------------------------- E5M2 operands (§2.2 second format)
+@pytest.mark.parametrize("fa,fb", [("e5m2", "e4m3"), ("e4m3", "e5m2"), ("e5m2", "e5m2")])
+@pytest.mark.parametrize("layout", ["nt", "tn", "nn", "tt"])
+def test_e5m2_operands_each_layout(fa, fb, layout):
+    p = workloads.make_problem(272, 528, 1040, 128, layout, seed=21, a_fmt=fa, b_fmt=fb)
+    full_parity(p, what=f"{fa} x {fb} {layout}")
+
+
+@pytest.mark.parametrize("fa,fb", [("e5m2", "e4m3"), ("e5m2", "e5m2")])
+@pytest.mark.parametrize("tuning,M,gran", [
+    ({"variant": "swap_ab", "bnq": 32, "splits": 3}, 24, 64),
+    ({"variant": "data_parallel", "bnq": 128, "stream_k": 1}, 600, 256),
+    ({"variant": "cta_pair"}, 600, 128),
+])
+def test_e5m2_operands_each_variant(fa, fb, tuning, M, gran):
+    p = workloads.make_problem(M, 784, 1536, gran, "nt", seed=22, a_fmt=fa, b_fmt=fb)
+    full_parity(p, tuning=tuning, what=f"{fa} x {fb} {tuning}")
+
+
+def test_e5m2_integer_exact_bit_for_bit():
+    """Small integers are exact in both formats; power-of-two scales keep every
+    partial sum exact, so the GPU must equal the oracle bit for bit."""
+    rng = np.random.default_rng(23)
+    M, N, K, g = 192, 272, 512, 128
+    vals5 = {0x00: 0, 0x3C: 1, 0x40: 2, 0x42: 3, 0x44: 4, 0xBC: -1, 0xC0: -2, 0xC2: -3, 0xC4: -4}
+    vals4 = {0x00: 0, 0x38: 1, 0x40: 2, 0x44: 3, 0x48: 4, 0xB8: -1, 0xC0: -2, 0xC4: -3, 0xC8: -4}
+    a = np.array(list(vals5))[rng.integers(0, 9, size=(M, K))].astype(np.uint8)
+    b = np.array(list(vals4))[rng.integers(0, 9, size=(N, K))].astype(np.uint8)
+    Kb = K // g
+    sa = np.exp2(rng.integers(-3, 2, size=(-(-M // g), Kb))).astype(np.float32)
+    sb = np.exp2(rng.integers(-3, 2, size=(-(-N // g), Kb))).astype(np.float32)
+    p = workloads.Problem(M, N, K, g, "nt", a, b, sa, sb, "int e5m2 x e4m3", "e5m2", "e4m3")
+    ref, bits = oracle.bsgemm("nt", a, b, sa, sb, M, N, K, g, "e5m2", "e4m3")
+    got = run_gpu(p).view(torch.int16).cpu().numpy().view(np.uint16)
+    assert np.array_equal(got, bits)
+
+
+def test_e5m2_binding_takes_format_from_dtype():
+    p = workloads.make_problem(128, 256, 256, 128, "nt", seed=24, a_fmt="e5m2", b_fmt="e4m3")
+    a, b, sa, sb = to_device(p)
+    out = bsg.gemm(a.view(torch.float8_e5m2), b.view(torch.float8_e4m3fn), sa, sb, layout="nt")
+    ref, _ = oracle.bsgemm("nt", p.a, p.b, p.sa, p.sb, p.M, p.N, p.K, 128, "e5m2", "e4m3")
+    check_close(gpu_as_f64(out), ref, "dtype-derived formats")
+    with pytest.raises(ValueError):
+        bsg.gemm(a.view(torch.float8_e5m2), b, sa, sb, a_format="e4m3")
+
+
 # ---------------------------------------------------------------- small M (decode-style)
 @pytest.mark.parametrize("M", [1, 8, 32, 64, 128])
 def test_small_m_reduced_k(M):

@@ -1,0 +1,73 @@
+"""GPU per-block FP8 quantiser (``bsgemm_quantize_fp8``) against the oracle's.
+
+The codes are integer decisions taken in FP32 on both sides (s = amax / FMAX,
+then x / s, both correctly rounded, then nearest-even with saturation), so the
+bar is bit-exact codes and scales (hncyxsy.com/news/191052 §4.4, §5.2).
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import workloads
+import fp8_block_scaled_bsgemm_b200 as bsg
+
+from gpu_util import check_close, gpu_as_f64
+
+pytestmark = pytest.mark.gpu
+
+
+def _source(rows, cols, seed, scale=3.0):
+    rng = np.random.default_rng(seed)
+    x = rng.standard_normal((rows, cols)).astype(np.float32) * np.float32(scale)
+    x[:40, :64] = 0.0                               # an all-zero region (whole block at g = 64)
+    x[rows // 2, 16] = np.float32(5e3)              # an outlier
+    return x
+
+
+@pytest.mark.parametrize("fmt", ["e4m3", "e5m2"])
+@pytest.mark.parametrize("g", [64, 128, 256])
+@pytest.mark.parametrize("rows,cols", [(300, 528), (64, 64), (1, 4096)])
+def test_quantiser_fp32_bit_exact(fmt, g, rows, cols):
+    x = _source(rows, cols, rows + g)
+    q, s = bsg.quantize(torch.from_numpy(x).cuda(), g, fmt)
+    q_ref, s_ref = oracle.quantize_blocks(x, g, fmt)
+    assert np.array_equal(s.cpu().numpy(), s_ref)
+    assert np.array_equal(q.cpu().numpy(), q_ref)
+
+
+@pytest.mark.parametrize("fmt", ["e4m3", "e5m2"])
+@pytest.mark.parametrize("g", [64, 128])
+def test_quantiser_bf16_bit_exact(fmt, g):
+    x32 = _source(200, 1040, 5)
+    xb = torch.from_numpy(x32).to(torch.bfloat16)
+    q, s = bsg.quantize(xb.cuda(), g, fmt)
+    q_ref, s_ref = oracle.quantize_blocks(xb.float().numpy(), g, fmt)   # BF16 -> FP32 is exact
+    assert np.array_equal(s.cpu().numpy(), s_ref)
+    assert np.array_equal(q.cpu().numpy(), q_ref)
+
+
+def test_quantise_then_gemm_matches_oracle_pipeline():
+    """Online activations: quantise A and B on the GPU, multiply on the GPU;
+    the same steps in the oracle give the reference."""
+    M, N, K, g = 320, 784, 1152, 128
+    rng = np.random.default_rng(9)
+    a32 = rng.standard_normal((M, K)).astype(np.float32)
+    b32 = (rng.standard_normal((N, K)) * 0.02).astype(np.float32)
+    qa, sa = bsg.quantize(torch.from_numpy(a32).cuda(), g)
+    qb, sb = bsg.quantize(torch.from_numpy(b32).cuda(), g, "e5m2")
+    out = bsg.gemm(qa, qb, sa, sb, layout="nt", gran=g, a_format="e4m3", b_format="e5m2")
+    oqa, osa = oracle.quantize_blocks(a32, g)
+    oqb, osb = oracle.quantize_blocks(b32, g, "e5m2")
+    ref, _ = oracle.bsgemm("nt", oqa, oqb, osa, osb, M, N, K, g, "e4m3", "e5m2")
+    check_close(gpu_as_f64(out), ref, "quantise + GEMM")
+
+
+def test_quantiser_host_errors():
+    x = torch.zeros((8, 40), device="cuda")
+    with pytest.raises(bsg.BsgemmError) as e:
+        bsg.quantize(x, 128)                          # cols % 16 != 0
+    assert e.value.status == 3
+    with pytest.raises(bsg.BsgemmError) as e:
+        bsg.quantize(torch.zeros((8, 64), device="cuda"), 32)
+    assert e.value.status == 2

@@ -304,3 +304,149 @@ def test_nan_code_is_reported():
     b = np.full((1, 16), 0x38, np.uint8)
     with pytest.raises(RuntimeError):
         oracle.bsgemm("nt", a, b, np.ones((1, 1), np.float32), np.ones((1, 1), np.float32), 1, 1, 16, 128)
+
+
+# --------------------------------------------------------------------------- E5M2 (second format, §2.2)
+def test_e5m2_table_matches_torch_decode():
+    codes = torch.arange(256, dtype=torch.int32).to(torch.uint8)
+    ref = codes.view(torch.float8_e5m2).to(torch.float64).numpy()
+    got = oracle.fp8_table("e5m2")
+    nan = np.isnan(ref)
+    assert sorted(np.nonzero(nan)[0].tolist()) == [0x7D, 0x7E, 0x7F, 0xFD, 0xFE, 0xFF]
+    assert np.array_equal(np.isnan(got), nan)
+    assert np.array_equal(got[~nan], ref[~nan])          # includes +-Inf at 0x7C / 0xFC
+
+
+@pytest.mark.parametrize("code,value", [
+    (0x3C, 1.0), (0x38, 0.5), (0x40, 2.0), (0x42, 3.0), (0x45, 5.0), (0xBC, -1.0),
+    (0x7B, 57344.0), (0xFB, -57344.0), (0x01, 2.0 ** -16), (0x03, 3 * 2.0 ** -16),
+    (0x04, 2.0 ** -14), (0x7C, math.inf), (0x00, 0.0),
+])
+def test_e5m2_hand_values(code, value):
+    assert oracle.fp8_value("e5m2", code) == value
+
+
+def test_e4m3_entry_equals_format_entry():
+    assert all(oracle.fp8_value("e4m3", c) == oracle.e4m3_value(c) or
+               (math.isnan(oracle.e4m3_value(c)) and math.isnan(oracle.fp8_value("e4m3", c)))
+               for c in range(256))
+
+
+def _dec_fmt(fmt):
+    dt = torch.float8_e5m2 if fmt == "e5m2" else torch.float8_e4m3fn
+    return torch.arange(256, dtype=torch.int32).to(torch.uint8).view(dt).to(torch.float64).tolist()
+
+
+def _finite_codes(fmt):
+    t = _dec_fmt(fmt)
+    return np.array([c for c in range(256) if math.isfinite(t[c])], dtype=np.uint8)
+
+
+@pytest.mark.parametrize("fa,fb", [("e5m2", "e4m3"), ("e4m3", "e5m2"), ("e5m2", "e5m2")])
+@pytest.mark.parametrize("M,N,K,g,seed", [(4, 3, 320, 64, 10), (3, 130, 256, 128, 11)])
+def test_brute_force_exact_rational_mixed_formats(fa, fb, M, N, K, g, seed):
+    """Exact rationals, per-element dequantisation, every finite code of each format."""
+    rng = np.random.default_rng(seed)
+    a = _finite_codes(fa)[rng.integers(0, _finite_codes(fa).size, size=(M, K))]
+    b = _finite_codes(fb)[rng.integers(0, _finite_codes(fb).size, size=(N, K))]
+    Kb = -(-K // g)
+    sa = rng.uniform(0.01, 3.0, size=(-(-M // g), Kb)).astype(np.float32)
+    sb = rng.uniform(0.01, 3.0, size=(-(-N // g), Kb)).astype(np.float32)
+    ref, out = oracle.bsgemm("nt", a, b, sa, sb, M, N, K, g, a_fmt=fa, b_fmt=fb)
+    da, db = _dec_fmt(fa), _dec_fmt(fb)
+    for m in range(M):
+        for n in range(N if N < 8 else 8):
+            ex = Fraction(0)
+            bound = Fraction(0)
+            for k in range(K):
+                t = Fraction(da[a[m, k]]) * Fraction(db[b[n, k]]) * \
+                    Fraction(float(sa[m // g, k // g])) * Fraction(float(sb[n // g, k // g]))
+                ex += t
+                bound += abs(t)
+            # block sums may need one more FP64 rounding with E5M2 operands
+            tol = bound * Fraction(2 * Kb + 2) * Fraction(2) ** -52
+            assert abs(Fraction(ref[m, n]) - ex) <= tol, (fa, fb, m, n)
+            lo, hi = float(ex - tol), float(ex + tol)
+            if _bf16_rne_exact(lo) == _bf16_rne_exact(hi):
+                assert out[m, n] == _bf16_rne_exact(float(ex)), (m, n)
+
+
+def test_e5m2_closed_form_all_ones():
+    # 0x3C is 1.0 in E5M2, 0x38 is 1.0 in E4M3: out = K * sA * sB per block
+    M, N, K, g = 3, 5, 384, 128
+    a = np.full((M, K), 0x3C, np.uint8)
+    b = np.full((N, K), 0x38, np.uint8)
+    sa = np.full((1, 3), 0.5, np.float32)
+    sb = np.array([[2.0, 4.0, 8.0]], np.float32)
+    ref, _ = oracle.bsgemm("nt", a, b, sa, sb, M, N, K, g, a_fmt="e5m2", b_fmt="e4m3")
+    assert np.all(ref == 128 * 0.5 * (2.0 + 4.0 + 8.0))
+
+
+def test_e5m2_nonfinite_codes_are_reported():
+    a = np.full((1, 16), 0x3C, np.uint8)
+    b = np.full((1, 16), 0x3C, np.uint8)
+    for bad in (0x7C, 0xFC, 0x7E):
+        a2 = a.copy(); a2[0, 5] = bad
+        with pytest.raises(RuntimeError):
+            oracle.bsgemm("nt", a2, b, np.ones((1, 1), np.float32), np.ones((1, 1), np.float32),
+                          1, 1, 16, 128, a_fmt="e5m2", b_fmt="e5m2")
+
+
+def test_workload_quantiser_e5m2_round_trip():
+    """The caller-side E5M2 quantiser: codes decode to values within E5M2 rounding of x / s."""
+    rng = np.random.default_rng(3)
+    x = rng.standard_normal((130, 200)).astype(np.float32)
+    q, s = workloads.quantize_blocks(x, 64, "e5m2")
+    dec = np.array(_dec_fmt("e5m2"))[q]
+    scale = np.repeat(np.repeat(s, 64, axis=0), 64, axis=1)[:130, :200].astype(np.float64)
+    back = dec * scale
+    # E5M2 keeps 3 significant bits: relative rounding error <= 2^-3 for normal values
+    assert np.all(np.abs(back - x) <= 2.0 ** -3 * np.abs(x) + scale * 2.0 ** -16)
+    assert np.isclose(np.max(np.abs(dec)), 57344.0)
+
+
+# --------------------------------------------------------------------------- quantiser (§4.4, §5.2)
+@pytest.mark.parametrize("fmt,tdtype,fmax", [("e4m3", torch.float8_e4m3fn, 448.0),
+                                             ("e5m2", torch.float8_e5m2, 57344.0)])
+def test_fp8_encode_matches_torch_saturating_cast(fmt, tdtype, fmax):
+    """torch's float32 -> float8 cast rounds to nearest even; clamping first
+    makes it saturating, which is what the oracle's encoder must equal."""
+    rng = np.random.default_rng(7)
+    mags = rng.choice([1e-7, 1e-5, 1e-3, 0.1, 1.0, 30.0, 300.0, 3e4], size=8000).astype(np.float32)
+    v = np.concatenate([rng.standard_normal(8000).astype(np.float32) * mags,
+                        np.array([0.0, -0.0, fmax, -fmax, 2 * fmax, -3 * fmax], np.float32)])
+    ours = np.array([oracle.fp8_encode(fmt, x) for x in v], np.uint8)
+    ref = torch.from_numpy(np.clip(v, -fmax, fmax)).to(tdtype).view(torch.uint8).numpy()
+    assert np.array_equal(ours, ref)
+
+
+@pytest.mark.parametrize("fmt,v,code", [
+    ("e4m3", 1.0625, 0x38), ("e4m3", 1.1875, 0x3A), ("e4m3", 3 * 2.0 ** -10, 0x02),  # ties -> even
+    ("e4m3", 2.0 ** -10, 0x00), ("e4m3", -2.0 ** -11, 0x80), ("e4m3", 464.0, 0x7E),   # underflow, saturation
+    ("e5m2", 1.125, 0x3C), ("e5m2", 1.375, 0x3E), ("e5m2", 61440.0, 0x7B), ("e5m2", -1e9, 0xFB),
+])
+def test_fp8_encode_hand_values(fmt, v, code):
+    assert oracle.fp8_encode(fmt, v) == code
+
+
+@pytest.mark.parametrize("fmt", ["e4m3", "e5m2"])
+@pytest.mark.parametrize("rows,cols,g", [(130, 208, 64), (257, 384, 128), (96, 512, 256)])
+def test_oracle_quantiser_matches_torch_quantiser(fmt, rows, cols, g):
+    """The C quantiser against the torch one in workloads (amax, FP32 divide,
+    clamp, cast): two independent restatements, bit for bit."""
+    rng = np.random.default_rng(rows + cols)
+    x = rng.standard_normal((rows, cols)).astype(np.float32) * np.float32(3.0)
+    x[: min(g, rows), :g] = 0.0                      # an all-zero block -> scale 1
+    x[-1, -5:] = np.float32(1e4)                     # a block dominated by outliers
+    q1, s1 = oracle.quantize_blocks(x, g, fmt)
+    q2, s2 = workloads.quantize_blocks(x, g, fmt)
+    assert s1[0, 0] == 1.0
+    assert np.array_equal(s1, s2) and np.array_equal(q1, q2)
+
+
+def test_oracle_quantiser_round_trip_error():
+    x = np.random.default_rng(2).standard_normal((128, 256)).astype(np.float32)
+    q, s = oracle.quantize_blocks(x, 128, "e4m3")
+    back = oracle.e4m3_table()[q] * np.repeat(np.repeat(s, 128, 0), 128, 1)
+    # E4M3 keeps 4 significant bits: relative error <= 2^-4 above the subnormal range
+    assert np.all(np.abs(back - x) <= 2.0 ** -4 * np.abs(x) + np.repeat(np.repeat(s, 128, 0), 128, 1) * 2.0 ** -9)

@@ -7,11 +7,13 @@ the library would (hncyxsy.com/news/191052 §4.4: quantisation happens outside
 the GEMM library, with a granularity that must match the GEMM's).
 
 Caller-side preparation, per g x g block of each operand:
-  scale = amax / 448       (448 is the largest finite E4M3 value; a block
-                            whose amax is 0 gets scale 1.0)
-  code  = E4M3(clamp(x / scale, -448, 448))   (round to nearest even)
-The cast uses torch's ``float8_e4m3fn`` conversion; the clamp makes it
-saturating. The scale tensors are row-major FP32 [ceil(rows/g), ceil(K/g)].
+  scale = amax / FMAX      (FMAX is the format's largest finite value: 448
+                            for E4M3, 57344 for E5M2; a block whose amax is 0
+                            gets scale 1.0)
+  code  = FP8(clamp(x / scale, -FMAX, FMAX))   (round to nearest even)
+The cast uses torch's ``float8_e4m3fn`` / ``float8_e5m2`` conversion; the
+clamp makes it saturating. The scale tensors are row-major FP32
+[ceil(rows/g), ceil(K/g)].
 
 Workloads (synthetic stand-ins for the transformer projection / FFN GEMMs
 the pages centre on; no dataset is involved):
@@ -33,6 +35,8 @@ import numpy as np
 import torch
 
 E4M3_MAX = 448.0
+E5M2_MAX = 57344.0
+FORMATS = {"e4m3": (E4M3_MAX, torch.float8_e4m3fn), "e5m2": (E5M2_MAX, torch.float8_e5m2)}
 
 LAYOUTS = ("nt", "tn", "nn", "tt")
 
@@ -45,22 +49,25 @@ class Problem:
     K: int
     gran: int
     layout: str
-    a: np.ndarray   # uint8 E4M3 codes; [M,K] for layouts n?, [K,M] for t?
-    b: np.ndarray   # uint8 E4M3 codes; [N,K] for ?t, [K,N] for ?n
+    a: np.ndarray   # uint8 FP8 codes; [M,K] for layouts n?, [K,M] for t?
+    b: np.ndarray   # uint8 FP8 codes; [N,K] for ?t, [K,N] for ?n
     sa: np.ndarray  # float32 [ceil(M/g), ceil(K/g)]
     sb: np.ndarray  # float32 [ceil(N/g), ceil(K/g)]
     name: str = ""
+    a_fmt: str = "e4m3"
+    b_fmt: str = "e4m3"
 
     @property
     def flops(self) -> int:
         return 2 * self.M * self.N * self.K
 
 
-def quantize_blocks(x: np.ndarray, gran: int):
-    """Caller-side per-block E4M3 quantisation of a logical [R, K] FP32 matrix.
+def quantize_blocks(x: np.ndarray, gran: int, fmt: str = "e4m3"):
+    """Caller-side per-block FP8 quantisation of a logical [R, K] FP32 matrix.
 
     Returns (codes uint8 [R, K], scales float32 [ceil(R/g), ceil(K/g)]).
     """
+    fmax, tdtype = FORMATS[fmt]
     x = np.ascontiguousarray(x, dtype=np.float32)
     R, K = x.shape
     Rb, Kb = -(-R // gran), -(-K // gran)
@@ -69,9 +76,9 @@ def quantize_blocks(x: np.ndarray, gran: int):
     pad[:R, :K] = t
     blocks = pad.view(Rb, gran, Kb, gran)
     amax = blocks.abs().amax(dim=(1, 3))
-    scale = torch.where(amax > 0, amax / E4M3_MAX, torch.ones_like(amax))
-    q = (blocks / scale[:, None, :, None]).clamp(-E4M3_MAX, E4M3_MAX)
-    codes = q.view(Rb * gran, Kb * gran)[:R, :K].to(torch.float8_e4m3fn)
+    scale = torch.where(amax > 0, amax / fmax, torch.ones_like(amax))
+    q = (blocks / scale[:, None, :, None]).clamp(-fmax, fmax)
+    codes = q.view(Rb * gran, Kb * gran)[:R, :K].to(tdtype)
     return codes.view(torch.uint8).numpy().copy(), scale.numpy().astype(np.float32)
 
 
@@ -91,7 +98,8 @@ def b_is_transposed(layout: str) -> bool:
 
 
 def make_problem(M, N, K, gran=128, layout="nt", seed=0, a_dist="normal", b_std=0.02,
-                 outlier_rows=0, outlier_mult=50.0, block_std_log2=None, name=""):
+                 outlier_rows=0, outlier_mult=50.0, block_std_log2=None, name="",
+                 a_fmt="e4m3", b_fmt="e4m3"):
     """Draw A [M,K] and B [N,K] in FP32, quantise per block, store per layout."""
     if layout not in LAYOUTS:
         raise ValueError(f"layout must be one of {LAYOUTS}")
@@ -115,10 +123,10 @@ def make_problem(M, N, K, gran=128, layout="nt", seed=0, a_dist="normal", b_std=
         std = np.exp2(rx.uniform(lo, hi, size=(bm, bk))).astype(np.float32)
         a32 *= np.repeat(np.repeat(std, 128, axis=0), 128, axis=1)[:M, :K]
     b32 = (rb.standard_normal((N, K), dtype=np.float32) * np.float32(b_std))
-    qa, sa = quantize_blocks(a32, gran)
-    qb, sb = quantize_blocks(b32, gran)
+    qa, sa = quantize_blocks(a32, gran, a_fmt)
+    qb, sb = quantize_blocks(b32, gran, b_fmt)
     return Problem(M, N, K, gran, layout, store(qa, a_is_transposed(layout)),
-                   store(qb, b_is_transposed(layout)), sa, sb, name)
+                   store(qb, b_is_transposed(layout)), sa, sb, name, a_fmt, b_fmt)
 
 
 def tiny(seed=0, layout="nt", gran=128):
@@ -160,7 +168,7 @@ def relayout(p: Problem, layout: str) -> Problem:
     """The same logical problem stored in another layout."""
     return Problem(p.M, p.N, p.K, p.gran, layout,
                    store(logical_a(p), a_is_transposed(layout)),
-                   store(logical_b(p), b_is_transposed(layout)), p.sa, p.sb, p.name)
+                   store(logical_b(p), b_is_transposed(layout)), p.sa, p.sb, p.name, p.a_fmt, p.b_fmt)
 
 
 def sample_indices(M, N, count, seed=0, include_corners=True):
