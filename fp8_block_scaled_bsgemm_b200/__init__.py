@@ -43,18 +43,25 @@ class Tuning(ctypes.Structure):
                 ("stream_k", ctypes.c_int)]
 
 
+class Epilogue(ctypes.Structure):
+    _fields_ = [("bias", ctypes.c_void_p), ("activation", ctypes.c_int), ("out_dtype", ctypes.c_int)]
+
+
+ACTIVATIONS = {None: 0, "none": 0, "relu": 1, "gelu": 2}
+
+
 class Plan(ctypes.Structure):
     _fields_ = [(n, ctypes.c_int) for n in ("layout", "gran", "swap_ab", "bnq", "tiles_p", "tiles_q",
                                             "splits", "kb_per_split", "grid", "group_p", "kernels",
                                             "sk_first_tile", "sk_units_per_tile", "sk_ctas", "sk_units",
-                                            "cta_pair")]
+                                            "cta_pair", "grouped")]
 
     def as_dict(self):
         return {n: getattr(self, n) for n, _ in self._fields_}
 
 
 EXPORTS = ("bsgemm_fp8_nt", "bsgemm_fp8_tn", "bsgemm_fp8_nn", "bsgemm_fp8_tt", "bsgemm_fp8_gemm_ex",
-           "bsgemm_fp8_gemm_fmt",
+           "bsgemm_fp8_gemm_fmt", "bsgemm_fp8_gemm_fused", "bsgemm_fp8_grouped_nt",
            "bsgemm_make_plan", "bsgemm_status_string", "bsgemm_get_last_device_status",
            "bsgemm_last_device_status_detail", "bsgemm_diag_wait_timeout", "bsgemm_version",
            "bsgemm_fp8_nt_noalloc", "bsgemm_quantize_fp8")
@@ -81,6 +88,11 @@ def lib():
             L.bsgemm_fp8_gemm_fmt.argtypes = [i32, i32, i32, p, p, p, p, p, i64, i64, i64, i32,
                                               ctypes.POINTER(Tuning), p]
             L.bsgemm_fp8_gemm_fmt.restype = i32
+            L.bsgemm_fp8_gemm_fused.argtypes = [i32, i32, i32, p, p, p, p, ctypes.POINTER(Epilogue), p,
+                                                i64, i64, i64, i32, ctypes.POINTER(Tuning), p]
+            L.bsgemm_fp8_gemm_fused.restype = i32
+            L.bsgemm_fp8_grouped_nt.argtypes = [i32, i32, p, p, p, p, p, p, i32, i64, i64, i64, i32, p]
+            L.bsgemm_fp8_grouped_nt.restype = i32
             L.bsgemm_make_plan.argtypes = [i32, i64, i64, i64, i32, i32, ctypes.POINTER(Tuning),
                                            ctypes.POINTER(Plan)]
             L.bsgemm_make_plan.restype = i32
@@ -151,11 +163,14 @@ def _format(x: torch.Tensor, given, name: str) -> int:
 
 
 def gemm(a, b, scale_a, scale_b, out=None, layout="nt", gran=128, tuning=None, stream=None,
-         a_format=None, b_format=None):
-    """out[M,N] (BF16) of the block-scaled FP8 GEMM; see ``include/bsgemm.h``.
+         a_format=None, b_format=None, bias=None, activation=None, out_dtype=torch.bfloat16):
+    """out[M,N] of the block-scaled FP8 GEMM; see ``include/bsgemm.h``.
 
     ``a_format`` / ``b_format``: "e4m3" or "e5m2"; taken from the tensor's
-    dtype when it is a float8 type, E4M3 for uint8 codes unless given."""
+    dtype when it is a float8 type, E4M3 for uint8 codes unless given.
+    Fused epilogue: out = activation(acc + bias[n]) with ``bias`` an FP32 [N]
+    CUDA tensor or None, ``activation`` None / "relu" / "gelu" (erf form), and
+    ``out_dtype`` torch.bfloat16 or torch.float32."""
     if layout not in LAYOUTS:
         raise ValueError(f"layout must be one of {sorted(LAYOUTS)}")
     fa = _format(a, a_format, "a")
@@ -166,13 +181,24 @@ def gemm(a, b, scale_a, scale_b, out=None, layout="nt", gran=128, tuning=None, s
     for s, nm in ((scale_a, "scale_a"), (scale_b, "scale_b")):
         if s.dtype != torch.float32 or not s.is_cuda or not s.is_contiguous():
             raise ValueError(f"{nm} must be a contiguous float32 CUDA tensor")
+    if out_dtype not in (torch.bfloat16, torch.float32):
+        raise ValueError("out_dtype must be torch.bfloat16 or torch.float32")
+    if activation not in ACTIVATIONS:
+        raise ValueError(f"activation must be one of {sorted(k for k in ACTIVATIONS if k)}")
+    if bias is not None and (bias.dtype != torch.float32 or not bias.is_cuda or not bias.is_contiguous()
+                             or bias.numel() != N):
+        raise ValueError("bias must be a contiguous float32 CUDA tensor of N elements")
     if out is None:
-        out = torch.empty((M, N), dtype=torch.bfloat16, device=a.device)
-    if out.dtype != torch.bfloat16 or tuple(out.shape) != (M, N) or not out.is_contiguous():
-        raise ValueError("out must be a contiguous bfloat16 [M, N] tensor")
-    st = lib().bsgemm_fp8_gemm_fmt(LAYOUTS[layout], fa, fb, a.data_ptr(), b.data_ptr(),
-                                   scale_a.data_ptr(), scale_b.data_ptr(), out.data_ptr(), M, N, K,
-                                   int(gran), _tuning(tuning), _stream_handle(stream))
+        out = torch.empty((M, N), dtype=out_dtype, device=a.device)
+    if out.dtype != out_dtype or tuple(out.shape) != (M, N) or not out.is_contiguous():
+        raise ValueError(f"out must be a contiguous {out_dtype} [M, N] tensor")
+    epi = None
+    if bias is not None or ACTIVATIONS[activation] or out_dtype == torch.float32:
+        epi = ctypes.byref(Epilogue(bias.data_ptr() if bias is not None else None, ACTIVATIONS[activation],
+                                    1 if out_dtype == torch.float32 else 0))
+    st = lib().bsgemm_fp8_gemm_fused(LAYOUTS[layout], fa, fb, a.data_ptr(), b.data_ptr(),
+                                     scale_a.data_ptr(), scale_b.data_ptr(), epi, out.data_ptr(), M, N,
+                                     K, int(gran), _tuning(tuning), _stream_handle(stream))
     if st != 0:
         raise BsgemmError(st, f"bsgemm {layout} M={M} N={N} K={K} g={gran}")
     return out
@@ -216,6 +242,34 @@ def quantize(x: torch.Tensor, gran: int = 128, fmt: str = "e4m3", q=None, scales
     if st != 0:
         raise BsgemmError(st, f"bsgemm_quantize_fp8 {rows}x{cols} g={gran}")
     return q, scales
+
+
+def grouped_gemm(a, b, scale_a, scale_b, group_m, out=None, gran=128, a_format=None, b_format=None,
+                 stream=None):
+    """Grouped NT GEMM: group i multiplies rows R_i .. R_i + M_i - 1 of ``a`` [max_rows, K]
+    by ``b[i]`` ([num_groups, N, K]); ``group_m`` is an int32 CUDA tensor of the M_i.
+    See ``bsgemm_fp8_grouped_nt`` for the scale layouts."""
+    fa = _format(a, a_format, "a")
+    fb = _format(b, b_format, "b")
+    a = _as_bytes(a, "a")
+    b = _as_bytes(b, "b")
+    if a.dim() != 2 or b.dim() != 3 or a.shape[1] != b.shape[2]:
+        raise ValueError("a must be [max_rows, K] and b [num_groups, N, K]")
+    if group_m.dtype != torch.int32 or not group_m.is_cuda or not group_m.is_contiguous() \
+            or group_m.numel() != b.shape[0]:
+        raise ValueError("group_m must be a contiguous int32 CUDA tensor with one entry per group")
+    max_rows, K = a.shape
+    G, N = b.shape[0], b.shape[1]
+    if out is None:
+        out = torch.empty((max_rows, N), dtype=torch.bfloat16, device=a.device)
+    if out.dtype != torch.bfloat16 or tuple(out.shape) != (max_rows, N) or not out.is_contiguous():
+        raise ValueError("out must be a contiguous bfloat16 [max_rows, N] tensor")
+    st = lib().bsgemm_fp8_grouped_nt(fa, fb, a.data_ptr(), b.data_ptr(), scale_a.data_ptr(),
+                                     scale_b.data_ptr(), out.data_ptr(), group_m.data_ptr(), G, max_rows,
+                                     N, K, int(gran), _stream_handle(stream))
+    if st != 0:
+        raise BsgemmError(st, f"bsgemm grouped G={G} max_rows={max_rows} N={N} K={K} g={gran}")
+    return out
 
 
 def scratch_bytes(plan: dict) -> int:

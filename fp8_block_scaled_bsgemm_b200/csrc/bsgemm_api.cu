@@ -290,13 +290,24 @@ extern "C" bsgemm_status bsgemm_make_plan(int layout, int64_t M, int64_t N, int6
 }
 
 // ------------------------------------------------------------------ entry points
-extern "C" bsgemm_status bsgemm_fp8_gemm_fmt(int layout, int a_format, int b_format, const void* a,
-                                             const void* b, const float* scale_a, const float* scale_b,
-                                             void* out, int64_t M, int64_t N, int64_t K, int gran,
-                                             const bsgemm_tuning* tuning, bsgemm_stream_t stream) {
+extern "C" bsgemm_status bsgemm_fp8_gemm_fused(int layout, int a_format, int b_format, const void* a,
+                                               const void* b, const float* scale_a, const float* scale_b,
+                                               const bsgemm_epilogue* epi, void* out, int64_t M, int64_t N,
+                                               int64_t K, int gran, const bsgemm_tuning* tuning,
+                                               bsgemm_stream_t stream) {
   if ((a_format != BSGEMM_FP8_E4M3 && a_format != BSGEMM_FP8_E5M2) ||
       (b_format != BSGEMM_FP8_E4M3 && b_format != BSGEMM_FP8_E5M2))
     return BSGEMM_ERR_INVALID_ARG;
+  bsg_host::CallOpts opts;
+  opts.a_fmt = a_format;
+  opts.b_fmt = b_format;
+  if (epi) {
+    if (epi->activation < BSGEMM_ACT_NONE || epi->activation > BSGEMM_ACT_GELU) return BSGEMM_ERR_INVALID_ARG;
+    if (epi->out_dtype != BSGEMM_OUT_BF16 && epi->out_dtype != BSGEMM_OUT_F32) return BSGEMM_ERR_INVALID_ARG;
+    if (epi->bias && (reinterpret_cast<uintptr_t>(epi->bias) & 3) != 0) return BSGEMM_ERR_MISALIGNED;
+    opts.bias = epi->bias;
+    opts.epi = epi->activation | (epi->out_dtype == BSGEMM_OUT_F32 ? bsg::kEpiOutF32 : 0);
+  }
   bsgemm_status st = check_args(layout, a, b, scale_a, scale_b, out, M, N, K, gran);
   if (st != BSGEMM_OK) return st;
   DeviceInfo dev;
@@ -307,8 +318,7 @@ extern "C" bsgemm_status bsgemm_fp8_gemm_fmt(int layout, int a_format, int b_for
   if (st != BSGEMM_OK) return st;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const int m = static_cast<int>(M), n = static_cast<int>(N), k = static_cast<int>(K);
-#define BSG_RUN(G, L) \
-  bsg_host::run_g##G##_##L(pl, a, b, scale_a, scale_b, out, m, n, k, a_format, b_format, s, dev)
+#define BSG_RUN(G, L) bsg_host::run_g##G##_##L(pl, a, b, scale_a, scale_b, out, m, n, k, opts, s, dev)
 #define BSG_RUN_LAYOUTS(G)                              \
   switch (layout) {                                     \
     case BSGEMM_LAYOUT_NT: return BSG_RUN(G, nt);       \
@@ -323,6 +333,54 @@ extern "C" bsgemm_status bsgemm_fp8_gemm_fmt(int layout, int a_format, int b_for
   }
 #undef BSG_RUN_LAYOUTS
 #undef BSG_RUN
+}
+
+extern "C" bsgemm_status bsgemm_fp8_grouped_nt(int a_format, int b_format, const void* a, const void* b,
+                                               const float* scale_a, const float* scale_b, void* out,
+                                               const int32_t* group_m, int num_groups, int64_t max_rows,
+                                               int64_t N, int64_t K, int gran, bsgemm_stream_t stream) {
+  if ((a_format != BSGEMM_FP8_E4M3 && a_format != BSGEMM_FP8_E5M2) ||
+      (b_format != BSGEMM_FP8_E4M3 && b_format != BSGEMM_FP8_E5M2))
+    return BSGEMM_ERR_INVALID_ARG;
+  if (!group_m || num_groups < 1 || max_rows < 1) return BSGEMM_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(group_m) & 3) != 0) return BSGEMM_ERR_MISALIGNED;
+  bsgemm_status st = check_args(BSGEMM_LAYOUT_NT, a, b, scale_a, scale_b, out, max_rows, N, K, gran);
+  if (st != BSGEMM_OK) return st;
+  if (static_cast<int64_t>(num_groups) * N > (1 << 30)) return BSGEMM_ERR_INVALID_ARG;
+  DeviceInfo dev;
+  st = device_info(dev);
+  if (st != BSGEMM_OK) return st;
+  bsgemm_plan pl{};
+  pl.layout = BSGEMM_LAYOUT_NT;
+  pl.gran = gran;
+  pl.grouped = 1;
+  pl.bnq = N <= 128 ? 128 : 256;
+  pl.tiles_q = static_cast<int>((N + pl.bnq - 1) / pl.bnq);
+  pl.splits = 1;
+  pl.kb_per_split = static_cast<int>((K + gran - 1) / gran);
+  pl.grid = dev.num_sms;
+  pl.group_p = 1;
+  pl.kernels = 1;
+  bsg_host::CallOpts opts;
+  opts.a_fmt = a_format;
+  opts.b_fmt = b_format;
+  opts.group_m = group_m;
+  opts.num_groups = num_groups;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const int m = static_cast<int>(max_rows), n = static_cast<int>(N), k = static_cast<int>(K);
+  switch (gran) {
+    case 64:  return bsg_host::run_g64_nt(pl, a, b, scale_a, scale_b, out, m, n, k, opts, s, dev);
+    case 128: return bsg_host::run_g128_nt(pl, a, b, scale_a, scale_b, out, m, n, k, opts, s, dev);
+    default:  return bsg_host::run_g256_nt(pl, a, b, scale_a, scale_b, out, m, n, k, opts, s, dev);
+  }
+}
+
+extern "C" bsgemm_status bsgemm_fp8_gemm_fmt(int layout, int a_format, int b_format, const void* a,
+                                             const void* b, const float* scale_a, const float* scale_b,
+                                             void* out, int64_t M, int64_t N, int64_t K, int gran,
+                                             const bsgemm_tuning* tuning, bsgemm_stream_t stream) {
+  return bsgemm_fp8_gemm_fused(layout, a_format, b_format, a, b, scale_a, scale_b, nullptr, out, M, N,
+                               K, gran, tuning, stream);
 }
 
 extern "C" bsgemm_status bsgemm_fp8_gemm_ex(int layout, const void* a, const void* b,

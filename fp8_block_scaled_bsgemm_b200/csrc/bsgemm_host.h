@@ -39,11 +39,20 @@ unsigned long long wait_timeout_ns();
 // call; allocates nothing).
 bsgemm_status device_status_address(int** out);
 
-// a_fmt, b_fmt: bsgemm_fp8_format of the logical A and B operands.
+// Per-call options beyond the plan: operand formats and the epilogue.
+struct CallOpts {
+  int a_fmt = BSGEMM_FP8_E4M3;   // bsgemm_fp8_format of the logical A operand
+  int b_fmt = BSGEMM_FP8_E4M3;   // ... and of B
+  const float* bias = nullptr;   // FP32 [N] or null
+  int epi = 0;                   // activation (bits 0-1) | FP32 output (bit 2)
+  const int* group_m = nullptr;  // grouped GEMM: device rows per group
+  int num_groups = 0;
+};
+
 #define BSG_RUN_DECL(G, L)                                                                       \
   bsgemm_status run_g##G##_##L(const bsgemm_plan& plan, const void* a, const void* b,          \
                                const float* sa, const float* sb, void* out, int M, int N, int K, \
-                               int a_fmt, int b_fmt, cudaStream_t stream, const DeviceInfo& dev);
+                               const CallOpts& opts, cudaStream_t stream, const DeviceInfo& dev);
 BSG_RUN_DECL(64, nt) BSG_RUN_DECL(64, tn) BSG_RUN_DECL(64, nn) BSG_RUN_DECL(64, tt)
 BSG_RUN_DECL(128, nt) BSG_RUN_DECL(128, tn) BSG_RUN_DECL(128, nn) BSG_RUN_DECL(128, tt)
 BSG_RUN_DECL(256, nt) BSG_RUN_DECL(256, tn) BSG_RUN_DECL(256, nn) BSG_RUN_DECL(256, tt)

@@ -33,18 +33,19 @@ inline uint32_t fmt_bits(int p_fmt, int q_fmt) {
   return (static_cast<uint32_t>(p_fmt) << 7) | (static_cast<uint32_t>(q_fmt) << 10);
 }
 
-template <int BNQ, int GRAN, bool SWAP, bool P_MN, bool Q_MN, bool SPLIT>
+template <int BNQ, int GRAN, bool SWAP, bool P_MN, bool Q_MN, bool SPLIT, bool GROUPED = false>
 bsgemm_status launch(const bsgemm_plan& plan, const void* a, const void* b, const float* sa,
-                     const float* sb, void* out, int M, int N, int K, int a_fmt, int b_fmt,
+                     const float* sb, void* out, int M, int N, int K, const CallOpts& opts,
                      cudaStream_t stream, const DeviceInfo& dev) {
   using SC = bsg::StageCfg<BNQ, Q_MN, SWAP>;
-  auto kern = bsg::bsgemm_kernel<BNQ, GRAN, SWAP, P_MN, Q_MN, SPLIT>;
+  auto kern = bsg::bsgemm_kernel<BNQ, GRAN, SWAP, P_MN, Q_MN, SPLIT, GROUPED>;
 
   // P/Q operands: normally P = A (M rows), Q = B (N rows); swapped P = B, Q = A
   const void* p_ptr = SWAP ? b : a;
   const void* q_ptr = SWAP ? a : b;
   const int P = SWAP ? N : M;
-  const int Q = SWAP ? M : N;
+  // grouped: B holds num_groups stacked [N, K] matrices
+  const int Q = SWAP ? M : (GROUPED ? N * opts.num_groups : N);
   CUtensorMap tm_p, tm_q;
   bool ok = true;
   if (P_MN) ok &= make_map_2d(&tm_p, p_ptr, CU_TENSOR_MAP_DATA_TYPE_UINT8, P, K, P, 128, bsg::BK);
@@ -56,8 +57,9 @@ bsgemm_status launch(const bsgemm_plan& plan, const void* a, const void* b, cons
   bsg::Params prm{};
   prm.M = M; prm.N = N; prm.K = K;
   prm.Kb = (K + GRAN - 1) / GRAN;
-  prm.Pb = (P + GRAN - 1) / GRAN;
-  prm.Qb = (Q + GRAN - 1) / GRAN;
+  // grouped: sA has ceil(max_rows / g) + num_groups rows, sB ceil(N / g) per group
+  prm.Pb = (P + GRAN - 1) / GRAN + (GROUPED ? opts.num_groups : 0);
+  prm.Qb = ((GROUPED ? N : Q) + GRAN - 1) / GRAN;
   prm.tiles_p = plan.tiles_p;
   prm.tiles_q = plan.tiles_q;
   const int num_tiles = plan.tiles_p * plan.tiles_q;
@@ -70,7 +72,11 @@ bsgemm_status launch(const bsgemm_plan& plan, const void* a, const void* b, cons
   prm.sk_q = plan.sk_ctas > 0 ? plan.sk_units / plan.sk_ctas : 0;
   prm.sk_r = plan.sk_ctas > 0 ? plan.sk_units % plan.sk_ctas : 0;
   prm.group_p = plan.group_p;
-  prm.fmt_bits = SWAP ? fmt_bits(b_fmt, a_fmt) : fmt_bits(a_fmt, b_fmt);
+  prm.fmt_bits = SWAP ? fmt_bits(opts.b_fmt, opts.a_fmt) : fmt_bits(opts.a_fmt, opts.b_fmt);
+  prm.epi = opts.epi;
+  prm.bias = opts.bias;
+  prm.group_m = opts.group_m;
+  prm.num_groups = GROUPED ? opts.num_groups : 0;
   prm.sP = SWAP ? sb : sa;
   prm.sQ = SWAP ? sa : sb;
   prm.out = static_cast<__nv_bfloat16*>(out);
@@ -106,7 +112,7 @@ bsgemm_status launch(const bsgemm_plan& plan, const void* a, const void* b, cons
 // 256 x 256 tiles on CTA pairs (cluster of 2); whole tiles only.
 template <int GRAN, bool P_MN, bool Q_MN>
 bsgemm_status launch_pair(const bsgemm_plan& plan, const void* a, const void* b, const float* sa,
-                          const float* sb, void* out, int M, int N, int K, int a_fmt, int b_fmt,
+                          const float* sb, void* out, int M, int N, int K, const CallOpts& opts,
                           cudaStream_t stream, const DeviceInfo& dev) {
   using PC = bsg::PairCfg;
   auto kern = bsg::bsgemm_pair_kernel<GRAN, P_MN, Q_MN>;
@@ -129,7 +135,9 @@ bsgemm_status launch_pair(const bsgemm_plan& plan, const void* a, const void* b,
   prm.kb_per_split = prm.Kb;
   prm.num_work = plan.tiles_p * plan.tiles_q;
   prm.group_p = plan.group_p;
-  prm.fmt_bits = fmt_bits(a_fmt, b_fmt);
+  prm.fmt_bits = fmt_bits(opts.a_fmt, opts.b_fmt);
+  prm.epi = opts.epi;
+  prm.bias = opts.bias;
   prm.sP = sa;
   prm.sQ = sb;
   prm.out = static_cast<__nv_bfloat16*>(out);
@@ -174,28 +182,37 @@ bsgemm_status launch_pair(const bsgemm_plan& plan, const void* a, const void* b,
 
 bsgemm_status BSG_RUN_NAME(BSG_GRAN, BSG_LAYOUT)(const bsgemm_plan& pl, const void* a, const void* b,
                                                  const float* sa, const float* sb, void* out, int M,
-                                                 int N, int K, int fa, int fb, cudaStream_t s,
+                                                 int N, int K, const CallOpts& o, cudaStream_t s,
                                                  const DeviceInfo& d) {
   constexpr int G = BSG_GRAN;
-  if (pl.cta_pair) return launch_pair<G, kAMn, kBMn>(pl, a, b, sa, sb, out, M, N, K, fa, fb, s, d);
+  if (pl.grouped) {
+    // grouped GEMM: NT only, whole tiles
+    if constexpr (!kAMn && !kBMn) {
+      if (pl.bnq == 128) return launch<128, G, false, false, false, false, true>(pl, a, b, sa, sb, out, M, N, K, o, s, d);
+      return launch<256, G, false, false, false, false, true>(pl, a, b, sa, sb, out, M, N, K, o, s, d);
+    } else {
+      return BSGEMM_ERR_INVALID_ARG;
+    }
+  }
+  if (pl.cta_pair) return launch_pair<G, kAMn, kBMn>(pl, a, b, sa, sb, out, M, N, K, o, s, d);
   if (pl.swap_ab) {
     // P = B, Q = A
     switch (pl.bnq) {
-      case 16:  return launch<16, G, true, kBMn, kAMn, true>(pl, a, b, sa, sb, out, M, N, K, fa, fb, s, d);
-      case 32:  return launch<32, G, true, kBMn, kAMn, true>(pl, a, b, sa, sb, out, M, N, K, fa, fb, s, d);
-      case 64:  return launch<64, G, true, kBMn, kAMn, true>(pl, a, b, sa, sb, out, M, N, K, fa, fb, s, d);
-      case 128: return launch<128, G, true, kBMn, kAMn, true>(pl, a, b, sa, sb, out, M, N, K, fa, fb, s, d);
+      case 16:  return launch<16, G, true, kBMn, kAMn, true>(pl, a, b, sa, sb, out, M, N, K, o, s, d);
+      case 32:  return launch<32, G, true, kBMn, kAMn, true>(pl, a, b, sa, sb, out, M, N, K, o, s, d);
+      case 64:  return launch<64, G, true, kBMn, kAMn, true>(pl, a, b, sa, sb, out, M, N, K, o, s, d);
+      case 128: return launch<128, G, true, kBMn, kAMn, true>(pl, a, b, sa, sb, out, M, N, K, o, s, d);
       default:  return BSGEMM_ERR_INVALID_ARG;
     }
   }
   const bool split = pl.splits > 1 || pl.sk_ctas > 0;
   switch (pl.bnq) {
     case 128:
-      return split ? launch<128, G, false, kAMn, kBMn, true>(pl, a, b, sa, sb, out, M, N, K, fa, fb, s, d)
-                   : launch<128, G, false, kAMn, kBMn, false>(pl, a, b, sa, sb, out, M, N, K, fa, fb, s, d);
+      return split ? launch<128, G, false, kAMn, kBMn, true>(pl, a, b, sa, sb, out, M, N, K, o, s, d)
+                   : launch<128, G, false, kAMn, kBMn, false>(pl, a, b, sa, sb, out, M, N, K, o, s, d);
     case 256:
-      return split ? launch<256, G, false, kAMn, kBMn, true>(pl, a, b, sa, sb, out, M, N, K, fa, fb, s, d)
-                   : launch<256, G, false, kAMn, kBMn, false>(pl, a, b, sa, sb, out, M, N, K, fa, fb, s, d);
+      return split ? launch<256, G, false, kAMn, kBMn, true>(pl, a, b, sa, sb, out, M, N, K, o, s, d)
+                   : launch<256, G, false, kAMn, kBMn, false>(pl, a, b, sa, sb, out, M, N, K, o, s, d);
     default:
       return BSGEMM_ERR_INVALID_ARG;
   }

@@ -88,9 +88,13 @@ struct Params {
                          // sk_r CTAs take sk_q + 1 of them, the others sk_q
   int group_p;           // raster group height in P tiles (L2 locality)
   uint32_t fmt_bits;     // instruction-descriptor format fields of P and Q (E4M3 0, E5M2 1)
+  int epi;               // epilogue: activation (bits 0-1: 0 none, 1 ReLU, 2 GELU), bit 2 FP32 output
+  int num_groups;        // grouped GEMM: number of groups (0 otherwise)
+  const float* bias;     // FP32 [N] added before the activation, or null
+  const int* group_m;    // grouped GEMM: rows of each group (device, num_groups entries)
   const float* sP;       // [Pb][Kb]
   const float* sQ;       // [Qb][Kb]
-  __nv_bfloat16* out;    // [M][N] row-major (direct stores in swap mode)
+  __nv_bfloat16* out;    // [M][N] row-major, BF16 (FP32 when epi bit 2 is set)
   float* ws;             // partial tiles [slot][BNQ][BM]: split-K slot tile*splits+split,
                          // stream-K slot 2*cta + (0: the CTA's first tile, 1: its last)
   int* counters;         // one per split or stream-K tile, zero between launches
@@ -200,6 +204,9 @@ __device__ __forceinline__ constexpr uint32_t instr_desc() {
 
 struct Work {
   int tile, tp, tq, kb0, kb1;  // output tile and its K-blocks [kb0, kb1)
+  // grouped GEMM (zero / unused otherwise): the group's first row in A, out
+  // and its first scale row in sA, its first row in B and in sB, its rows
+  int g_row, g_srow, g_qrow, g_sqrow, g_rows;
 };
 
 // Tile index -> (P tile, Q tile) in grouped raster order: group_p P-tiles
@@ -233,19 +240,65 @@ __device__ __forceinline__ int sk_owner(const Params& p, int u) {
 struct WorkIter {
   int wi;  // next whole-tile / split-K item
   int u;   // next stream-K unit
+  // grouped GEMM cursor: current group, its first tile, rows, tiles, first
+  // row and first scale row
+  int g, g_first, g_m, g_tiles, g_row, g_srow;
 };
 
-template <bool SPLIT>
+// Grouped GEMM: advance the cursor to the group that holds tile it.wi (tiles
+// are numbered group by group; each group has ceil(rows / 128) x tiles_q).
+// Returns false once every group is used up.
+template <int GRAN>
+__device__ __forceinline__ bool group_seek(const Params& p, WorkIter& it) {
+  while (it.wi >= it.g_first + it.g_tiles) {
+    it.g_first += it.g_tiles;
+    it.g_row += it.g_m;
+    it.g_srow += (it.g_m + GRAN - 1) / GRAN;
+    if (++it.g >= p.num_groups) return false;
+    it.g_m = max(0, __ldg(p.group_m + it.g));
+    it.g_tiles = (it.g_m + BM - 1) / BM * p.tiles_q;
+  }
+  return true;
+}
+
+template <bool SPLIT, bool GROUPED = false>
 __device__ __forceinline__ void work_begin(const Params& p, WorkIter& it) {
   it.wi = blockIdx.x;
   it.u = 0;
   if (SPLIT && static_cast<int>(blockIdx.x) < p.sk_ctas) it.u = sk_start(p, blockIdx.x);
+  if constexpr (GROUPED) {
+    it.g = 0;
+    it.g_first = 0;
+    it.g_row = 0;
+    it.g_srow = 0;
+    it.g_m = max(0, __ldg(p.group_m));
+    it.g_tiles = (it.g_m + BM - 1) / BM * p.tiles_q;
+  }
 }
 
 // Instances without the partial-tile fix-up (SPLIT false) never get a
 // stream-K range, so their walk is the whole-tile loop alone.
-template <int GRAN, bool SPLIT>
+template <int GRAN, bool SPLIT, bool GROUPED = false>
 __device__ __forceinline__ bool work_next(const Params& p, WorkIter& it, Work& w) {
+  if constexpr (GROUPED) {
+    // whole tiles, group by group; within a group the P (row) tile varies
+    // fastest, so CTAs running together share the group's B tiles
+    if (!group_seek<GRAN>(p, it)) return false;
+    const int lt = it.wi - it.g_first;
+    const int tiles_p = (it.g_m + BM - 1) / BM;
+    w.tile = it.wi;
+    w.tp = lt % tiles_p;
+    w.tq = lt / tiles_p;
+    w.kb0 = 0;
+    w.kb1 = p.Kb;
+    w.g_row = it.g_row;
+    w.g_srow = it.g_srow;
+    w.g_qrow = it.g * p.N;
+    w.g_sqrow = it.g * p.Qb;
+    w.g_rows = it.g_m;
+    it.wi += gridDim.x;
+    return true;
+  }
   if (it.wi < p.num_work) {
     w.tile = it.wi / p.splits;
     const int split = it.wi - w.tile * p.splits;
@@ -340,8 +393,63 @@ __device__ __forceinline__ void stage_range(const Params& p, const Work& w, int&
   if (st1 > nst) st1 = nst;
 }
 
+// ---------------------------------------------------------------- epilogue
+// out = act(acc + bias[n]), the pages' fused-epilogue extension point
+// (hncyxsy.com/news/191052 §2.3, §6). GELU is the erf form,
+// 0.5 v (1 + erf(v / sqrt 2)).
+constexpr int kEpiRelu = 1, kEpiGelu = 2, kEpiOutF32 = 4;
+
+__device__ __forceinline__ float epi_act(float v, int act) {
+  if (act == kEpiRelu) return fmaxf(v, 0.f);
+  if (act == kEpiGelu) return 0.5f * v * (1.0f + erff(v * 0.70710678118654752f));
+  return v;
+}
+
+// One thread's run of columns [n0, n0 + 2 * NP) of row m: acc pairs in
+// column order. Applies the epilogue in place and stores BF16 (8 per 16-byte
+// store) or FP32 (4 per 16-byte store); N % 8 == 0, so a group of 8 columns
+// is wholly inside or outside the matrix.
+template <int NP>
+__device__ __forceinline__ void store_row_run(const Params& p, int m, int n0, float2 (&acc)[NP]) {
+  const int act = p.epi & 3;
+  if (p.bias != nullptr || act != 0) {
+#pragma unroll
+    for (int i = 0; i < NP; ++i) {
+      const int n = n0 + 2 * i;
+      float b0 = 0.f, b1 = 0.f;
+      if (p.bias != nullptr && n < p.N) {
+        b0 = __ldg(p.bias + n);
+        b1 = __ldg(p.bias + n + 1);
+      }
+      acc[i].x = epi_act(acc[i].x + b0, act);
+      acc[i].y = epi_act(acc[i].y + b1, act);
+    }
+  }
+  if (p.epi & kEpiOutF32) {
+    float* row = reinterpret_cast<float*>(p.out) + static_cast<size_t>(m) * p.N + n0;
+#pragma unroll
+    for (int c = 0; c < NP / 2; ++c)
+      if (n0 + c * 4 < p.N)
+        *reinterpret_cast<float4*>(row + c * 4) =
+            make_float4(acc[2 * c].x, acc[2 * c].y, acc[2 * c + 1].x, acc[2 * c + 1].y);
+  } else {
+    __nv_bfloat16* row = p.out + static_cast<size_t>(m) * p.N + n0;
+#pragma unroll
+    for (int c = 0; c < NP / 4; ++c) {
+      if (n0 + c * 8 < p.N) {
+        uint4 v;
+        v.x = pack_bf16x2(acc[c * 4].x, acc[c * 4].y);
+        v.y = pack_bf16x2(acc[c * 4 + 1].x, acc[c * 4 + 1].y);
+        v.z = pack_bf16x2(acc[c * 4 + 2].x, acc[c * 4 + 2].y);
+        v.w = pack_bf16x2(acc[c * 4 + 3].x, acc[c * 4 + 3].y);
+        *reinterpret_cast<uint4*>(row + c * 8) = v;
+      }
+    }
+  }
+}
+
 // ---------------------------------------------------------------- kernel
-template <int BNQ, int GRAN, bool SWAP, bool P_MN, bool Q_MN, bool SPLIT>
+template <int BNQ, int GRAN, bool SWAP, bool P_MN, bool Q_MN, bool SPLIT, bool GROUPED = false>
 __global__ void __launch_bounds__(kNumThreads, 1)
     bsgemm_kernel(const __grid_constant__ CUtensorMap tm_p, const __grid_constant__ CUtensorMap tm_q,
                   const Params p) {
@@ -409,8 +517,8 @@ __global__ void __launch_bounds__(kNumThreads, 1)
       uint32_t it = 0;  // stage-slot uses so far
       bool ok = true;
       WorkIter wit;
-      work_begin<SPLIT>(p, wit);
-      for (Work w; ok && work_next<GRAN, SPLIT>(p, wit, w);) {
+      work_begin<SPLIT, GROUPED>(p, wit);
+      for (Work w; ok && work_next<GRAN, SPLIT, GROUPED>(p, wit, w);) {
         int st0, st1;
         stage_range<GRAN>(p, w, st0, st1);
         for (int st = st0; st < st1; ++st, ++it) {
@@ -422,14 +530,16 @@ __global__ void __launch_bounds__(kNumThreads, 1)
           const uint32_t pd = smem_addr(p_tiles + s * TL::kPBytes);
           const uint32_t qd = smem_addr(q_tiles + s * TL::kQBytes);
           const int k = st * BK;
-          if constexpr (P_MN) tma_load_2d(pd, &tm_p, fb, w.tp * BM, k);
-          else                tma_load_2d(pd, &tm_p, fb, k, w.tp * BM);
+          const int prow = (GROUPED ? w.g_row : 0) + w.tp * BM;
+          const int qrow = (GROUPED ? w.g_qrow : 0) + w.tq * BNQ;
+          if constexpr (P_MN) tma_load_2d(pd, &tm_p, fb, prow, k);
+          else                tma_load_2d(pd, &tm_p, fb, k, prow);
           if constexpr (Q_MN) {
 #pragma unroll
             for (int c = 0; c < TL::kQRows / 128; ++c)
-              tma_load_2d(qd + c * 128 * BK, &tm_q, fb, w.tq * BNQ + c * 128, k);
+              tma_load_2d(qd + c * 128 * BK, &tm_q, fb, qrow + c * 128, k);
           } else {
-            tma_load_2d(qd, &tm_q, fb, k, w.tq * BNQ);
+            tma_load_2d(qd, &tm_q, fb, k, qrow);
           }
         }
       }
@@ -464,8 +574,8 @@ __global__ void __launch_bounds__(kNumThreads, 1)
       uint32_t b = 0, bph = 0;    // TMEM buffer and its phase
       bool ok = true;
       WorkIter wit;
-      work_begin<SPLIT>(p, wit);
-      for (Work w; ok && work_next<GRAN, SPLIT>(p, wit, w);) {
+      work_begin<SPLIT, GROUPED>(p, wit);
+      for (Work w; ok && work_next<GRAN, SPLIT, GROUPED>(p, wit, w);) {
         for (int kb = w.kb0; kb < w.kb1; ++kb) {
           // Order of the waits: the stage's operands first (normally already
           // loaded, so that wait is cheap and happens while the tensor pipe
@@ -540,8 +650,8 @@ __global__ void __launch_bounds__(kNumThreads, 1)
     float2 acc[kHalf / 2];    // this thread's row, columns [half*kHalf, (half+1)*kHalf)
 
     WorkIter wit;
-    work_begin<SPLIT>(p, wit);
-    for (Work w; ok && work_next<GRAN, SPLIT>(p, wit, w);) {
+    work_begin<SPLIT, GROUPED>(p, wit);
+    for (Work w; ok && work_next<GRAN, SPLIT, GROUPED>(p, wit, w);) {
       if constexpr (SPLIT) {
         // where this item's partial goes: worked out while the accumulator
         // is dead and parked in shared memory (registers are short during
@@ -561,12 +671,19 @@ __global__ void __launch_bounds__(kNumThreads, 1)
       // scale rows for this warp: one P block, kNumGroups Q blocks (clamped:
       // rows past the end of P/Q hold zeros and are never stored)
       int pb = (w.tp * BM + quad * 32) / GRAN;
-      pb = pb < p.Pb - 1 ? pb : p.Pb - 1;
       int qb[kNumGroups];
+      if constexpr (GROUPED) {
+        // the group's own scale rows (clamped inside the group and inside sA)
+        const int last = max(0, (w.g_rows - 1) / GRAN);
+        pb = w.g_srow + (pb < last ? pb : last);
+        pb = pb < p.Pb - 1 ? pb : p.Pb - 1;
+      } else {
+        pb = pb < p.Pb - 1 ? pb : p.Pb - 1;
+      }
 #pragma unroll
       for (int j = 0; j < kNumGroups; ++j) {
         const int b = (w.tq * BNQ + half * kHalf + j * kGroupCols) / GRAN;
-        qb[j] = b < p.Qb - 1 ? b : p.Qb - 1;
+        qb[j] = (b < p.Qb - 1 ? b : p.Qb - 1) + (GROUPED ? w.g_sqrow : 0);
       }
       const float* sp_row = p.sP + static_cast<size_t>(pb) * p.Kb;
       // lane i holds sP*sQ of K-block (chunk base + i); the next chunk is in flight
@@ -678,37 +795,29 @@ __global__ void __launch_bounds__(kNumThreads, 1)
         }
       }
 
-      // ---------------------------------------------------------- BF16 store
+      // ---------------------------------------------------------- epilogue + store
       if constexpr (SWAP) {
         // tile rows are N, tile columns are M: out[m][n]
         const int n = w.tp * BM + row_in_tile;
         if (n < p.N) {
+          const int act = p.epi & 3;
+          const float bn = p.bias != nullptr ? __ldg(p.bias + n) : 0.f;
 #pragma unroll
           for (int i = 0; i < kHalf; ++i) {
             const int m = w.tq * BNQ + half * kHalf + i;
-            const float v = (i & 1) ? acc[i / 2].y : acc[i / 2].x;
-            if (m < p.M) p.out[static_cast<size_t>(m) * p.N + n] = __float2bfloat16_rn(v);
-          }
-        }
-      } else {
-        // this thread owns row m, columns [n0, n0 + kHalf): 16-byte stores of
-        // 8 BF16 values (N % 8 == 0, so a group is either all in or all out)
-        const int m = w.tp * BM + row_in_tile;
-        const int n0 = w.tq * BNQ + half * kHalf;
-        if (m < p.M) {
-          __nv_bfloat16* row = p.out + static_cast<size_t>(m) * p.N + n0;
-#pragma unroll
-          for (int c = 0; c < kHalf / 8; ++c) {
-            if (n0 + c * 8 < p.N) {
-              uint4 v;
-              v.x = pack_bf16x2(acc[c * 4].x, acc[c * 4].y);
-              v.y = pack_bf16x2(acc[c * 4 + 1].x, acc[c * 4 + 1].y);
-              v.z = pack_bf16x2(acc[c * 4 + 2].x, acc[c * 4 + 2].y);
-              v.w = pack_bf16x2(acc[c * 4 + 3].x, acc[c * 4 + 3].y);
-              *reinterpret_cast<uint4*>(row + c * 8) = v;
+            const float v = epi_act(((i & 1) ? acc[i / 2].y : acc[i / 2].x) + bn, act);
+            if (m < p.M) {
+              if (p.epi & kEpiOutF32) reinterpret_cast<float*>(p.out)[static_cast<size_t>(m) * p.N + n] = v;
+              else p.out[static_cast<size_t>(m) * p.N + n] = __float2bfloat16_rn(v);
             }
           }
         }
+      } else {
+        // this thread owns row m, columns [n0, n0 + kHalf)
+        const int m_local = w.tp * BM + row_in_tile;
+        const int m = (GROUPED ? w.g_row : 0) + m_local;
+        const int n0 = w.tq * BNQ + half * kHalf;
+        if (m < p.M && (!GROUPED || m_local < w.g_rows)) store_row_run<kHalf / 2>(p, m, n0, acc);
       }
     }
   }

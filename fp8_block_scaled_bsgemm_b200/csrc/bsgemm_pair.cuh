@@ -301,23 +301,10 @@ __global__ void __launch_bounds__(kNumThreads, 1)
       }
       if (!ok) break;
 
-      // ---------------------------------------------------------- BF16 store
+      // ---------------------------------------------------------- epilogue + store
       const int m = prow0 + row_in_tile;
       const int n0 = tq * kPairN + half * kHalf;
-      if (m < p.M) {
-        __nv_bfloat16* row = p.out + static_cast<size_t>(m) * p.N + n0;
-#pragma unroll
-        for (int c = 0; c < kHalf / 8; ++c) {
-          if (n0 + c * 8 < p.N) {
-            uint4 v;
-            v.x = pack_bf16x2(acc[c * 4].x, acc[c * 4].y);
-            v.y = pack_bf16x2(acc[c * 4 + 1].x, acc[c * 4 + 1].y);
-            v.z = pack_bf16x2(acc[c * 4 + 2].x, acc[c * 4 + 2].y);
-            v.w = pack_bf16x2(acc[c * 4 + 3].x, acc[c * 4 + 3].y);
-            *reinterpret_cast<uint4*>(row + c * 8) = v;
-          }
-        }
-      }
+      if (m < p.M) store_row_run<kHalf / 2>(p, m, n0, acc);
     }
   }
   __syncwarp();

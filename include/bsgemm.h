@@ -145,6 +145,7 @@ typedef struct {
     int sk_units;       /* stream-K: units of all stream-K tiles together */
     int cta_pair;       /* 1: 256 x 256 tiles on CTA pairs (tiles_p, tiles_q count those;
                            grid counts CTAs, two per pair) */
+    int grouped;        /* 1: grouped GEMM (tiles_p is per group, found on the device) */
 } bsgemm_plan;
 
 /* FP8 formats of the operands (hncyxsy.com/news/191052 §2.2 names both).
@@ -201,6 +202,68 @@ typedef enum {
 bsgemm_status bsgemm_quantize_fp8(int src_dtype, int fp8_format, const void *x, int64_t rows,
                                   int64_t cols, int gran, void *q, float *scales,
                                   bsgemm_stream_t stream);
+
+/* ---- fused epilogue -------------------------------------------------------
+ * The pages' extension point for work fused before write-back (§2.3, §6):
+ *   out[m,n] = act(acc[m,n] + bias[n])
+ * where acc is the block-scaled product in FP32, bias an optional FP32 [N]
+ * vector, and act one of: none, ReLU (max(v, 0)), GELU in its erf form
+ * (0.5 v (1 + erf(v / sqrt 2))). The result is stored as BF16 (round to
+ * nearest even) or FP32 [M,N] row-major. With split-K or stream-K the
+ * epilogue runs once, after the pieces are summed. */
+typedef enum {
+    BSGEMM_ACT_NONE = 0,
+    BSGEMM_ACT_RELU = 1,
+    BSGEMM_ACT_GELU = 2
+} bsgemm_activation;
+
+typedef enum {
+    BSGEMM_OUT_BF16 = 0,
+    BSGEMM_OUT_F32 = 1
+} bsgemm_out_dtype;
+
+typedef struct {
+    const float *bias; /* device FP32 [N], 4-byte aligned, or NULL */
+    int activation;    /* bsgemm_activation */
+    int out_dtype;     /* bsgemm_out_dtype: the element type of out */
+} bsgemm_epilogue;
+
+/* bsgemm_fp8_gemm_fmt with a fused epilogue (NULL = none: BF16 output).
+ * out must be [M,N] of epi->out_dtype; same alignment rules (16-byte base,
+ * N % 8 == 0). Unknown activation or out_dtype -> BSGEMM_ERR_INVALID_ARG,
+ * misaligned bias -> BSGEMM_ERR_MISALIGNED. */
+bsgemm_status bsgemm_fp8_gemm_fused(int layout, int a_format, int b_format, const void *a,
+                                    const void *b, const float *scale_a, const float *scale_b,
+                                    const bsgemm_epilogue *epi, void *out, int64_t M, int64_t N,
+                                    int64_t K, int gran, const bsgemm_tuning *tuning,
+                                    bsgemm_stream_t stream);
+
+/* ---- grouped GEMM ---------------------------------------------------------
+ * Many independent NT products in one persistent launch, the pages' "batch
+ * of matrices with different shapes" (§2.1) for a shared N and K, e.g. one
+ * weight matrix per expert and a variable number of rows per expert:
+ *   for group i with M_i = group_m[i] rows (M_i >= 0):
+ *     out_i[M_i, N] = block-scaled product of A_i [M_i, K] and B_i [N, K]
+ * Storage (all device memory owned by the caller):
+ *   a       [max_rows, K] codes; group i's rows start at row R_i = sum_{j<i} M_j
+ *   scale_a FP32 [S_rows, Kb] with group i's blocks starting at row
+ *           S_i = sum_{j<i} ceil(M_j / gran); S_rows >= ceil(max_rows / gran)
+ *           + num_groups covers every split of max_rows into groups
+ *   b       [num_groups, N, K] codes; scale_b FP32 [num_groups, ceil(N/gran), Kb]
+ *   out     [max_rows, N] BF16; rows R_i .. R_i + M_i - 1 are written, the
+ *           rest untouched
+ *   group_m int32 [num_groups] on the device, read by the kernel (so sizes
+ *           produced on the GPU need no copy to the host)
+ * sum M_i must not exceed max_rows: rows past max_rows are neither read
+ * (they load as zeros) nor written, and scale reads stay inside the S_rows
+ * bound above. The scale blocks never straddle groups.
+ * Errors as bsgemm_fp8_gemm_fmt, plus BSGEMM_ERR_INVALID_ARG for
+ * num_groups < 1 or max_rows < 1, BSGEMM_ERR_MISALIGNED for a group_m
+ * pointer that is not 4-byte aligned. */
+bsgemm_status bsgemm_fp8_grouped_nt(int a_format, int b_format, const void *a, const void *b,
+                                    const float *scale_a, const float *scale_b, void *out,
+                                    const int32_t *group_m, int num_groups, int64_t max_rows,
+                                    int64_t N, int64_t K, int gran, bsgemm_stream_t stream);
 
 /* Host-only: the plan a call with these sizes would use on a device with
  * `num_sms` SMs. Touches no device. */

@@ -70,6 +70,8 @@ def _load():
             lib.oracle_fp8_encode.argtypes = [i32, ctypes.c_float]
             lib.oracle_quantize_blocks.restype = ctypes.c_int
             lib.oracle_quantize_blocks.argtypes = [i32, p, i64, i64, i64, p, p]
+            lib.oracle_epilogue.restype = ctypes.c_int
+            lib.oracle_epilogue.argtypes = [p, i64, i64, p, i32, p, p]
             lib.oracle_num_threads.restype = ctypes.c_int
             lib.oracle_num_threads.argtypes = []
             _lib = lib
@@ -173,3 +175,22 @@ def quantize_blocks(x, gran: int, fmt: str = "e4m3"):
     if rc != 0:
         raise RuntimeError(f"oracle_quantize_blocks failed with code {rc}")
     return q, s
+
+
+ACTIVATIONS = {None: 0, "none": 0, "relu": 1, "gelu": 2}
+
+
+def epilogue(ref, bias=None, activation=None):
+    """act(ref + bias[n]) in FP64 on an FP64 [M,N] product. Returns (value float64, bf16 bits uint16)."""
+    ref = np.ascontiguousarray(ref, dtype=np.float64)
+    M, N = ref.shape
+    b = None if bias is None else np.ascontiguousarray(bias, dtype=np.float32)
+    if b is not None and b.size != N:
+        raise ValueError("bias must have N elements")
+    v = np.empty((M, N), dtype=np.float64)
+    out = np.empty((M, N), dtype=np.uint16)
+    rc = _load().oracle_epilogue(_ptr(ref), M, N, None if b is None else _ptr(b), ACTIVATIONS[activation],
+                                 _ptr(v), _ptr(out))
+    if rc != 0:
+        raise RuntimeError(f"oracle_epilogue failed with code {rc}")
+    return v, out

@@ -389,3 +389,27 @@ int oracle_quantize_blocks(int fmt, const float *x, int64_t rows, int64_t cols, 
     }
     return OR_OK;
 }
+
+/* ---- fused epilogue (§2.3, §6: bias and activation applied before the
+ * result is written back) ----------------------------------------------------
+ *   v[m,n] = act(ref[m,n] + bias[n])      in FP64, bias may be NULL
+ *   act: 0 none, 1 ReLU = max(v, 0), 2 GELU = 0.5 v (1 + erf(v / sqrt 2))
+ * epi_ref receives v (FP64); out receives bf16_rne(v) (may be NULL).      */
+int oracle_epilogue(const double *ref, int64_t M, int64_t N, const float *bias, int act,
+                    double *epi_ref, uint16_t *out)
+{
+    if (!ref || !epi_ref || M <= 0 || N <= 0 || act < 0 || act > 2)
+        return OR_ERR_ARG;
+    for (int64_t m = 0; m < M; ++m)
+        for (int64_t n = 0; n < N; ++n) {
+            double v = ref[m * N + n] + (bias ? (double)bias[n] : 0.0);
+            if (act == 1)
+                v = v > 0.0 ? v : 0.0;
+            else if (act == 2)
+                v = 0.5 * v * (1.0 + erf(v / sqrt(2.0)));
+            epi_ref[m * N + n] = v;
+            if (out)
+                out[m * N + n] = oracle_bf16_rne(v);
+        }
+    return OR_OK;
+}

@@ -162,7 +162,7 @@ def test_register_split_kernels_have_the_planned_launch_registers():
     bsg_build.build()
     logs = glob.glob(os.path.join(ROOT, "_build", "bsgemm_inst_g*.log"))
     assert len(logs) == 12
-    seen = 0
+    seen = pairs = 0
     for log in logs:
         cur = None
         for ln in open(log):
@@ -170,11 +170,18 @@ def test_register_split_kernels_have_the_planned_launch_registers():
             if m:
                 cur = int(m.group(1))
                 continue
+            if "Compiling entry function '_ZN3bsg18bsgemm_pair_kernel" in ln:
+                cur = -1   # CTA-pair tiles: always the 256-wide register split
+                continue
             if cur is not None and "Used" in ln:
                 regs = int(re.search(r"Used (\d+) registers", ln).group(1))
-                if cur == 256:
+                if cur in (256, -1):
                     assert regs == 168, (log, ln)
-                    seen += 1
+                    seen += cur == 256
+                    pairs += cur == -1
                 assert regs <= 168
                 cur = None
-    assert seen == 24   # 12 (granularity, layout) units x {split, no split}
+    # 12 (granularity, layout) units x {split, no split}, plus the grouped
+    # instance in each of the 3 NT units; one CTA-pair kernel per unit
+    assert seen == 24 + 3
+    assert pairs == 12

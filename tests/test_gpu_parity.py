@@ -151,6 +151,50 @@ def test_e5m2_binding_takes_format_from_dtype():
         bsg.gemm(a.view(torch.float8_e5m2), b, sa, sb, a_format="e4m3")
 
 
+# ---------------------------------------------------------------- fused epilogue (§2.3, §6)
+@pytest.mark.parametrize("activation", [None, "relu", "gelu"])
+@pytest.mark.parametrize("out_dtype", [torch.bfloat16, torch.float32])
+@pytest.mark.parametrize("tuning,M,layout", [
+    (None, 400, "nt"),
+    ({"variant": "swap_ab", "bnq": 64, "splits": 3}, 48, "tn"),
+    ({"variant": "data_parallel", "bnq": 128, "stream_k": 1}, 640, "nn"),
+    ({"variant": "cta_pair"}, 528, "tt"),
+])
+def test_fused_epilogue(activation, out_dtype, tuning, M, layout):
+    """out = act(acc + bias[n]) stored as BF16 or FP32, against the oracle's FP64 epilogue."""
+    p = workloads.make_problem(M, 784, 1280, 128, layout, seed=31)
+    rng = np.random.default_rng(32)
+    bias = (rng.standard_normal(784) * 0.5).astype(np.float32)
+    a, b, sa, sb = to_device(p)
+    out = bsg.gemm(a, b, sa, sb, layout=layout, gran=128, tuning=tuning, bias=torch.from_numpy(bias).cuda(),
+                   activation=activation, out_dtype=out_dtype)
+    torch.cuda.synchronize()
+    ref, _ = oracle.bsgemm(layout, p.a, p.b, p.sa, p.sb, p.M, p.N, p.K, 128)
+    want, bits = oracle.epilogue(ref, bias, activation)
+    assert out.dtype == out_dtype
+    check_close(gpu_as_f64(out), want, f"epilogue {activation} {out_dtype} {tuning}")
+
+
+def test_fused_epilogue_fp32_output_without_bias_keeps_fp32_precision():
+    """FP32 output: the values before BF16 rounding, so the error is the FP32
+    accumulation's alone -- far inside the BF16 tolerance."""
+    p = workloads.make_problem(256, 512, 1024, 128, "nt", seed=33)
+    a, b, sa, sb = to_device(p)
+    out = bsg.gemm(a, b, sa, sb, out_dtype=torch.float32)
+    ref, _ = oracle.bsgemm("nt", p.a, p.b, p.sa, p.sb, p.M, p.N, p.K, 128)
+    got = gpu_as_f64(out)
+    assert np.max(np.abs(got - ref) / (np.abs(ref) + 1e-3 * np.sqrt(np.mean(ref ** 2)))) < 2.0 ** -12
+
+
+def test_fused_epilogue_argument_errors():
+    p = workloads.make_problem(128, 256, 256, 128, "nt", seed=34)
+    a, b, sa, sb = to_device(p)
+    with pytest.raises(ValueError):
+        bsg.gemm(a, b, sa, sb, activation="tanh")
+    with pytest.raises(ValueError):
+        bsg.gemm(a, b, sa, sb, bias=torch.zeros(255, device="cuda"))
+
+
 # ---------------------------------------------------------------- small M (decode-style)
 @pytest.mark.parametrize("M", [1, 8, 32, 64, 128])
 def test_small_m_reduced_k(M):

@@ -450,3 +450,33 @@ def test_oracle_quantiser_round_trip_error():
     back = oracle.e4m3_table()[q] * np.repeat(np.repeat(s, 128, 0), 128, 1)
     # E4M3 keeps 4 significant bits: relative error <= 2^-4 above the subnormal range
     assert np.all(np.abs(back - x) <= 2.0 ** -4 * np.abs(x) + np.repeat(np.repeat(s, 128, 0), 128, 1) * 2.0 ** -9)
+
+
+# --------------------------------------------------------------------------- fused epilogue (§2.3, §6)
+def test_epilogue_hand_values():
+    ref = np.array([[-2.0, -0.5, 0.0, 0.5, 1.0, 3.0]])
+    bias = np.array([0.0, 0.0, 0.0, 0.25, -1.0, 0.0], np.float32)
+    v, _ = oracle.epilogue(ref, bias, "relu")
+    assert v.tolist() == [[0.0, 0.0, 0.0, 0.75, 0.0, 3.0]]
+    v, _ = oracle.epilogue(ref, None, "gelu")
+    want = [0.5 * x * (1.0 + math.erf(x / math.sqrt(2.0))) for x in ref[0]]
+    assert np.allclose(v[0], want, rtol=0, atol=1e-15)
+    assert abs(v[0, 4] - 0.8413447460685429) < 1e-15          # GELU(1) = Phi(1)
+    v, bits = oracle.epilogue(ref, bias, None)
+    assert np.array_equal(v, ref + bias.astype(np.float64))
+    assert bits[0, 4] == oracle.bf16_rne(0.0)
+
+
+def test_epilogue_all_zero_operands_give_act_of_bias():
+    """A = 0: the product is exactly 0, so the output is act(bias) per column."""
+    M, N, K, g = 3, 16, 128, 128
+    a = np.zeros((M, K), np.uint8)
+    b = np.full((N, K), 0x38, np.uint8)
+    ref, _ = oracle.bsgemm("nt", a, b, np.ones((1, 1), np.float32), np.ones((1, 1), np.float32), M, N, K, g)
+    bias = np.linspace(-2, 2, N).astype(np.float32)
+    for act in (None, "relu", "gelu"):
+        v, _ = oracle.epilogue(ref, bias, act)
+        x = bias.astype(np.float64)
+        want = x if act is None else (np.maximum(x, 0) if act == "relu" else
+                                      0.5 * x * (1 + np.array([math.erf(t / math.sqrt(2)) for t in x])))
+        assert np.allclose(v, np.broadcast_to(want, (M, N)), rtol=0, atol=1e-15)
