@@ -228,7 +228,11 @@ def _rows_sample(p, rows):
 
 
 # ---------------------------------------------------------------- distributed plumbing
-def dist_setup(n_gpus: int):
+def dist_setup(n_gpus: int, backend: str = "nccl"):
+    """One process per GPU (torchrun sets RANK / WORLD_SIZE / LOCAL_RANK). The
+    GEMM has no exchange step, so ranks are independent replicas; the process
+    group serves only the barriers and the max over ranks of the step time.
+    ``backend="gloo"`` runs the same plumbing on CPU (tests)."""
     import torch
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -236,10 +240,13 @@ def dist_setup(n_gpus: int):
     if world > 1:
         import datetime
         import torch.distributed as dist
-        torch.cuda.set_device(local)
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                device_id=torch.device("cuda", local))
-    elif torch.cuda.is_available():
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+            dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                    device_id=torch.device("cuda", local))
+        else:
+            dist.init_process_group(backend, timeout=datetime.timedelta(seconds=60))
+    elif backend == "nccl" and torch.cuda.is_available():
         torch.cuda.set_device(0)
     return rank, world, local
 
@@ -250,14 +257,21 @@ def barrier(world):
         dist.barrier()
 
 
-def max_over_ranks(x: float, world: int) -> float:
+def max_over_ranks(x: float, world: int, device: str = "cuda") -> float:
+    """The slowest rank's value: the job's step time is set by its slowest replica."""
     if world == 1:
         return x
     import torch
     import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    t = torch.tensor([x], dtype=torch.float64, device=device)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def job_tflops(flops_per_rank: int, world: int, ms_max: float) -> float:
+    """Whole-job throughput of `world` replicas that each did `flops_per_rank`
+    in at most `ms_max` ms (weak scaling: per-GPU work fixed as N grows)."""
+    return world * flops_per_rank / (ms_max * 1e-3) / 1e12
 
 
 # ---------------------------------------------------------------- our arm
@@ -366,7 +380,7 @@ def run_ours(args):
                 "frac": achieved / peak, "traffic": profiled_traffic(args.workload), "peak_source": f"{peaks['source']} hbm copy",
                 "algorithmic_bytes_per_launch": bytes_}
     line = {
-        "metric": METRIC, "value": world * p.flops / (ms_max * 1e-3) / 1e12, "unit": "TFLOP/s",
+        "metric": METRIC, "value": job_tflops(p.flops, world, ms_max), "unit": "TFLOP/s",
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_max,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "fp8_e4m3",
         "data": "synthetic", "config": workload_config(p, args.workload) | {"parallelism": f"replicas{world}",
