@@ -176,6 +176,15 @@ __device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, const P
   return ok != 0;
 }
 
+// Bounded wait run by every lane of a converged warp; the answer is made
+// warp-uniform (a lane whose deadline ran out makes the whole warp give up),
+// so the warp stays converged.
+__device__ __forceinline__ bool warp_wait_all(uint32_t bar, uint32_t parity, const Params& p,
+                                              Barriers* bars, int where, bool ignore_abort = false) {
+  const bool ok = bounded_wait(bar, parity, p, bars, where, ignore_abort);
+  return __all_sync(0xffffffffu, ok);
+}
+
 // Shared-memory matrix descriptor for tcgen05 (sm_100 format, version 1),
 // 128-byte swizzle.  K-major: rows of 128 B, 8-row groups 1024 B apart (SBO);
 // MN-major: k-rows of 128 B, 8-k-row groups 1024 B apart (SBO), 128-element
@@ -553,15 +562,15 @@ __global__ void __launch_bounds__(kNumThreads, 1)
     }
   } else if (warp == kMmaWarp) {
     // ============================================================ MMA issuer
-    // One thread issues: per K-block it claims a TMEM buffer, issues the
-    // block's MMAs (K = 32 each) stage by stage -- waiting for a stage at its
-    // first k-step, releasing it after its last -- and commits the buffer to
-    // the promotion warps as soon as the block's last MMA is issued (the
-    // promotion of block kb gates the MMAs of block kb + kBufs).  The issue
-    // path is straight-line code on one lane: measured in this kernel, both a
-    // converged warp that branches per MMA and a converged warp whose lanes
-    // all wait (one lane issuing) are slower.
-    if (lane == 0) {
+    // Per K-block the issuer claims a TMEM buffer, issues the block's MMAs
+    // (K = 32 each) stage by stage -- waiting for a stage at its first k-step,
+    // releasing it after its last -- and commits the buffer to the promotion
+    // warps as soon as the block's last MMA is issued (the promotion of block
+    // kb gates the MMAs of block kb + kBufs). The whole warp runs the loop,
+    // converged: every lane polls the barriers, descriptors are warp-uniform,
+    // and each tcgen05 instruction is predicated on elect.sync, so one lane
+    // (always the same) issues it without the warp ever diverging.
+    {
       const uint32_t idesc = instr_desc<BNQ, P_MN, Q_MN>() | p.fmt_bits;
       // descriptor steps: per k-step of 32 (K-major +32 B, MN-major +32 rows
       // of 128 B) and per pipeline stage, in the descriptor's 16-byte units
@@ -592,8 +601,8 @@ __global__ void __launch_bounds__(kNumThreads, 1)
               const int k0 = kb * GRAN + j * BK;
               if (k0 >= p.K) break;
               // TMA writes and MMA reads are async-proxy accesses ordered by this barrier
-              if (!bounded_wait(smem_addr(&bars->full[s]), ph, p, bars, 2)) { ok = false; break; }
-              if (j == 0 && !bounded_wait(smem_addr(&bars->tmem_empty[b]), bph ^ 1, p, bars, 3)) {
+              if (!warp_wait_all(smem_addr(&bars->full[s]), ph, p, bars, 2)) { ok = false; break; }
+              if (j == 0 && !warp_wait_all(smem_addr(&bars->tmem_empty[b]), bph ^ 1, p, bars, 3)) {
                 ok = false;
                 break;
               }
@@ -601,14 +610,14 @@ __global__ void __launch_bounds__(kNumThreads, 1)
               if (k0 + BK <= p.K) {
 #pragma unroll
                 for (int t = 0; t < BK / kMmaK; ++t)
-                  mma_f8f6f4(d_tmem, ad + t * kPStep, bd + t * kQStep, idesc, (j > 0 || t > 0) ? 1u : 0u);
+                  mma_f8f6f4_elect(d_tmem, ad + t * kPStep, bd + t * kQStep, idesc, (j > 0 || t > 0) ? 1u : 0u);
               } else {
                 const int nsteps = (p.K - k0 + kMmaK - 1) / kMmaK;
                 for (int t = 0; t < nsteps; ++t)
-                  mma_f8f6f4(d_tmem, ad + t * kPStep, bd + t * kQStep, idesc, (j > 0 || t > 0) ? 1u : 0u);
+                  mma_f8f6f4_elect(d_tmem, ad + t * kPStep, bd + t * kQStep, idesc, (j > 0 || t > 0) ? 1u : 0u);
               }
-              if (j == GRAN / BK - 1 || k0 + BK >= p.K) mma_commit(smem_addr(&bars->tmem_full[b]));
-              mma_commit(smem_addr(&bars->empty[s]));  // stage free once these MMAs finish
+              if (j == GRAN / BK - 1 || k0 + BK >= p.K) mma_commit_elect(smem_addr(&bars->tmem_full[b]));
+              mma_commit_elect(smem_addr(&bars->empty[s]));  // stage free once these MMAs finish
               if (++s == STAGES) { s = 0; ph ^= 1; }
             }
             if (!ok) break;
@@ -617,24 +626,24 @@ __global__ void __launch_bounds__(kNumThreads, 1)
             // stage, odd blocks (or the K tail) release it
             const int k0 = kb * GRAN;
             const int t0 = (kb & 1) * 2;
-            if (t0 == 0 && !bounded_wait(smem_addr(&bars->full[s]), ph, p, bars, 2)) { ok = false; break; }
-            if (!bounded_wait(smem_addr(&bars->tmem_empty[b]), bph ^ 1, p, bars, 3)) { ok = false; break; }
+            if (t0 == 0 && !warp_wait_all(smem_addr(&bars->full[s]), ph, p, bars, 2)) { ok = false; break; }
+            if (!warp_wait_all(smem_addr(&bars->tmem_empty[b]), bph ^ 1, p, bars, 3)) { ok = false; break; }
             const uint64_t ad = ad0 + s * kPStage, bd = bd0 + s * kQStage;
             const int nsteps = (p.K - k0 >= GRAN) ? 2 : (p.K - k0 + kMmaK - 1) / kMmaK;
             for (int t = 0; t < nsteps; ++t)
-              mma_f8f6f4(d_tmem, ad + (t0 + t) * kPStep, bd + (t0 + t) * kQStep, idesc, t > 0 ? 1u : 0u);
-            mma_commit(smem_addr(&bars->tmem_full[b]));
+              mma_f8f6f4_elect(d_tmem, ad + (t0 + t) * kPStep, bd + (t0 + t) * kQStep, idesc, t > 0 ? 1u : 0u);
+            mma_commit_elect(smem_addr(&bars->tmem_full[b]));
             if (t0 == 2 || k0 + GRAN >= p.K) {
-              mma_commit(smem_addr(&bars->empty[s]));
+              mma_commit_elect(smem_addr(&bars->empty[s]));
               if (++s == STAGES) { s = 0; ph ^= 1; }
             }
           }
           if (++b == kBufs) { b = 0; bph ^= 1; }
         }
       }
-      // all MMAs issued by this thread complete before TMEM is freed
-      mma_commit(smem_addr(&bars->mma_done));
-      bounded_wait(smem_addr(&bars->mma_done), 0, p, bars, 8, true);
+      // all MMAs issued by the elected lane complete before TMEM is freed
+      mma_commit_elect(smem_addr(&bars->mma_done));
+      warp_wait_all(smem_addr(&bars->mma_done), 0, p, bars, 8, true);
     }
   }
   } else {
