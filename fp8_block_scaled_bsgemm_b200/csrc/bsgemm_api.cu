@@ -176,7 +176,16 @@ extern "C" bsgemm_status bsgemm_make_plan(int layout, int64_t M, int64_t N, int6
   bsgemm_plan pl{};
   const int Kb = static_cast<int>((K + gran - 1) / gran);
   int variant = t ? t->variant : BSGEMM_VARIANT_AUTO;
-  if (variant == BSGEMM_VARIANT_AUTO) variant = (M <= 128) ? BSGEMM_VARIANT_SWAP_AB : BSGEMM_VARIANT_DATA_PARALLEL;
+  if (variant == BSGEMM_VARIANT_AUTO) {
+    variant = (M <= 128) ? BSGEMM_VARIANT_SWAP_AB : BSGEMM_VARIANT_DATA_PARALLEL;
+    // CTA pairs halve each SM's operand traffic and double its pipeline
+    // depth; measured on B200 that pays where the promotion hand-off is rare
+    // (g = 256: one per two stages) and there is at least a full wave of
+    // 256 x 256 tiles (long_k g = 256: 219 vs 234 us), not at g = 128.
+    const bool tuned = t && (t->bnq != 0 || t->splits != 0 || t->stream_k != 0);
+    const int64_t pair_tiles = ((M + 255) / 256) * ((N + 255) / 256);
+    if (!tuned && gran == 256 && M > 128 && pair_tiles >= num_sms / 2) variant = BSGEMM_VARIANT_CTA_PAIR;
+  }
   if (variant == BSGEMM_VARIANT_CTA_PAIR) {
     // 256 x 256 tiles on CTA pairs, whole tiles walked by persistent pairs
     if ((t && t->bnq != 0 && t->bnq != 256) || (t && t->splits > 1) || (t && t->stream_k > 0))

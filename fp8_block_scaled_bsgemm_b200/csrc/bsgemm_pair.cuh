@@ -155,7 +155,9 @@ __global__ void __launch_bounds__(kNumThreads, 1)
     }
   } else if (warp == kMmaWarp) {
     // ============================================================ MMA issuer (even CTA)
-    if (rank == 0 && lane == 0) {
+    // the whole warp, converged; each tcgen05 instruction is predicated on
+    // elect.sync, so one lane (always the same) issues without divergence
+    if (rank == 0) {
       const uint32_t idesc = instr_desc_pair<P_MN, Q_MN>() | p.fmt_bits;
       constexpr uint64_t kPStep = P_MN ? (kMmaK * 128) >> 4 : kMmaK >> 4;
       constexpr uint64_t kQStep = Q_MN ? (kMmaK * 128) >> 4 : kMmaK >> 4;
@@ -176,8 +178,8 @@ __global__ void __launch_bounds__(kNumThreads, 1)
             for (int j = 0; j < GRAN / BK; ++j) {
               const int k0 = kb * GRAN + j * BK;
               if (k0 >= p.K) break;
-              if (!bounded_wait(smem_addr(&bars->full[s]), ph, p, bars, 2)) { ok = false; break; }
-              if (j == 0 && !bounded_wait(smem_addr(&bars->tmem_empty[b]), bph ^ 1, p, bars, 3)) {
+              if (!warp_wait_all(smem_addr(&bars->full[s]), ph, p, bars, 2)) { ok = false; break; }
+              if (j == 0 && !warp_wait_all(smem_addr(&bars->tmem_empty[b]), bph ^ 1, p, bars, 3)) {
                 ok = false;
                 break;
               }
@@ -185,14 +187,14 @@ __global__ void __launch_bounds__(kNumThreads, 1)
               if (k0 + BK <= p.K) {
 #pragma unroll
                 for (int u = 0; u < BK / kMmaK; ++u)
-                  mma_f8f6f4_pair(d_tmem, ad + u * kPStep, bd + u * kQStep, idesc, (j > 0 || u > 0) ? 1u : 0u);
+                  mma_f8f6f4_pair_elect(d_tmem, ad + u * kPStep, bd + u * kQStep, idesc, (j > 0 || u > 0) ? 1u : 0u);
               } else {
                 const int nsteps = (p.K - k0 + kMmaK - 1) / kMmaK;
                 for (int u = 0; u < nsteps; ++u)
-                  mma_f8f6f4_pair(d_tmem, ad + u * kPStep, bd + u * kQStep, idesc, (j > 0 || u > 0) ? 1u : 0u);
+                  mma_f8f6f4_pair_elect(d_tmem, ad + u * kPStep, bd + u * kQStep, idesc, (j > 0 || u > 0) ? 1u : 0u);
               }
-              if (j == GRAN / BK - 1 || k0 + BK >= p.K) mma_commit_pair(smem_addr(&bars->tmem_full[b]), kBoth);
-              mma_commit_pair(smem_addr(&bars->empty[s]), kBoth);
+              if (j == GRAN / BK - 1 || k0 + BK >= p.K) mma_commit_pair_elect(smem_addr(&bars->tmem_full[b]), kBoth);
+              mma_commit_pair_elect(smem_addr(&bars->empty[s]), kBoth);
               if (++s == STAGES) { s = 0; ph ^= 1; }
             }
             if (!ok) break;
@@ -200,24 +202,24 @@ __global__ void __launch_bounds__(kNumThreads, 1)
             // GRAN == 64: a K-block is half a stage
             const int k0 = kb * GRAN;
             const int t0 = (kb & 1) * 2;
-            if (t0 == 0 && !bounded_wait(smem_addr(&bars->full[s]), ph, p, bars, 2)) { ok = false; break; }
-            if (!bounded_wait(smem_addr(&bars->tmem_empty[b]), bph ^ 1, p, bars, 3)) { ok = false; break; }
+            if (t0 == 0 && !warp_wait_all(smem_addr(&bars->full[s]), ph, p, bars, 2)) { ok = false; break; }
+            if (!warp_wait_all(smem_addr(&bars->tmem_empty[b]), bph ^ 1, p, bars, 3)) { ok = false; break; }
             const uint64_t ad = ad0 + s * kPStage, bd = bd0 + s * kQStage;
             const int nsteps = (p.K - k0 >= GRAN) ? 2 : (p.K - k0 + kMmaK - 1) / kMmaK;
             for (int u = 0; u < nsteps; ++u)
-              mma_f8f6f4_pair(d_tmem, ad + (t0 + u) * kPStep, bd + (t0 + u) * kQStep, idesc, u > 0 ? 1u : 0u);
-            mma_commit_pair(smem_addr(&bars->tmem_full[b]), kBoth);
+              mma_f8f6f4_pair_elect(d_tmem, ad + (t0 + u) * kPStep, bd + (t0 + u) * kQStep, idesc, u > 0 ? 1u : 0u);
+            mma_commit_pair_elect(smem_addr(&bars->tmem_full[b]), kBoth);
             if (t0 == 2 || k0 + GRAN >= p.K) {
-              mma_commit_pair(smem_addr(&bars->empty[s]), kBoth);
+              mma_commit_pair_elect(smem_addr(&bars->empty[s]), kBoth);
               if (++s == STAGES) { s = 0; ph ^= 1; }
             }
           }
           if (++b == kBufs) { b = 0; bph ^= 1; }
         }
       }
-      // every pair MMA this thread issued completes before TMEM is freed
-      mma_commit_pair(smem_addr(&bars->mma_done), 0x1);
-      bounded_wait(smem_addr(&bars->mma_done), 0, p, bars, 8, true);
+      // every pair MMA the elected lane issued completes before TMEM is freed
+      mma_commit_pair_elect(smem_addr(&bars->mma_done), 0x1);
+      warp_wait_all(smem_addr(&bars->mma_done), 0, p, bars, 8, true);
     }
   }
   } else {

@@ -123,21 +123,12 @@ __device__ __forceinline__ void tc_fence_after() {
   asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
 }
 
-// D[tmem] (+)= A[smem desc] * B[smem desc]^T, FP8 x FP8 -> FP32, one CTA.
-__device__ __forceinline__ void mma_f8f6f4(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
-                                           uint32_t idesc, uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
-      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
-      : "memory");
-}
-
-// The same two instructions issued from a converged warp: elect.sync picks one
-// lane (the lowest active one, so the same lane on every call from a fully
-// converged warp) and only that lane executes the tcgen05 instruction. The
-// warp never diverges and the operands stay warp-uniform.
+// D[tmem] (+)= A[smem desc] * B[smem desc]^T, FP8 x FP8 -> FP32, one CTA, and
+// the commit that arrives once on `bar` when all tcgen05 ops issued so far by
+// the issuing thread finish. Both are issued from a converged warp: elect.sync
+// picks one lane (the lowest active one, so the same lane on every call from a
+// fully converged warp) and only that lane executes the tcgen05 instruction.
+// The warp never diverges and the operands stay warp-uniform.
 __device__ __forceinline__ void mma_f8f6f4_elect(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
                                                  uint32_t idesc, uint32_t accumulate) {
   asm volatile(
@@ -155,13 +146,6 @@ __device__ __forceinline__ void mma_commit_elect(uint32_t bar) {
       "elect.sync _|e, 0xffffffff;\n\t"
       "@e tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n\t}" ::"r"(bar)
       : "memory");
-}
-
-// Arrive once on `bar` when all tcgen05 ops issued so far by this thread finish.
-__device__ __forceinline__ void mma_commit(uint32_t bar) {
-  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
-                   bar)
-               : "memory");
 }
 
 // 32 lanes x 32 bit, 8 consecutive columns per thread.
@@ -297,23 +281,27 @@ __device__ __forceinline__ void tmem_dealloc_pair(uint32_t taddr, uint32_t ncols
 
 // D (+)= A * B^T over the CTA pair (M = 256: 128 rows of A and half of B's
 // N columns in each CTA's shared memory, at the same offsets; each CTA's TMEM
-// gets its 128 rows of D).  Issued by one thread of the even CTA.
-__device__ __forceinline__ void mma_f8f6f4_pair(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
-                                                uint32_t idesc, uint32_t accumulate) {
+// gets its 128 rows of D), issued by one elected lane (always the same) of a
+// converged warp of the even CTA.
+__device__ __forceinline__ void mma_f8f6f4_pair_elect(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                                      uint32_t idesc, uint32_t accumulate) {
   asm volatile(
-      "{\n\t.reg .pred p;\n\t"
+      "{\n\t.reg .pred p, e;\n\t"
       "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::2.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "elect.sync _|e, 0xffffffff;\n\t"
+      "@e tcgen05.mma.cta_group::2.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
       "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
       : "memory");
 }
 
 // Arrive once on the mbarrier at offset `bar` in every CTA of `cta_mask` when
-// the pair MMAs issued so far by this thread finish.
-__device__ __forceinline__ void mma_commit_pair(uint32_t bar, uint16_t cta_mask) {
+// the pair MMAs issued so far by the elected lane finish.
+__device__ __forceinline__ void mma_commit_pair_elect(uint32_t bar, uint16_t cta_mask) {
   asm volatile(
-      "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64"
-      " [%0], %1;" ::"r"(bar),
+      "{\n\t.reg .pred e;\n\t"
+      "elect.sync _|e, 0xffffffff;\n\t"
+      "@e tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64"
+      " [%0], %1;\n\t}" ::"r"(bar),
       "h"(cta_mask)
       : "memory");
 }

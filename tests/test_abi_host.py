@@ -97,6 +97,11 @@ def test_plan_for_cta_pairs():
         with pytest.raises(bsg.BsgemmError):
             bsg.make_plan(4096, 4096, 4096, 128, "nt", 148, bad)
     assert bsg.make_plan(4096, 4096, 4096, 128, "nt", 148)["cta_pair"] == 0
+    # the heuristic takes CTA pairs only at g = 256 with a full wave of 256 x 256 tiles
+    assert bsg.make_plan(2048, 4096, 32768, 256, "nt", 148)["cta_pair"] == 1
+    assert bsg.make_plan(2048, 4096, 32768, 128, "nt", 148)["cta_pair"] == 0
+    assert bsg.make_plan(512, 512, 4096, 256, "nt", 148)["cta_pair"] == 0          # 4 pair tiles
+    assert bsg.make_plan(2048, 4096, 32768, 256, "nt", 148, {"stream_k": -1})["cta_pair"] == 0
 
 
 def _sk_partition(tiles_sk, U, G):
