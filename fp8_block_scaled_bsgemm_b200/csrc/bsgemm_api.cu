@@ -70,6 +70,7 @@ bsgemm_status device_info(DeviceInfo& out) {
   auto it = g_dev.find(dev);
   if (it == g_dev.end()) {
     DeviceInfo d;
+    d.ordinal = dev;
     int major = 0, minor = 0;
     if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
         cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess ||

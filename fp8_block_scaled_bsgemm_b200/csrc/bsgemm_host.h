@@ -4,6 +4,7 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include <atomic>
 #include <cstddef>
 #include <cstdint>
 
@@ -13,8 +14,25 @@ namespace bsg_host {
 
 struct DeviceInfo {
   bool ok = false;
+  int ordinal = 0;        // CUDA device number
   int num_sms = 0;
   int* status = nullptr;  // device address of the status word
+};
+
+// One-time per-device launch setup of one kernel instance (function
+// attributes are set per device): a bit per device for devices 0..63;
+// higher-numbered devices simply redo the setup on every launch.
+class PerDeviceOnce {
+ public:
+  bool done(int dev) const {
+    return dev >= 0 && dev < 64 && ((bits_.load(std::memory_order_acquire) >> dev) & 1u);
+  }
+  void mark(int dev) {
+    if (dev >= 0 && dev < 64) bits_.fetch_or(uint64_t(1) << dev, std::memory_order_acq_rel);
+  }
+
+ private:
+  std::atomic<uint64_t> bits_{0};
 };
 
 struct Workspace {

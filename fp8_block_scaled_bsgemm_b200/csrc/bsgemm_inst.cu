@@ -93,8 +93,8 @@ bsgemm_status launch(const bsgemm_plan& plan, const void* a, const void* b, cons
     prm.counters = w.counters;
   }
 
-  static bool attr_set = false;  // once per instance
-  if (!attr_set) {
+  static PerDeviceOnce setup;  // once per instance and device
+  if (!setup.done(dev.ordinal)) {
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SC::kSmemBytes) != cudaSuccess)
       return BSGEMM_ERR_CUDA;
     if (bsg::RegSplit<BNQ>::kEnabled) {
@@ -103,7 +103,7 @@ bsgemm_status launch(const bsgemm_plan& plan, const void* a, const void* b, cons
       if (cudaFuncGetAttributes(&fa, kern) != cudaSuccess || fa.numRegs != bsg::kLaunchRegs)
         return BSGEMM_ERR_CUDA;
     }
-    attr_set = true;
+    setup.mark(dev.ordinal);
   }
   kern<<<plan.grid, bsg::kNumThreads, SC::kSmemBytes, stream>>>(tm_p, tm_q, prm);
   return cudaGetLastError() == cudaSuccess ? BSGEMM_OK : BSGEMM_ERR_CUDA;
@@ -156,7 +156,11 @@ bsgemm_status launch_pair(const bsgemm_plan& plan, const void* a, const void* b,
   cfg.attrs = attr;
   cfg.numAttrs = 1;
 
-  static int max_pairs = 0;  // co-resident CTA pairs, once per instance
+  // co-resident CTA pairs, found once per instance and device
+  static PerDeviceOnce setup;
+  static std::atomic<int> resident_pairs[64];
+  const int slot = dev.ordinal >= 0 && dev.ordinal < 64 ? dev.ordinal : -1;
+  int max_pairs = slot >= 0 && setup.done(slot) ? resident_pairs[slot].load(std::memory_order_relaxed) : 0;
   if (max_pairs == 0) {
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, PC::kSmemBytes) != cudaSuccess)
       return BSGEMM_ERR_CUDA;
@@ -168,6 +172,10 @@ bsgemm_status launch_pair(const bsgemm_plan& plan, const void* a, const void* b,
     int n = 0;
     if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) != cudaSuccess || n < 1) return BSGEMM_ERR_CUDA;
     max_pairs = n;
+    if (slot >= 0) {
+      resident_pairs[slot].store(n, std::memory_order_relaxed);
+      setup.mark(slot);
+    }
   }
   // a persistent grid no larger than the pairs that can be resident at once
   int pairs = plan.grid / 2;
