@@ -1,6 +1,6 @@
 """Helpers shared by the GPU parity tests (not a test module).
 
-Tolerance (per element, spec parity bar for this GEMM):
+Tolerance (per element, the parity bar for this GEMM):
     |gpu - ref| <= 2^-7 * |ref| + 2^-8 * rms(ref)
 where ref is the oracle's FP64 value before BF16 rounding and rms is taken
 over the whole checked set.  2^-7 is one BF16 rounding (2^-8) plus the same

@@ -190,3 +190,31 @@ def test_register_split_kernels_have_the_planned_launch_registers():
     # instance in each of the 3 NT units; one CTA-pair kernel per unit
     assert seen == 24 + 3
     assert pairs == 12
+
+
+def test_new_entry_points_reject_bad_arguments_on_the_host():
+    """Formats, epilogue options, quantiser and grouped arguments are checked
+    before any CUDA call (no device is touched here)."""
+    L = bsg.lib()
+    A = 256  # a 16-byte aligned stand-in address; nothing is dereferenced
+    # unknown FP8 format
+    assert L.bsgemm_fp8_gemm_fmt(0, 2, 0, A, A, A, A, A, 16, 16, 16, 128, None, None) == 1
+    assert L.bsgemm_fp8_gemm_fmt(0, 0, -1, A, A, A, A, A, 16, 16, 16, 128, None, None) == 1
+    # epilogue: unknown activation, unknown output type, misaligned bias
+    epi = bsg.Epilogue(None, 7, 0)
+    assert L.bsgemm_fp8_gemm_fused(0, 0, 0, A, A, A, A, ctypes.byref(epi), A, 16, 16, 16, 128, None, None) == 1
+    epi = bsg.Epilogue(None, 1, 5)
+    assert L.bsgemm_fp8_gemm_fused(0, 0, 0, A, A, A, A, ctypes.byref(epi), A, 16, 16, 16, 128, None, None) == 1
+    epi = bsg.Epilogue(A + 2, 0, 0)
+    assert L.bsgemm_fp8_gemm_fused(0, 0, 0, A, A, A, A, ctypes.byref(epi), A, 16, 16, 16, 128, None, None) == 3
+    # quantiser: null pointer, bad source type, bad gran, cols % 16, misaligned source
+    assert L.bsgemm_quantize_fp8(0, 0, None, 16, 16, 128, A, A, None) == 1
+    assert L.bsgemm_quantize_fp8(3, 0, A, 16, 16, 128, A, A, None) == 1
+    assert L.bsgemm_quantize_fp8(0, 0, A, 16, 16, 96, A, A, None) == 2
+    assert L.bsgemm_quantize_fp8(0, 0, A, 16, 40, 128, A, A, None) == 3
+    assert L.bsgemm_quantize_fp8(1, 1, A + 8, 16, 32, 128, A, A, None) == 3
+    # grouped: no groups, no rows, misaligned group sizes, K % 16
+    assert L.bsgemm_fp8_grouped_nt(0, 0, A, A, A, A, A, A, 0, 64, 128, 128, 128, None) == 1
+    assert L.bsgemm_fp8_grouped_nt(0, 0, A, A, A, A, A, A, 2, 0, 128, 128, 128, None) == 1
+    assert L.bsgemm_fp8_grouped_nt(0, 0, A, A, A, A, A, A + 2, 2, 64, 128, 128, 128, None) == 3
+    assert L.bsgemm_fp8_grouped_nt(0, 0, A, A, A, A, A, A, 2, 64, 128, 40, 128, None) == 3
