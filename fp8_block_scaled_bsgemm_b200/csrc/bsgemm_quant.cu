@@ -12,8 +12,10 @@
 // to scales [ceil(rows/g), ceil(cols/g)] (row-major FP32): exactly the
 // operand and scale tensors the GEMM takes.
 //
-// One CTA of 256 threads per block. The block is read twice (amax, then
-// encode); the second read comes from L2. Each thread handles runs of 8
+// One CTA of 256 threads per block. For g <= 128 each thread keeps its part
+// of the block in registers between the amax pass and the encode pass; for
+// g = 256 the block is read twice, the second time from L2. Each thread
+// handles runs of 8
 // consecutive columns: 32-byte (FP32) or 16-byte (BF16) loads, 8-byte stores
 // of 8 codes. This is HBM-bound work: no tensor cores.
 #include <cuda_bf16.h>
@@ -29,22 +31,50 @@ namespace bsgq {
 constexpr int kThreads = 256;
 constexpr int kVec = 8;  // columns per run
 
+// One run of 8 source values as loaded: one 16-byte word of BF16 values, or
+// two of FP32 values. A run is held in this form and widened on use, so a
+// BF16 run costs 4 registers rather than 8.
 template <bool BF16_IN>
-__device__ __forceinline__ void load8(const void* x, int64_t off, float (&v)[kVec]) {
+struct Run {
+  uint4 w[BF16_IN ? 1 : 2];
+};
+
+template <bool BF16_IN>
+__device__ __forceinline__ Run<BF16_IN> load_run(const void* x, int64_t off) {
+  Run<BF16_IN> r;
   if constexpr (BF16_IN) {
-    const uint4 u = __ldg(reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(x) + off));
-    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+    r.w[0] = __ldg(reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(x) + off));
+  } else {
+    const uint4* p = reinterpret_cast<const uint4*>(static_cast<const float*>(x) + off);
+    r.w[0] = __ldg(p);
+    r.w[1] = __ldg(p + 1);
+  }
+  return r;
+}
+
+template <bool BF16_IN>
+__device__ __forceinline__ void widen(const Run<BF16_IN>& r, float (&v)[kVec]) {
+  if constexpr (BF16_IN) {
+    const uint32_t w[4] = {r.w[0].x, r.w[0].y, r.w[0].z, r.w[0].w};
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
       v[2 * i] = __uint_as_float(w[i] << 16);
       v[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
     }
   } else {
-    const float4* p = reinterpret_cast<const float4*>(static_cast<const float*>(x) + off);
-    const float4 a = __ldg(p), b = __ldg(p + 1);
-    v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
-    v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      v[4 * h + 0] = __uint_as_float(r.w[h].x);
+      v[4 * h + 1] = __uint_as_float(r.w[h].y);
+      v[4 * h + 2] = __uint_as_float(r.w[h].z);
+      v[4 * h + 3] = __uint_as_float(r.w[h].w);
+    }
   }
+}
+
+template <bool BF16_IN>
+__device__ __forceinline__ void load8(const void* x, int64_t off, float (&v)[kVec]) {
+  widen<BF16_IN>(load_run<BF16_IN>(x, off), v);
 }
 
 template <int FMT>
@@ -67,17 +97,61 @@ __global__ void __launch_bounds__(kThreads)
   const int64_t blk = blockIdx.x;
   const int64_t r0 = (blk / col_blocks) * G;
   const int64_t c0 = (blk % col_blocks) * G;
+  // g <= 128: the thread's runs stay in registers between the two passes
+  // (at most 8 runs); g = 256 reads the block again from L2
+  constexpr int kHeld = kRuns / kThreads <= 8 ? kRuns / kThreads : 0;
+  Run<BF16_IN> held[kHeld > 0 ? kHeld : 1];
 
   // ---- pass 1: amax over the block (elements outside the matrix are skipped)
   float amax = 0.f;
-  for (int run = threadIdx.x; run < kRuns; run += kThreads) {
-    const int64_t r = r0 + run / kRunsPerRow;
-    const int64_t c = c0 + (run % kRunsPerRow) * kVec;
-    if (r < rows && c < cols) {  // cols % 8 == 0: a run is wholly in or out
-      float v[kVec];
-      load8<BF16_IN>(x, r * cols + c, v);
+  if constexpr (kHeld > 0) {
 #pragma unroll
-      for (int i = 0; i < kVec; ++i) amax = fmaxf(amax, fabsf(v[i]));
+    for (int j = 0; j < kHeld; ++j) {
+      const int run = threadIdx.x + j * kThreads;
+      const int64_t r = r0 + run / kRunsPerRow;
+      const int64_t c = c0 + (run % kRunsPerRow) * kVec;
+      if (r < rows && c < cols) {  // cols % 8 == 0: a run is wholly in or out
+        held[j] = load_run<BF16_IN>(x, r * cols + c);
+      } else {
+#pragma unroll
+        for (int h = 0; h < (BF16_IN ? 1 : 2); ++h) held[j].w[h] = make_uint4(0, 0, 0, 0);
+      }
+    }
+    if constexpr (BF16_IN) {
+      // |x| max on packed pairs (NaN-ignoring, like fmaxf): the runs stay
+      // packed until the encode pass widens them
+      __nv_bfloat162 m2 = __float2bfloat162_rn(0.f);
+#pragma unroll
+      for (int j = 0; j < kHeld; ++j) {
+        const uint32_t w[4] = {held[j].w[0].x, held[j].w[0].y, held[j].w[0].z, held[j].w[0].w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          __nv_bfloat162_raw raw;
+          raw.x = static_cast<unsigned short>(w[i] & 0xFFFFu);
+          raw.y = static_cast<unsigned short>(w[i] >> 16);
+          m2 = __hmax2(m2, __habs2(__nv_bfloat162(raw)));
+        }
+      }
+      amax = fmaxf(__low2float(m2), __high2float(m2));
+    } else {
+#pragma unroll
+      for (int j = 0; j < kHeld; ++j) {
+        float v[kVec];
+        widen<BF16_IN>(held[j], v);
+#pragma unroll
+        for (int i = 0; i < kVec; ++i) amax = fmaxf(amax, fabsf(v[i]));
+      }
+    }
+  } else {
+    for (int run = threadIdx.x; run < kRuns; run += kThreads) {
+      const int64_t r = r0 + run / kRunsPerRow;
+      const int64_t c = c0 + (run % kRunsPerRow) * kVec;
+      if (r < rows && c < cols) {
+        float v[kVec];
+        load8<BF16_IN>(x, r * cols + c, v);
+#pragma unroll
+        for (int i = 0; i < kVec; ++i) amax = fmaxf(amax, fabsf(v[i]));
+      }
     }
   }
 #pragma unroll
@@ -96,19 +170,36 @@ __global__ void __launch_bounds__(kThreads)
   const float s = block_scale;
 
   // ---- pass 2: encode
-  for (int run = threadIdx.x; run < kRuns; run += kThreads) {
-    const int64_t r = r0 + run / kRunsPerRow;
-    const int64_t c = c0 + (run % kRunsPerRow) * kVec;
-    if (r < rows && c < cols) {
-      float v[kVec];
-      load8<BF16_IN>(x, r * cols + c, v);
-      uint32_t lo = 0, hi = 0;
+  auto encode_run = [&](const float (&v)[kVec], int64_t r, int64_t c) {
+    uint32_t lo = 0, hi = 0;
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        lo |= encode<FMT>(__fdiv_rn(v[i], s)) << (8 * i);
-        hi |= encode<FMT>(__fdiv_rn(v[4 + i], s)) << (8 * i);
+    for (int i = 0; i < 4; ++i) {
+      lo |= encode<FMT>(__fdiv_rn(v[i], s)) << (8 * i);
+      hi |= encode<FMT>(__fdiv_rn(v[4 + i], s)) << (8 * i);
+    }
+    *reinterpret_cast<uint2*>(q + r * cols + c) = make_uint2(lo, hi);
+  };
+  if constexpr (kHeld > 0) {
+#pragma unroll
+    for (int j = 0; j < kHeld; ++j) {
+      const int run = threadIdx.x + j * kThreads;
+      const int64_t r = r0 + run / kRunsPerRow;
+      const int64_t c = c0 + (run % kRunsPerRow) * kVec;
+      if (r < rows && c < cols) {
+        float v[kVec];
+        widen<BF16_IN>(held[j], v);
+        encode_run(v, r, c);
       }
-      *reinterpret_cast<uint2*>(q + r * cols + c) = make_uint2(lo, hi);
+    }
+  } else {
+    for (int run = threadIdx.x; run < kRuns; run += kThreads) {
+      const int64_t r = r0 + run / kRunsPerRow;
+      const int64_t c = c0 + (run % kRunsPerRow) * kVec;
+      if (r < rows && c < cols) {
+        float v[kVec];
+        load8<BF16_IN>(x, r * cols + c, v);
+        encode_run(v, r, c);
+      }
     }
   }
 }
