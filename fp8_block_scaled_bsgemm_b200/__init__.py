@@ -132,12 +132,35 @@ def _tuning(tuning):
     return ctypes.byref(t)
 
 
-def _as_bytes(x: torch.Tensor, name: str) -> torch.Tensor:
+def _as_bytes(x: torch.Tensor, name: str, device=None) -> torch.Tensor:
     if x.dtype not in (torch.float8_e4m3fn, torch.float8_e5m2, torch.uint8):
         raise TypeError(f"{name} must be float8_e4m3fn, float8_e5m2 or uint8 codes, got {x.dtype}")
     if not x.is_cuda or not x.is_contiguous():
         raise ValueError(f"{name} must be a contiguous CUDA tensor")
+    if device is not None and x.device != device:
+        raise ValueError(f"{name} is on {x.device}, the first operand on {device}")
     return x
+
+
+def _device_tensor(t, name: str, dtype, device, numel=None, min_numel=None):
+    """Check a tensor whose data pointer goes to the library: the kernels get
+    only the pointer, so its type, placement and size are checked here."""
+    if not isinstance(t, torch.Tensor) or t.dtype != dtype or not t.is_cuda or not t.is_contiguous():
+        raise ValueError(f"{name} must be a contiguous {dtype} CUDA tensor")
+    if t.device != device:
+        raise ValueError(f"{name} is on {t.device}, the first operand on {device}")
+    if numel is not None and t.numel() != numel:
+        raise ValueError(f"{name} must have {numel} elements, got {t.numel()}")
+    if min_numel is not None and t.numel() < min_numel:
+        raise ValueError(f"{name} must have at least {min_numel} elements, got {t.numel()}")
+    return t
+
+
+def _blocks(n: int, gran) -> int:
+    return -(-int(n) // int(gran))
+
+
+_GRANS = (64, 128, 256)   # other values go to the library, which rejects them
 
 
 def shapes(layout: str, a: torch.Tensor, b: torch.Tensor):
@@ -176,29 +199,33 @@ def gemm(a, b, scale_a, scale_b, out=None, layout="nt", gran=128, tuning=None, s
     fa = _format(a, a_format, "a")
     fb = _format(b, b_format, "b")
     a = _as_bytes(a, "a")
-    b = _as_bytes(b, "b")
+    dev = a.device
+    b = _as_bytes(b, "b", dev)
     M, N, K = shapes(layout, a, b)
-    for s, nm in ((scale_a, "scale_a"), (scale_b, "scale_b")):
-        if s.dtype != torch.float32 or not s.is_cuda or not s.is_contiguous():
-            raise ValueError(f"{nm} must be a contiguous float32 CUDA tensor")
+    ok_g = gran in _GRANS
+    _device_tensor(scale_a, "scale_a", torch.float32, dev,
+                   _blocks(M, gran) * _blocks(K, gran) if ok_g else None)
+    _device_tensor(scale_b, "scale_b", torch.float32, dev,
+                   _blocks(N, gran) * _blocks(K, gran) if ok_g else None)
     if out_dtype not in (torch.bfloat16, torch.float32):
         raise ValueError("out_dtype must be torch.bfloat16 or torch.float32")
     if activation not in ACTIVATIONS:
         raise ValueError(f"activation must be one of {sorted(k for k in ACTIVATIONS if k)}")
-    if bias is not None and (bias.dtype != torch.float32 or not bias.is_cuda or not bias.is_contiguous()
-                             or bias.numel() != N):
-        raise ValueError("bias must be a contiguous float32 CUDA tensor of N elements")
+    if bias is not None:
+        _device_tensor(bias, "bias", torch.float32, dev, N)
     if out is None:
-        out = torch.empty((M, N), dtype=out_dtype, device=a.device)
-    if out.dtype != out_dtype or tuple(out.shape) != (M, N) or not out.is_contiguous():
-        raise ValueError(f"out must be a contiguous {out_dtype} [M, N] tensor")
+        out = torch.empty((M, N), dtype=out_dtype, device=dev)
+    _device_tensor(out, "out", out_dtype, dev)
+    if tuple(out.shape) != (M, N):
+        raise ValueError(f"out must be a {out_dtype} [M, N] = [{M}, {N}] tensor, got {tuple(out.shape)}")
     epi = None
     if bias is not None or ACTIVATIONS[activation] or out_dtype == torch.float32:
         epi = ctypes.byref(Epilogue(bias.data_ptr() if bias is not None else None, ACTIVATIONS[activation],
                                     1 if out_dtype == torch.float32 else 0))
-    st = lib().bsgemm_fp8_gemm_fused(LAYOUTS[layout], fa, fb, a.data_ptr(), b.data_ptr(),
-                                     scale_a.data_ptr(), scale_b.data_ptr(), epi, out.data_ptr(), M, N,
-                                     K, int(gran), _tuning(tuning), _stream_handle(stream))
+    with torch.cuda.device(dev):
+        st = lib().bsgemm_fp8_gemm_fused(LAYOUTS[layout], fa, fb, a.data_ptr(), b.data_ptr(),
+                                         scale_a.data_ptr(), scale_b.data_ptr(), epi, out.data_ptr(), M,
+                                         N, K, int(gran), _tuning(tuning), _stream_handle(stream))
     if st != 0:
         raise BsgemmError(st, f"bsgemm {layout} M={M} N={N} K={K} g={gran}")
     return out
@@ -233,12 +260,19 @@ def quantize(x: torch.Tensor, gran: int = 128, fmt: str = "e4m3", q=None, scales
     if fmt not in FORMATS:
         raise ValueError(f"fmt must be one of {sorted(FORMATS)}")
     rows, cols = x.shape
+    dev = x.device
     if q is None:
-        q = torch.empty((rows, cols), dtype=torch.uint8, device=x.device)
+        q = torch.empty((rows, cols), dtype=torch.uint8, device=dev)
+    _device_tensor(q, "q", torch.uint8, dev, rows * cols)
+    ok_g = gran in _GRANS
     if scales is None:
-        scales = torch.empty((-(-rows // gran), -(-cols // gran)), dtype=torch.float32, device=x.device)
-    st = lib().bsgemm_quantize_fp8(src, FORMATS[fmt], x.data_ptr(), rows, cols, int(gran), q.data_ptr(),
-                                   scales.data_ptr(), _stream_handle(stream))
+        scales = torch.empty((_blocks(rows, gran), _blocks(cols, gran)) if ok_g else (1,),
+                             dtype=torch.float32, device=dev)
+    _device_tensor(scales, "scales", torch.float32, dev,
+                   _blocks(rows, gran) * _blocks(cols, gran) if ok_g else None)
+    with torch.cuda.device(dev):
+        st = lib().bsgemm_quantize_fp8(src, FORMATS[fmt], x.data_ptr(), rows, cols, int(gran), q.data_ptr(),
+                                       scales.data_ptr(), _stream_handle(stream))
     if st != 0:
         raise BsgemmError(st, f"bsgemm_quantize_fp8 {rows}x{cols} g={gran}")
     return q, scales
@@ -252,21 +286,30 @@ def grouped_gemm(a, b, scale_a, scale_b, group_m, out=None, gran=128, a_format=N
     fa = _format(a, a_format, "a")
     fb = _format(b, b_format, "b")
     a = _as_bytes(a, "a")
-    b = _as_bytes(b, "b")
+    dev = a.device
+    b = _as_bytes(b, "b", dev)
     if a.dim() != 2 or b.dim() != 3 or a.shape[1] != b.shape[2]:
         raise ValueError("a must be [max_rows, K] and b [num_groups, N, K]")
-    if group_m.dtype != torch.int32 or not group_m.is_cuda or not group_m.is_contiguous() \
-            or group_m.numel() != b.shape[0]:
-        raise ValueError("group_m must be a contiguous int32 CUDA tensor with one entry per group")
     max_rows, K = a.shape
     G, N = b.shape[0], b.shape[1]
+    _device_tensor(group_m, "group_m (one int32 entry per group)", torch.int32, dev, G)
+    if gran in _GRANS:
+        kb = _blocks(K, gran)
+        _device_tensor(scale_a, "scale_a", torch.float32, dev,
+                       min_numel=(_blocks(max_rows, gran) + G) * kb)
+        _device_tensor(scale_b, "scale_b", torch.float32, dev, G * _blocks(N, gran) * kb)
+    else:
+        _device_tensor(scale_a, "scale_a", torch.float32, dev)
+        _device_tensor(scale_b, "scale_b", torch.float32, dev)
     if out is None:
-        out = torch.empty((max_rows, N), dtype=torch.bfloat16, device=a.device)
-    if out.dtype != torch.bfloat16 or tuple(out.shape) != (max_rows, N) or not out.is_contiguous():
-        raise ValueError("out must be a contiguous bfloat16 [max_rows, N] tensor")
-    st = lib().bsgemm_fp8_grouped_nt(fa, fb, a.data_ptr(), b.data_ptr(), scale_a.data_ptr(),
-                                     scale_b.data_ptr(), out.data_ptr(), group_m.data_ptr(), G, max_rows,
-                                     N, K, int(gran), _stream_handle(stream))
+        out = torch.empty((max_rows, N), dtype=torch.bfloat16, device=dev)
+    _device_tensor(out, "out", torch.bfloat16, dev)
+    if tuple(out.shape) != (max_rows, N):
+        raise ValueError(f"out must be a bfloat16 [max_rows, N] = [{max_rows}, {N}] tensor")
+    with torch.cuda.device(dev):
+        st = lib().bsgemm_fp8_grouped_nt(fa, fb, a.data_ptr(), b.data_ptr(), scale_a.data_ptr(),
+                                         scale_b.data_ptr(), out.data_ptr(), group_m.data_ptr(), G,
+                                         max_rows, N, K, int(gran), _stream_handle(stream))
     if st != 0:
         raise BsgemmError(st, f"bsgemm grouped G={G} max_rows={max_rows} N={N} K={K} g={gran}")
     return out

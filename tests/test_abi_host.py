@@ -218,3 +218,18 @@ def test_new_entry_points_reject_bad_arguments_on_the_host():
     assert L.bsgemm_fp8_grouped_nt(0, 0, A, A, A, A, A, A, 2, 0, 128, 128, 128, None) == 1
     assert L.bsgemm_fp8_grouped_nt(0, 0, A, A, A, A, A, A + 2, 2, 64, 128, 128, 128, None) == 3
     assert L.bsgemm_fp8_grouped_nt(0, 0, A, A, A, A, A, A, 2, 64, 128, 40, 128, None) == 3
+
+
+def test_binding_rejects_host_tensors_before_calling_the_library():
+    """The binding hands bare pointers to the kernels: a host tensor is refused
+    in Python, with nothing passed to the library."""
+    import torch
+    a = torch.zeros((128, 256), dtype=torch.uint8)
+    s = torch.ones((1, 2))
+    with pytest.raises(ValueError):
+        bsg.gemm(a, a, s, s)
+    with pytest.raises(ValueError):
+        bsg.quantize(torch.zeros((128, 256)), 128)
+    with pytest.raises(ValueError):
+        bsg.grouped_gemm(a, a.reshape(1, 128, 256), torch.ones((2, 2)), s,
+                         torch.zeros(1, dtype=torch.int32))

@@ -82,3 +82,10 @@ def test_grouped_gemm_argument_errors():
         bsg.grouped_gemm(a, b, sa, sb, torch.zeros(2, dtype=torch.int64, device="cuda"))
     with pytest.raises(ValueError):
         bsg.grouped_gemm(a, b, sa, sb, torch.zeros(3, dtype=torch.int32, device="cuda"))
+    gm = torch.zeros(2, dtype=torch.int32, device="cuda")
+    with pytest.raises(ValueError):                  # fewer scale rows than ceil(64/128) + 2 groups
+        bsg.grouped_gemm(a, b, sa[:2].contiguous(), sb, gm)
+    with pytest.raises(ValueError):
+        bsg.grouped_gemm(a, b, sa, sb.cpu(), gm)
+    with pytest.raises(ValueError):
+        bsg.grouped_gemm(a, b, sa, sb, gm.cpu())

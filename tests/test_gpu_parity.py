@@ -186,6 +186,30 @@ def test_fused_epilogue_fp32_output_without_bias_keeps_fp32_precision():
     assert np.max(np.abs(got - ref) / (np.abs(ref) + 1e-3 * np.sqrt(np.mean(ref ** 2)))) < 2.0 ** -12
 
 
+def test_binding_checks_the_tensors_it_hands_to_the_library():
+    """The kernels receive bare pointers, so the binding rejects a tensor on the
+    host, on another device, or too small for the sizes it implies."""
+    p = workloads.make_problem(128, 256, 256, 128, "nt", seed=35)
+    a, b, sa, sb = to_device(p)                                   # sa, sb: [1, 2], [2, 2]
+    for bad in (dict(scale_a=sa.cpu()), dict(scale_a=sa[:, :1].contiguous()),
+                dict(scale_b=sb.reshape(-1)[:3].contiguous()), dict(b=b.cpu())):
+        args = dict(a=a, b=b, scale_a=sa, scale_b=sb)
+        args.update(bad)
+        with pytest.raises(ValueError):
+            bsg.gemm(args["a"], args["b"], args["scale_a"], args["scale_b"])
+    with pytest.raises(ValueError):
+        bsg.gemm(a, b, sa, sb, out=torch.empty((128, 256), dtype=torch.bfloat16))
+    with pytest.raises(ValueError):
+        bsg.gemm(a, b, sa, sb, bias=torch.zeros(256))
+    x = torch.zeros((128, 256), device="cuda")
+    with pytest.raises(ValueError):
+        bsg.quantize(x, 128, q=torch.empty((128, 256), dtype=torch.uint8))
+    with pytest.raises(ValueError):
+        bsg.quantize(x, 128, scales=torch.empty((1, 1), device="cuda"))
+    torch.cuda.synchronize()
+    assert bsg.get_last_device_status() == 0
+
+
 def test_fused_epilogue_argument_errors():
     p = workloads.make_problem(128, 256, 256, 128, "nt", seed=34)
     a, b, sa, sb = to_device(p)
