@@ -173,6 +173,7 @@ extern "C" bsgemm_status bsgemm_make_plan(int layout, int64_t M, int64_t N, int6
   if (!plan || num_sms <= 0) return BSGEMM_ERR_INVALID_ARG;
   if (layout < BSGEMM_LAYOUT_NT || layout > BSGEMM_LAYOUT_TT) return BSGEMM_ERR_INVALID_ARG;
   if (M <= 0 || N <= 0 || K <= 0) return BSGEMM_ERR_INVALID_ARG;
+  if (M > (1 << 30) || N > (1 << 30) || K > (1 << 30)) return BSGEMM_ERR_INVALID_ARG;
   if (gran != 64 && gran != 128 && gran != 256) return BSGEMM_ERR_UNSUPPORTED_GRAN;
   bsgemm_plan pl{};
   const int Kb = static_cast<int>((K + gran - 1) / gran);
@@ -289,6 +290,7 @@ extern "C" bsgemm_status bsgemm_make_plan(int layout, int64_t M, int64_t N, int6
   pl.kb_per_split = per;
   const int64_t whole = pl.sk_ctas > 0 ? pl.sk_first_tile : tiles;
   int64_t work = whole * pl.splits;
+  if (work > (1 << 30)) return BSGEMM_ERR_INVALID_ARG;  // work items are counted in 32 bits
   if (work < pl.sk_ctas) work = pl.sk_ctas;
   pl.grid = static_cast<int>(work < num_sms ? work : num_sms);
   pl.group_p = 16;

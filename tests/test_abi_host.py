@@ -233,3 +233,20 @@ def test_binding_rejects_host_tensors_before_calling_the_library():
     with pytest.raises(ValueError):
         bsg.grouped_gemm(a, a.reshape(1, 128, 256), torch.ones((2, 2)), s,
                          torch.zeros(1, dtype=torch.int32))
+
+
+def test_plan_rejects_sizes_past_its_32_bit_counts():
+    """Tile and work-item counts are 32-bit in the launch; a size or forced
+    split count that would overflow them is refused, not truncated."""
+    for M, N, K in ((1 << 31, 256, 256), (256, (1 << 30) + 8, 256), (256, 256, 1 << 31)):
+        with pytest.raises(bsg.BsgemmError) as e:
+            bsg.make_plan(M, N, K, 128, "nt", 148)
+        assert e.value.status == 1
+    with pytest.raises(bsg.BsgemmError):          # 2^45 tiles of 128 x 256
+        bsg.make_plan(1 << 30, 1 << 30, 128, 128, "nt", 148)
+    # 2^20 tiles x 2^14 forced K splits = 2^34 work items
+    with pytest.raises(bsg.BsgemmError):
+        bsg.make_plan(1 << 20, 1 << 15, 1 << 20, 64, "nt", 148, {"splits": 1 << 14})
+    # the largest sizes themselves still plan
+    pl = bsg.make_plan(1 << 30, 256, 1 << 30, 128, "nt", 148)
+    assert pl["tiles_p"] == (1 << 23) and pl["tiles_q"] == 1 and pl["splits"] == 1
