@@ -263,3 +263,199 @@ def test_model_catches_planted_protocol_mistakes(mutation):
                 caught = True
                 break
         assert caught, (mutation, bnq, q_mn, gran)
+
+
+# ---------------------------------------------------------------- CTA pairs
+# ``csrc/bsgemm_pair.cuh``: both CTAs' producers wait their own empty[s] and
+# load their halves of stage s; both copies complete on the even CTA's full[s],
+# whose phase also needs the even producer's arrive (with the byte count). The
+# even CTA's MMA warp waits full[s] and its tmem_empty[b], issues the pair MMAs
+# and commits to both CTAs' tmem_full[b] and empty[s]. Each CTA's promotion warps
+# wait their own tmem_full[b] and arrive on the even CTA's tmem_empty[b], whose
+# phase needs both CTAs' arrivals.
+PAIR_STAGES = min(8, BUDGET // (2 * 128 * BK))   # 16 KB of A and 16 KB of B per stage: 7
+PAIR_BUFS = 2
+
+
+class PhaseBar:
+    """A barrier whose phase completes when every expected contribution of that
+    phase has arrived; a contribution meant for another phase is an error."""
+    __slots__ = ("c", "need", "got")
+
+    def __init__(self, need):
+        self.c, self.need, self.got = 0, set(need), set()
+
+    def passes(self, k):
+        return (self.c & 1) != (k & 1)
+
+    def add(self, who, phase, errors, what):
+        if phase != self.c:
+            errors.append(f"{what}: contribution for phase {phase} arrived during phase {self.c}")
+            return
+        self.got.add(who)
+        if self.got >= self.need:
+            self.c += 1
+            self.got = set()
+
+
+def simulate_pair(gran, K, tiles, rng, mutation=None):
+    S, B = PAIR_STAGES, PAIR_BUFS
+    errors = []
+
+    def check(bar, k, what):
+        if bar.c != k + 1:
+            errors.append(f"{what}: waited for phase {k}, count was {bar.c}")
+
+    nst = -(-K // BK)
+    Kb = -(-K // gran)
+    items = [(0, Kb)] * tiles
+    full = [PhaseBar({"arrive", "land0", "land1"}) for _ in range(S)]
+    empty = [[Bar() for _ in range(S)] for _ in range(2)]
+    tfull = [[Bar() for _ in range(B)] for _ in range(2)]
+    tempty = [PhaseBar({0, 1} if mutation != "tmem_empty_one_cta" else {0}) for _ in range(B)]
+    mma = []
+    for kb0, kb1 in items:
+        for kb in range(kb0, kb1):
+            if gran >= BK:
+                for j in range(gran // BK):
+                    k0 = kb * gran + j * BK
+                    if k0 >= K:
+                        break
+                    mma.append((True, j == 0, j == gran // BK - 1 or k0 + BK >= K, True))
+            else:
+                k0 = kb * gran
+                mma.append(((kb & 1) == 0, True, True, (kb & 1) == 1 or k0 + gran >= K))
+    nprod = nst * tiles
+    nblocks = Kb * tiles
+
+    p_it = [0, 0]
+    landing = []
+    landed = [set(), set()]
+    m_i = m_st = m_blk = m_sub = 0
+    inflight = []
+    promo = [0, 0]
+    reading = [0] * S
+    stage_done = 0
+    blocks_done = 0
+    slow = {r for r in ("prod0", "prod1", "land", "mma", "m_done", "promo0", "promo1") if rng.random() < 0.3}
+    guard = 0
+    while min(promo) < nblocks and not errors:
+        guard += 1
+        if guard > 400000:
+            errors.append("no progress")
+            break
+        acts = []
+        for r in (0, 1):
+            if p_it[r] < nprod:
+                it = p_it[r]
+                k = it // S - 1
+                if k < 0 or (r == 1 and mutation == "odd_skips_stage_wait") or empty[r][it % S].passes(k):
+                    acts.append(("prod", r))
+        if landing:
+            acts.append(("land",))
+        if m_i < len(mma):
+            wf, wt, _, _ = mma[m_i]
+            if m_sub == 0 and wf:
+                if full[m_st % S].passes(m_st // S):
+                    acts.append(("m_full",))
+            else:
+                b, k = m_blk % B, m_blk // B - 1
+                if not wt or k < 0 or tempty[b].passes(k):
+                    acts.append(("m_issue",))
+        if inflight:
+            acts.append(("m_done",))
+        for r in (0, 1):
+            if promo[r] < nblocks and tfull[r][promo[r] % B].passes(promo[r] // B):
+                acts.append(("promo", r))
+        if not acts:
+            errors.append(f"deadlock: producers {p_it}/{nprod}, mma {m_i}/{len(mma)}, promotion {promo}")
+            break
+
+        def role(a):
+            return {"prod": f"prod{a[1] if len(a) > 1 else ''}", "promo": f"promo{a[1] if len(a) > 1 else ''}",
+                    "m_full": "mma", "m_issue": "mma"}.get(a[0], a[0])
+        a = rng.choices(acts, [0.03 if role(x) in slow else 1.0 for x in acts])[0]
+        if a[0] == "prod":
+            r = a[1]
+            it = p_it[r]
+            if (reading[it % S] or stage_done < it - S + 1):
+                errors.append(f"producer {r} slot {it}: stage {it % S} overwritten while in use")
+            if r == 0:
+                full[it % S].add("arrive", it // S, errors, f"even producer slot {it}")
+            landing.append((r, it))
+            p_it[r] += 1
+        elif a[0] == "land":
+            r, it = landing.pop(rng.randrange(len(landing)))
+            landed[r].add(it)
+            full[it % S].add(f"land{r}", it // S, errors, f"copy of CTA {r} slot {it}")
+        elif a[0] == "m_full":
+            check(full[m_st % S], m_st // S, f"mma step {m_i} (full)")
+            m_sub = 1
+        elif a[0] == "m_issue":
+            wf, wt, ctf, cem = mma[m_i]
+            if wt and m_blk // B - 1 >= 0:
+                check(tempty[m_blk % B], m_blk // B - 1, f"mma step {m_i} (tmem_empty)")
+            if m_st not in landed[0] or m_st not in landed[1]:
+                errors.append(f"mma step {m_i}: stage slot {m_st} read before both copies landed")
+            if wt and min(promo) < m_blk - B + 1:
+                errors.append(f"mma step {m_i}: buffer {m_blk % B} rewritten before block "
+                              f"{m_blk - B} was promoted in both CTAs")
+            reading[m_st % S] += 1
+            if mutation == "early_release" and cem:
+                for r in (0, 1):
+                    empty[r][m_st % S].c += 1
+                stage_done += 1
+                cem = False
+            inflight.append((m_blk % B if ctf else None, m_st % S if cem else None, m_st % S))
+            if ctf:
+                m_blk += 1
+            if mma[m_i][3]:
+                m_st += 1
+            m_i += 1
+            m_sub = 0
+        elif a[0] == "m_done":
+            tb, es, rs = inflight.pop(0)
+            reading[rs] -= 1
+            if tb is not None:
+                for r in ((0,) if mutation == "tmem_full_even_only" else (0, 1)):
+                    tfull[r][tb].c += 1
+                blocks_done += 1
+            if es is not None:
+                for r in (0, 1):
+                    empty[r][es].c += 1
+                stage_done += 1
+        else:
+            r = a[1]
+            blk = promo[r]
+            check(tfull[r][blk % B], blk // B, f"promotion of CTA {r}, block {blk}")
+            if blocks_done < blk + 1:
+                errors.append(f"promotion of CTA {r}, block {blk}: read an unfinished partial")
+            if mutation == "tmem_empty_one_cta" and r == 1:
+                pass            # the planted mistake: the odd CTA's arrival is not counted
+            else:
+                tempty[blk % B].add(r, blk // B, errors, f"promotion of CTA {r}, block {blk}")
+            promo[r] += 1
+    if not errors and (m_i != len(mma) or p_it != [nprod, nprod]):
+        errors.append("roles finished out of step")
+    return errors
+
+
+@pytest.mark.parametrize("gran", [64, 128, 256])
+def test_pair_handoff_never_aliases_or_deadlocks(gran):
+    rng = random.Random(77 + gran)
+    for _ in range(150):
+        K = rng.choice([BK, 2 * BK, 3 * BK, 5 * BK + 16, 9 * BK + 64, 17 * BK])
+        errors = simulate_pair(gran, K, rng.randint(1, 3), rng)
+        assert not errors, (gran, K, errors[0])
+
+
+PAIR_MUTATIONS = ["odd_skips_stage_wait", "tmem_full_even_only", "tmem_empty_one_cta", "early_release"]
+
+
+@pytest.mark.parametrize("mutation", PAIR_MUTATIONS)
+def test_pair_model_catches_planted_mistakes(mutation):
+    rng = random.Random(len(mutation))
+    for gran in (64, 128, 256):
+        caught = any(simulate_pair(gran, rng.choice([9 * BK, 17 * BK]), rng.randint(1, 3), rng, mutation)
+                     for _ in range(300))
+        assert caught, (mutation, gran)
