@@ -90,7 +90,9 @@ bsgemm_status device_info(DeviceInfo& out) {
 
 // Workspace of at least `ws_bytes` and `n_counters` zeroed counters for
 // (current device, stream). Growing frees the old buffers (cudaFree waits for
-// the device, so no launch still uses them).
+// the device, so no launch still uses them). New counters are zeroed on the
+// call's own stream: a memset on the legacy default stream would not be
+// ordered before the kernel when the caller's stream is non-blocking.
 bsgemm_status get_workspace(cudaStream_t stream, size_t ws_bytes, size_t n_counters, Workspace& out) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return BSGEMM_ERR_CUDA;
@@ -110,7 +112,7 @@ bsgemm_status get_workspace(cudaStream_t stream, size_t ws_bytes, size_t n_count
     w.n_counters = 0;
     size_t want = n_counters < 1024 ? 1024 : n_counters * 2;
     if (cudaMalloc(&w.counters, want * sizeof(int)) != cudaSuccess) return BSGEMM_ERR_CUDA;
-    if (cudaMemset(w.counters, 0, want * sizeof(int)) != cudaSuccess) return BSGEMM_ERR_CUDA;
+    if (cudaMemsetAsync(w.counters, 0, want * sizeof(int), stream) != cudaSuccess) return BSGEMM_ERR_CUDA;
     w.n_counters = want;
   }
   out = w;
