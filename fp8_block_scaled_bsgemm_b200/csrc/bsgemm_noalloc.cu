@@ -209,10 +209,18 @@ extern "C" bsgemm_status bsgemm_fp8_nt_noalloc(const void* a, const void* b, con
   DeviceScratch* d = nullptr;
   bsgemm_status st = setup_current_device(d);
   if (st != BSGEMM_OK) return st;
-  // the regular plan when its scratch fits; otherwise the plan without stream-K
+  // the regular plan when its scratch fits; otherwise the plan without stream-K.
+  // This entry point launches single-CTA tiles only: where the regular plan
+  // takes CTA pairs (large g = 256 problems), it takes 128-row data-parallel
+  // tiles instead.
   bsgemm_plan pl;
   st = bsgemm_make_plan(BSGEMM_LAYOUT_NT, M, N, K, gran, d->num_sms, nullptr, &pl);
   if (st != BSGEMM_OK) return st;
+  if (pl.cta_pair) {
+    const bsgemm_tuning dp = {BSGEMM_VARIANT_DATA_PARALLEL, 0, 0, 0};
+    st = bsgemm_make_plan(BSGEMM_LAYOUT_NT, M, N, K, gran, d->num_sms, &dp, &pl);
+    if (st != BSGEMM_OK) return st;
+  }
   if (!fits(pl)) {
     const bsgemm_tuning no_sk = {0, 0, 0, -1};
     st = bsgemm_make_plan(BSGEMM_LAYOUT_NT, M, N, K, gran, d->num_sms, &no_sk, &pl);

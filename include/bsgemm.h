@@ -300,8 +300,10 @@ bsgemm_status bsgemm_diag_wait_timeout(unsigned long long timeout_ns, bsgemm_str
  * (no cudaMalloc, cudaFree or allocating library call, torch's included).
  *
  * It computes exactly what bsgemm_fp8_nt computes, with the same arguments,
- * rules and errors, and with the same kernels.  It takes the same plan when
- * that plan's scratch fits the array, otherwise the plan without stream-K.
+ * rules and errors, and with the same single-CTA kernels.  It takes the same
+ * plan when that plan's scratch fits the array, otherwise the plan without
+ * stream-K; where the regular plan pairs CTAs (large g = 256 problems) it
+ * takes 128-row data-parallel tiles instead.
  * Its split-K / stream-K scratch is a fixed array inside the library's device
  * memory: each GPU that loads
  * the library holds BSGEMM_NOALLOC_SCRATCH_BYTES of FP32 partial tiles plus

@@ -250,3 +250,16 @@ def test_plan_rejects_sizes_past_its_32_bit_counts():
     # the largest sizes themselves still plan
     pl = bsg.make_plan(1 << 30, 256, 1 << 30, 128, "nt", 148)
     assert pl["tiles_p"] == (1 << 23) and pl["tiles_q"] == 1 and pl["splits"] == 1
+
+
+def test_allocation_free_plan_never_pairs_ctas():
+    """bsgemm_fp8_nt_noalloc launches single-CTA tiles only. Where the regular
+    plan pairs CTAs (large g = 256 problems) it re-plans with the data-parallel
+    variant named, which keeps the regular stream-K choice and has no pairs."""
+    pl = bsg.make_plan(2304, 2304, 1024, 256, "nt", 148)
+    assert pl["cta_pair"] == 1 and (pl["tiles_p"], pl["tiles_q"]) == (9, 9)
+    dp = bsg.make_plan(2304, 2304, 1024, 256, "nt", 148, {"variant": "data_parallel"})
+    assert dp["cta_pair"] == 0 and dp["swap_ab"] == 0 and dp["bnq"] == 256
+    assert (dp["tiles_p"], dp["tiles_q"]) == (18, 9)
+    # the fallback plan without stream-K never pairs either
+    assert bsg.make_plan(2304, 2304, 1024, 256, "nt", 148, {"stream_k": -1})["cta_pair"] == 0

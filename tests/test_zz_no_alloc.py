@@ -32,9 +32,12 @@ def _num_sms():
 
 
 def _fixed_plan(M, N, K, g):
-    """The plan the allocation-free entry point takes: the regular one when its
-    scratch fits the fixed array, otherwise the one without stream-K."""
+    """The plan the allocation-free entry point takes: the regular one (with
+    128-row tiles where that one pairs CTAs) when its scratch fits the fixed
+    array, otherwise the one without stream-K."""
     plan = bsg.make_plan(M, N, K, g, "nt", _num_sms())
+    if plan["cta_pair"]:
+        plan = bsg.make_plan(M, N, K, g, "nt", _num_sms(), {"variant": "data_parallel"})
     if bsg.scratch_bytes(plan) > LIMIT_BYTES:
         plan = bsg.make_plan(M, N, K, g, "nt", _num_sms(), {"stream_k": -1})
     return plan
@@ -61,6 +64,28 @@ def test_no_alloc_matches_regular_entry_point_twice(M, N, K, g):
         assert _call(L.bsgemm_fp8_nt_noalloc, a, b, sa, sb, got, M, N, K, g) == 0
         torch.cuda.synchronize()
         check_close(gpu_as_f64(got), ref, f"allocation-free call {call}, {M}x{N}x{K} g={g}")
+    assert bsg.get_last_device_status() == 0
+
+
+def test_no_alloc_takes_single_cta_tiles_where_the_regular_plan_pairs():
+    """Large g = 256 problems get CTA-pair tiles from the regular entry point; the
+    allocation-free one has no pair kernel and takes 128-row tiles, with the same
+    product and every row written."""
+    M, N, K, g = 2304, 2304, 1024, 256
+    if not bsg.make_plan(M, N, K, g, "nt", _num_sms())["cta_pair"]:
+        pytest.skip("the regular plan does not pair CTAs on this device")
+    assert _fixed_plan(M, N, K, g)["cta_pair"] == 0
+    p = workloads.make_problem(M, N, K, g, "nt", seed=32)
+    a, b, sa, sb = to_device(p)
+    L = bsg.lib()
+    want = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+    assert _call(L.bsgemm_fp8_nt, a, b, sa, sb, want, M, N, K, g) == 0
+    torch.cuda.synchronize()
+    got = torch.full((M, N), float("nan"), dtype=torch.bfloat16, device="cuda")
+    assert _call(L.bsgemm_fp8_nt_noalloc, a, b, sa, sb, got, M, N, K, g) == 0
+    torch.cuda.synchronize()
+    assert not torch.isnan(got).any()
+    check_close(gpu_as_f64(got), gpu_as_f64(want), f"allocation-free call, {M}x{N}x{K} g={g}")
     assert bsg.get_last_device_status() == 0
 
 
