@@ -263,3 +263,71 @@ def test_allocation_free_plan_never_pairs_ctas():
     assert (dp["tiles_p"], dp["tiles_q"]) == (18, 9)
     # the fallback plan without stream-K never pairs either
     assert bsg.make_plan(2304, 2304, 1024, 256, "nt", 148, {"stream_k": -1})["cta_pair"] == 0
+
+
+def _cdiv(a, b):
+    return -(-a // b)
+
+
+def _grouped_walk(ms, tiles_q, grid, gran):
+    """Mirror of the grouped kernel's work cursor (work_begin / group_seek /
+    work_next with GROUPED): per CTA, the (group, tp, tq, g_row, g_srow, g_m)
+    of each tile it takes."""
+    BM = 128
+    items = []
+    for cta in range(grid):
+        wi, g, g_first, g_row, g_srow = cta, 0, 0, 0, 0
+        g_m = max(0, ms[0])
+        g_tiles = _cdiv(g_m, BM) * tiles_q
+        while True:
+            alive = True
+            while wi >= g_first + g_tiles:
+                g_first += g_tiles
+                g_row += g_m
+                g_srow += _cdiv(g_m, gran)
+                g += 1
+                if g >= len(ms):
+                    alive = False
+                    break
+                g_m = max(0, ms[g])
+                g_tiles = _cdiv(g_m, BM) * tiles_q
+            if not alive:
+                break
+            lt = wi - g_first
+            tiles_p = _cdiv(g_m, BM)
+            items.append((cta, g, lt % tiles_p, lt // tiles_p, g_row, g_srow, g_m))
+            wi += grid
+    return items
+
+
+@pytest.mark.parametrize("seed", range(6))
+def test_grouped_cursor_covers_each_tile_once_inside_its_group(seed):
+    import random
+    rng = random.Random(seed)
+    for _ in range(25):
+        G = rng.randint(1, 12)
+        ms = [rng.choice([0, 0, 1, 5, 127, 128, 129, 300, 513]) for _ in range(G)]
+        gran = rng.choice([64, 128, 256])
+        bnq = rng.choice([128, 256])
+        N = rng.choice([128, 256, 384, 1000])
+        tiles_q = _cdiv(N, bnq)
+        max_rows = sum(ms) + rng.choice([0, 1, 40])
+        grid = rng.choice([1, 3, 148])
+        items = _grouped_walk(ms, tiles_q, grid, gran)
+        want = {(g, tp, tq) for g, m in enumerate(ms) for tp in range(_cdiv(m, 128)) for tq in range(tiles_q)}
+        got = [(g, tp, tq) for _, g, tp, tq, _, _, _ in items]
+        assert len(got) == len(set(got)) and set(got) == want, (ms, grid)
+        Pb = _cdiv(max_rows, gran) + G          # scale_a rows the call documents
+        for _, g, tp, tq, g_row, g_srow, g_m in items:
+            assert g_row == sum(ms[:g]) and g_m == ms[g]
+            assert g_srow == sum(_cdiv(m, gran) for m in ms[:g])
+            # each promotion warp's scale row (clamped as the kernel does) is one of
+            # the group's own rows, inside the documented scale_a bound
+            last = max(0, (g_m - 1) // gran)
+            for quad in range(4):
+                pb = g_srow + min((tp * 128 + quad * 32) // gran, last)
+                pb = min(pb, Pb - 1)
+                assert g_srow <= pb <= g_srow + _cdiv(g_m, gran) - 1 <= Pb - 1
+            # rows stored: the tile's rows that lie in the group, all below max_rows
+            lo, hi = g_row + tp * 128, g_row + min(g_m, tp * 128 + 128)
+            assert g_row <= lo < hi <= g_row + g_m <= max_rows
