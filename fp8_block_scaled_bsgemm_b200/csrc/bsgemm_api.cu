@@ -188,7 +188,8 @@ extern "C" bsgemm_status bsgemm_make_plan(int layout, int64_t M, int64_t N, int6
     // 256 x 256 tiles (long_k g = 256: 219 vs 234 us), not at g = 128.
     const bool tuned = t && (t->bnq != 0 || t->splits != 0 || t->stream_k != 0);
     const int64_t pair_tiles = ((M + 255) / 256) * ((N + 255) / 256);
-    if (!tuned && gran == 256 && M > 128 && pair_tiles >= num_sms / 2) variant = BSGEMM_VARIANT_CTA_PAIR;
+    if (!tuned && gran == 256 && M > 128 && num_sms >= 2 && pair_tiles >= num_sms / 2)
+      variant = BSGEMM_VARIANT_CTA_PAIR;
   }
   if (variant == BSGEMM_VARIANT_CTA_PAIR) {
     // 256 x 256 tiles on CTA pairs, whole tiles walked by persistent pairs

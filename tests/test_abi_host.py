@@ -331,3 +331,13 @@ def test_grouped_cursor_covers_each_tile_once_inside_its_group(seed):
             # rows stored: the tile's rows that lie in the group, all below max_rows
             lo, hi = g_row + tp * 128, g_row + min(g_m, tp * 128 + 128)
             assert g_row <= lo < hi <= g_row + g_m <= max_rows
+
+
+def test_automatic_plan_works_for_any_sm_count():
+    """The heuristic only pairs CTAs where pairs can run (two SMs or more); the
+    plan for one SM is a plain single-CTA plan."""
+    for sms in (1, 2, 3, 148):
+        for M, N, K, g in ((4096, 4096, 4096, 256), (1, 7168, 7168, 128), (300, 200, 64, 64)):
+            pl = bsg.make_plan(M, N, K, g, "nt", sms)
+            assert 1 <= pl["grid"] <= sms
+            assert pl["cta_pair"] == 0 or sms >= 2
