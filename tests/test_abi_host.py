@@ -341,3 +341,30 @@ def test_automatic_plan_works_for_any_sm_count():
             pl = bsg.make_plan(M, N, K, g, "nt", sms)
             assert 1 <= pl["grid"] <= sms
             assert pl["cta_pair"] == 0 or sms >= 2
+
+
+def _tile_coords(tiles_p, tiles_q, group_p, tile):
+    """Mirror of the kernels' grouped raster (tile_coords)."""
+    per_group = group_p * tiles_q
+    grp = tile // per_group
+    first_p = grp * group_p
+    rows = min(tiles_p - first_p, group_p)
+    local = tile - grp * per_group
+    return first_p + local % rows, local // rows
+
+
+@pytest.mark.parametrize("group_p", [1, 8, 16])
+def test_raster_maps_work_items_onto_the_tile_grid_one_to_one(group_p):
+    """Every tile index in [0, tiles) names a distinct tile of the grid (the
+    last, shorter group of rows included), and the tiles a group's CTAs take
+    together share their B (Q-side) tile column."""
+    import random
+    rng = random.Random(group_p)
+    for _ in range(200):
+        tp_n, tq_n = rng.randint(1, 70), rng.randint(1, 70)
+        seen = [_tile_coords(tp_n, tq_n, group_p, t) for t in range(tp_n * tq_n)]
+        assert sorted(seen) == [(a, b) for a in range(tp_n) for b in range(tq_n)]
+        for t in range(tp_n * tq_n - 1):
+            (a0, b0), (a1, b1) = seen[t], seen[t + 1]
+            if a1 == a0 + 1:                 # next row of the same group: same B column
+                assert b1 == b0
