@@ -364,7 +364,8 @@ def test_raster_maps_work_items_onto_the_tile_grid_one_to_one(group_p):
         tp_n, tq_n = rng.randint(1, 70), rng.randint(1, 70)
         seen = [_tile_coords(tp_n, tq_n, group_p, t) for t in range(tp_n * tq_n)]
         assert sorted(seen) == [(a, b) for a in range(tp_n) for b in range(tq_n)]
+        per_group = group_p * tq_n
         for t in range(tp_n * tq_n - 1):
             (a0, b0), (a1, b1) = seen[t], seen[t + 1]
-            if a1 == a0 + 1:                 # next row of the same group: same B column
-                assert b1 == b0
+            if t // per_group == (t + 1) // per_group and a1 == a0 + 1:
+                assert b1 == b0              # next row of the same group: same B column
