@@ -89,3 +89,28 @@ def test_peaks_fall_back_without_a_measured_file(monkeypatch):
         assert pk == {"hbm_gbs": 7000.5, "bf16_tflops": 1600.25, "source": "measured"}
     finally:
         shutil.rmtree(d, ignore_errors=True)
+
+
+def test_reference_arm_prints_one_contract_line(capsys, monkeypatch):
+    """bench.py --impl reference (the oracle, on host cores) on the tiny
+    workload: one JSON line with the contract's keys, no GPU touched."""
+    import json
+    monkeypatch.delenv("RANK", raising=False)
+    bench.main(["--impl", "reference", "--workload", "tiny", "--steps", "1", "--warmup", "0",
+                "--cpu-seconds", "0.5"])
+    lines = [ln for ln in capsys.readouterr().out.splitlines() if ln.strip()]
+    assert len(lines) == 1
+    d = json.loads(lines[0])
+    for key in ("impl", "metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step",
+                "higher_is_better", "scaling", "vs_baseline", "dtype", "data", "config",
+                "cpu_baseline", "e2e"):
+        assert key in d, key
+    assert d["impl"] == "reference" and d["value"] > 0 and d["unit"] == "TFLOP/s"
+    assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["cores"] >= 1
+    assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["config"]["workload"]
+
+
+def test_reference_arm_runs_on_rank_zero_only(capsys, monkeypatch):
+    monkeypatch.setenv("RANK", "1")
+    bench.main(["--impl", "reference", "--workload", "tiny", "--steps", "1", "--warmup", "0"])
+    assert capsys.readouterr().out.strip() == ""
