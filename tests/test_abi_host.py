@@ -190,6 +190,21 @@ def test_register_split_kernels_have_the_planned_launch_registers():
     # instance in each of the 3 NT units; one CTA-pair kernel per unit
     assert seen == 24 + 3
     assert pairs == 12
+    # the allocation-free unit instantiates its own split kernels: one
+    # 256-wide instance per granularity, under the same rule
+    wide = 0
+    cur = None
+    for ln in open(os.path.join(ROOT, "_build", "bsgemm_noalloc.o.log")):
+        m = re.search(r"Compiling entry function '_ZN3bsg13bsgemm_kernelILi(\d+)E", ln)
+        if m:
+            cur = int(m.group(1))
+            continue
+        if cur is not None and "Used" in ln:
+            regs = int(re.search(r"Used (\d+) registers", ln).group(1))
+            assert regs == 168 if cur == 256 else regs <= 168, ln
+            wide += cur == 256
+            cur = None
+    assert wide == 3
 
 
 def test_new_entry_points_reject_bad_arguments_on_the_host():
