@@ -39,8 +39,7 @@
  *   - term = blocksum * 2^-(qa+qb) * (sA*sB) is one FP64 rounding, and the
  *     terms are added in ascending kb in FP64.
  *
- * Readings of points the pages leave open (each one is also listed in the
- * design notes): both operands use g x g blocks; the scale tensors are
+ * Readings of points the pages leave open: both operands use g x g blocks; the scale tensors are
  * row-major FP32 [ceil(rows/g)][ceil(K/g)] in logical block coordinates for
  * every storage layout; a partial last block (rows or K not a multiple of g)
  * simply has fewer terms; for the layout flags the first letter is A and the
