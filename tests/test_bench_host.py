@@ -114,3 +114,24 @@ def test_reference_arm_runs_on_rank_zero_only(capsys, monkeypatch):
     monkeypatch.setenv("RANK", "1")
     bench.main(["--impl", "reference", "--workload", "tiny", "--steps", "1", "--warmup", "0"])
     assert capsys.readouterr().out.strip() == ""
+
+
+def test_clock_summary_reports_median_clock_and_active_throttle_reasons():
+    """The clocks key: median SM MHz under load, the max clock, and the names of
+    the throttle reasons nvidia-smi reported active during the timed region."""
+    base = os.path.join(ROOT, "_build")
+    os.makedirs(base, exist_ok=True)
+    fd, path = tempfile.mkstemp(prefix="clocks_", suffix=".csv", dir=base)
+    os.close(fd)
+    with open(path, "w") as f:
+        f.write("0, 1965, 1965, 700.50, 0x0000000000000000, Not Active, Not Active, Not Active, Not Active\n"
+                "0, 1800, 1965, 990.10, 0x0000000000000004, Not Active, Not Active, Not Active, Active\n"
+                "0, 1950, 1965, 980.00, 0x0000000000000000, Not Active, Not Active, Not Active, Not Active\n"
+                "garbage line\n")
+    cs = bench.ClockSampler(0)
+    cs.proc, cs.path = object(), path          # as if nvidia-smi had run
+    s = cs.summary()
+    assert s == {"sm_mhz": 1950.0, "sm_max_mhz": 1965.0, "reasons": ["sw_power_cap"], "samples": 3}
+    assert not os.path.exists(path)
+    cs2 = bench.ClockSampler(0)                # nvidia-smi missing: no clocks key value
+    assert cs2.summary() is None
