@@ -27,3 +27,17 @@ def pytest_collection_modifyitems(config, items):
     for item in items:
         if "gpu" in item.keywords:
             item.add_marker(skip)
+
+
+def pytest_terminal_summary(terminalreporter):
+    """After a GPU run: how close the checked outputs came to the parity bound."""
+    gu = sys.modules.get("gpu_util")
+    log = getattr(gu, "PARITY_LOG", None) if gu else None
+    if not log:
+        return
+    worst = max(log, key=lambda r: r[1])
+    terminalreporter.write_sep("-", "parity against the oracle")
+    terminalreporter.write_line(
+        f"{len(log)} checks, {sum(r[3] for r in log)} elements compared; worst max err/tol "
+        f"{worst[1]:.3f} ({worst[0]}); largest fraction of elements above half the tolerance "
+        f"{max(r[2] for r in log):.4f}")

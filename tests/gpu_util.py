@@ -44,6 +44,11 @@ def tolerance(ref: np.ndarray) -> np.ndarray:
     return 2.0 ** -7 * np.abs(ref) + 2.0 ** -8 * rms
 
 
+# One record per passing check: (what, max err/tol, fraction of elements above
+# half the tolerance, elements compared). The session summary prints the worst.
+PARITY_LOG = []
+
+
 def check_close(got: np.ndarray, ref: np.ndarray, what=""):
     tol = tolerance(ref)
     err = np.abs(got - ref)
@@ -53,7 +58,11 @@ def check_close(got: np.ndarray, ref: np.ndarray, what=""):
         raise AssertionError(f"{what}: {int(bad.sum())} of {ref.size} elements out of tolerance; "
                              f"max err/tol {float(np.nanmax(err / np.maximum(tol, 1e-300))):.3g}; "
                              f"first {idx.tolist()} got {got[bad][:8]} want {ref[bad][:8]}")
-    return float(np.max(err / np.maximum(tol, 1e-300))) if ref.size else 0.0
+    if not ref.size:
+        return 0.0
+    ratio = float(np.max(err / np.maximum(tol, 1e-300)))
+    PARITY_LOG.append((what, ratio, float(np.mean(err > 0.5 * tol)), int(ref.size)))
+    return ratio
 
 
 def full_parity(p: workloads.Problem, tuning=None, what=""):
