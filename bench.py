@@ -10,14 +10,20 @@ Default workload: the square 4096^3 NT GEMM with 128x128 block scales and 41
 outlier rows of A (x50).  Other workloads (``--workload``): tiny, ffn, ffn_tn,
 ffn_tt, small_m:<M>, long_k:<g>.
 
-Timing: W warm-up steps, then K timed steps.  Inputs are resident in HBM; the
-L2 cache is flushed (a 512 MiB memset) before every timed step, outside the
-events that bracket the GEMM itself.  CUDA events on the launching stream give
-the device time of each launch; the reported time per step is their mean and
-the whole-job value is total FLOPs / time, max over ranks.  ``e2e`` repeats the
-measurement through the public API with the inputs in pinned host memory:
-host->device copies, the GEMM and the device->host copy of the output are all
-inside the timed region.
+Timing: W warm-up launches, then K timed launches.  Inputs are resident in
+HBM.  By default the launches cycle over R >= 3 copies of the inputs at
+distinct addresses (R x set size >= 2x L2), so no launch finds its operands in
+L2; the K launches are captured once in a CUDA graph and replayed between two
+CUDA events on the launching stream (the host's per-call overhead never
+starves the GPU), and the time per step is the span / K.  ``--l2 flush``
+instead flushes L2 with a 512 MiB memset before each launch and brackets each
+launch with its own events.  The whole-job value is total FLOPs / time, max
+over ranks.  The default run also measures the HBM-bound small-M shapes
+(``--hbm-points``, M x 7168 x 7168) the same way and reports them under
+``hbm_bound`` with their own roofline.  ``e2e`` repeats the main workload
+through the public API with the inputs in pinned host memory: host->device
+copies, the GEMM and the device->host copy of the output are all inside the
+timed region.
 
 Multi-GPU (torchrun, one rank per GPU): every rank runs the same GEMM on its
 own GPU (replicas; the GEMM has no exchange step), the step time is the max
@@ -57,6 +63,13 @@ def parse_args(argv=None):
     ap.add_argument("--workload", default="square")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--l2", default="rotate", choices=["rotate", "flush"],
+                    help="keep operands out of L2 by rotating input sets (default) or by a memset per launch")
+    ap.add_argument("--quantize-a", action="store_true",
+                    help="each step first quantises A from BF16 with the library's quantiser, then runs "
+                         "the GEMM (NT layouts): the two-kernel activation pipeline")
+    ap.add_argument("--hbm-points", default="1,128",
+                    help="small-M sizes (M of M x 7168 x 7168) also measured and reported in the line; '' for none")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="target CPU seconds of the oracle sample")
     ap.add_argument("--variant", default="auto", choices=["auto", "data_parallel", "swap_ab", "cta_pair"],
@@ -87,10 +100,10 @@ def make_workload(name: str) -> workloads.Problem:
     raise SystemExit(f"unknown workload {name}")
 
 
-def workload_config(p: workloads.Problem, name: str) -> dict:
+def workload_config(p: workloads.Problem, name: str, l2_mode: str = "rotate") -> dict:
     return {"workload": p.name, "name": name, "M": p.M, "N": p.N, "K": p.K, "gran": p.gran,
             "layout": p.layout, "inputs": "E4M3 codes + FP32 block scales, seeded synthetic",
-            "l2": "flushed (512 MiB memset) before every timed step"}
+            "l2": l2_note(l2_mode)}
 
 
 def algorithmic_bytes(p: workloads.Problem) -> int:
@@ -278,53 +291,163 @@ def job_tflops(flops_per_rank: int, world: int, ms_max: float) -> float:
 
 
 # ---------------------------------------------------------------- our arm
+def input_sets(p: workloads.Problem, dev, l2_bytes: int, mode: str):
+    """Device copies of the workload's inputs (and an output each).
+
+    mode "rotate": R >= 3 copies at distinct addresses, R large enough that
+    the copies together are at least twice the L2 size, so by the time a
+    launch comes back to a copy the cache holds none of it.  mode "flush":
+    one copy (the L2 is flushed before every launch instead)."""
+    import torch
+    a = torch.from_numpy(p.a).to(dev)
+    b = torch.from_numpy(p.b).to(dev)
+    sa = torch.from_numpy(p.sa).to(dev)
+    sb = torch.from_numpy(p.sb).to(dev)
+    per_set = sum(x.numel() * x.element_size() for x in (a, b, sa, sb)) + 2 * p.M * p.N
+    r = 1 if mode == "flush" else max(3, -(-2 * l2_bytes // per_set))
+    sets = []
+    for i in range(r):
+        cp = (a, b, sa, sb) if i == 0 else tuple(x.clone() for x in (a, b, sa, sb))
+        sets.append(cp + (torch.empty((p.M, p.N), dtype=torch.bfloat16, device=dev),))
+    return sets, per_set
+
+
+def l2_note(mode: str) -> str:
+    if mode == "flush":
+        return "flushed (512 MiB memset) before every timed launch, outside the events"
+    return "rotating input sets at distinct addresses, together >= 2x L2, launches back to back"
+
+
+def time_device(call, n_sets: int, steps: int, warmup: int, stream, world: int, mode: str):
+    """Device time per launch of `call(i)` (i selects the input set), in ms.
+
+    rotate: the `steps` launches are captured once in a CUDA graph and the
+    graph is replayed once between two events, so the host's call overhead
+    never leaves the GPU idle between launches; per-launch time = the span /
+    steps.  flush: each launch is bracketed by its own events after a 512 MiB
+    memset.  Returns (mean ms, per-launch ms list or None)."""
+    import torch
+    for i in range(warmup):
+        call(i % n_sets)
+    torch.cuda.synchronize()
+    if mode == "flush":
+        flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=stream.device)
+        st = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+        en = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+        barrier(world)
+        torch.cuda.synchronize()
+        for i in range(steps):
+            flush.zero_()
+            st[i].record(stream)
+            call(i % n_sets)
+            en[i].record(stream)
+        torch.cuda.synchronize()
+        barrier(world)
+        per = [s.elapsed_time(e) for s, e in zip(st, en)]
+        return sum(per) / len(per), per
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream):
+        for i in range(steps):
+            call((warmup + i) % n_sets)
+    torch.cuda.synchronize()
+    g.replay()  # the graph's own first replay uploads it; not timed
+    torch.cuda.synchronize()
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    barrier(world)
+    torch.cuda.synchronize()
+    t0.record(stream)
+    g.replay()
+    t1.record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    ms = t0.elapsed_time(t1) / steps
+    del g
+    return ms, None
+
+
+def roofline(p: workloads.Problem, ms: float, name: str, peaks: dict) -> dict:
+    """Roofline of one launch: tensor-bound (FLOPs vs the FP8 peak) for
+    M > 128, HBM-bound (algorithmic bytes vs the copy bandwidth) otherwise."""
+    if p.M > 128:
+        # FP8 dense peak = measured BF16 burst x the nominal FP8/BF16 ratio (4.5 / 2.25)
+        peak = peaks["bf16_tflops"] * 2.0
+        achieved = p.flops / (ms * 1e-3) / 1e12
+        return {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                "frac": achieved / peak, "traffic": profiled_traffic(name),
+                "peak_source": f"{peaks['source']} bf16 burst x 2 (FP8/BF16 nominal ratio)",
+                "frac_of_nominal_4500": achieved / 4500.0}
+    bytes_ = algorithmic_bytes(p)
+    peak = peaks["hbm_gbs"]
+    achieved = bytes_ / (ms * 1e-3) / 1e9
+    return {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
+            "traffic": profiled_traffic(name), "peak_source": f"{peaks['source']} hbm copy",
+            "algorithmic_bytes_per_launch": bytes_}
+
+
 def run_ours(args):
     import torch
     import fp8_block_scaled_bsgemm_b200 as bsg
 
     rank, world, local = dist_setup(args.gpus)
-    p = make_workload(args.workload)
     dev = torch.device("cuda", local if world > 1 else 0)
-    stream = torch.cuda.current_stream(dev)
-    a = torch.from_numpy(p.a).to(dev)
-    b = torch.from_numpy(p.b).to(dev)
-    sa = torch.from_numpy(p.sa).to(dev)
-    sb = torch.from_numpy(p.sb).to(dev)
-    out = torch.empty((p.M, p.N), dtype=torch.bfloat16, device=dev)
-    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
-    num_sms = torch.cuda.get_device_properties(dev).multi_processor_count
+    torch.cuda.set_device(dev)
+    stream = torch.cuda.Stream(dev)   # every launch, warm-up, capture and timing on this stream
+    props = torch.cuda.get_device_properties(dev)
+    num_sms = props.multi_processor_count
+    l2_bytes = int(getattr(props, "L2_cache_size", 126 << 20))
     tuning = None
     if args.variant != "auto" or args.bnq or args.splits or args.stream_k:
         tuning = {"variant": args.variant, "bnq": args.bnq, "splits": args.splits, "stream_k": args.stream_k}
-    plan = bsg.make_plan(p.M, p.N, p.K, p.gran, p.layout, num_sms, tuning)
+    peaks = measured_peaks()
 
-    def gemm():
-        bsg.gemm(a, b, sa, sb, out=out, layout=p.layout, gran=p.gran, tuning=tuning, stream=stream)
+    def measure(name, steps, warmup, tune, quantize_a=False):
+        p = make_workload(name)
+        sets, per_set = input_sets(p, dev, l2_bytes, args.l2)
+        plan = bsg.make_plan(p.M, p.N, p.K, p.gran, p.layout, num_sms, tune)
+        if quantize_a:
+            if p.layout[0] != "n":
+                raise SystemExit("--quantize-a needs A stored [M, K] (nt or nn)")
+            # a BF16 activation per set: the set's own A, dequantised (codes x block scales)
+            xs = []
+            for a, _, sa, _, _ in sets:
+                deq = a.view(torch.float8_e4m3fn).float()
+                sc = sa.repeat_interleave(p.gran, 0)[:p.M].repeat_interleave(p.gran, 1)[:, :p.K]
+                xs.append((deq * sc).to(torch.bfloat16))
+            per_set += p.M * p.K * 2
 
-    for _ in range(args.warmup):
-        flush.zero_()
-        gemm()
-    torch.cuda.synchronize()
-    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
-    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
-    barrier(world)
-    torch.cuda.synchronize()
-    with ClockSampler(torch.cuda.current_device()) as clk:
-        t_wall = time.perf_counter()
-        for i in range(args.steps):
-            flush.zero_()
-            starts[i].record(stream)
-            gemm()
-            ends[i].record(stream)
-        torch.cuda.synchronize()
-        t_wall = time.perf_counter() - t_wall
-    barrier(world)
-    times_ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
-    ms = sum(times_ms) / len(times_ms)
+        def call(i):
+            a, b, sa, sb, out = sets[i]
+            if quantize_a:
+                bsg.quantize(xs[i], p.gran, "e4m3", q=a, scales=sa, stream=stream)
+            bsg.gemm(a, b, sa, sb, out=out, layout=p.layout, gran=p.gran, tuning=tune, stream=stream)
+
+        with torch.cuda.stream(stream):
+            ms, per = time_device(call, len(sets), steps, warmup, stream, world, args.l2)
+        status = bsg.get_last_device_status(stream)
+        if status != 0:
+            raise SystemExit(f"device status {status} after the timed region of {name}")
+        return p, sets, plan, ms, per, per_set, call
+
+    p, sets, plan, ms, per, per_set, call = measure(args.workload, args.steps, args.warmup, tuning,
+                                                    args.quantize_a)
     ms_max = max_over_ranks(ms, world)
-    status = bsg.get_last_device_status(stream)
-    if status != 0:
-        raise SystemExit(f"device status {status} after the timed region")
+
+    # clocks under this load: the sampler covers ~0.4 s of the same launches,
+    # eager and back to back, right after the timed region (which itself is
+    # far shorter than nvidia-smi's sampling interval)
+    with ClockSampler(torch.cuda.current_device()) as clk:
+        t_soak = time.perf_counter()
+        with torch.cuda.stream(stream):
+            i = 0
+            while time.perf_counter() - t_soak < 0.4:
+                for _ in range(20):
+                    call(i % len(sets))
+                    i += 1
+                stream.synchronize()
+    clocks = clk.summary()
+    if clocks is not None:
+        clocks["window"] = "0.4 s of the benchmark's own launches, back to back, after the timed region"
 
     # ---- e2e through the public API from pinned host memory
     e2e = None
@@ -335,63 +458,68 @@ def run_ours(args):
         hsb = torch.from_numpy(p.sb).pin_memory()
         hout = torch.empty((p.M, p.N), dtype=torch.bfloat16).pin_memory()
         da, db, dsa, dsb = (torch.empty_like(x, device=dev) for x in (ha, hb, hsa, hsb))
+        dout = sets[0][4]
 
         def e2e_step():
             da.copy_(ha, non_blocking=True)
             db.copy_(hb, non_blocking=True)
             dsa.copy_(hsa, non_blocking=True)
             dsb.copy_(hsb, non_blocking=True)
-            bsg.gemm(da, db, dsa, dsb, out=out, layout=p.layout, gran=p.gran, tuning=tuning, stream=stream)
-            hout.copy_(out, non_blocking=True)
+            bsg.gemm(da, db, dsa, dsb, out=dout, layout=p.layout, gran=p.gran, tuning=tuning, stream=stream)
+            hout.copy_(dout, non_blocking=True)
 
-        for _ in range(max(1, args.warmup)):
-            e2e_step()
-        torch.cuda.synchronize()
-        es = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
-        ee = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
-        barrier(world)
-        for i in range(args.steps):
-            flush.zero_()
-            es[i].record(stream)
-            e2e_step()
-            ee[i].record(stream)
-        torch.cuda.synchronize()
-        barrier(world)
-        e_ms = max_over_ranks(sum(s.elapsed_time(e) for s, e in zip(es, ee)) / args.steps, world)
+        with torch.cuda.stream(stream):
+            for _ in range(max(1, args.warmup)):
+                e2e_step()
+            torch.cuda.synchronize()
+            es = torch.cuda.Event(enable_timing=True)
+            ee = torch.cuda.Event(enable_timing=True)
+            barrier(world)
+            torch.cuda.synchronize()
+            es.record(stream)
+            for _ in range(args.steps):
+                e2e_step()
+            ee.record(stream)
+            torch.cuda.synchronize()
+            barrier(world)
+        e_ms = max_over_ranks(es.elapsed_time(ee) / args.steps, world)
         h2d = sum(x.numel() * x.element_size() for x in (ha, hb, hsa, hsb))
         e2e = {"value": world * p.flops / (e_ms * 1e-3) / 1e12, "unit": "TFLOP/s", "ms_per_step": e_ms,
-               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": hout.numel() * hout.element_size()}
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": hout.numel() * hout.element_size(),
+               "path": "pinned host -> device copies (torch), the GEMM through the public binding "
+                       "(its C ABI takes device pointers), device -> pinned host copy of out; "
+                       "all on one stream inside the events"}
+
+    # ---- the HBM-bound half of the metric: small-M decode shapes
+    hbm_points = []
+    if args.hbm_points and world == 1:
+        for m in [int(x) for x in args.hbm_points.split(",") if x]:
+            name = f"small_m:{m}"
+            hp, hsets, hplan, hms, _, _, _ = measure(name, max(args.steps, 50), max(args.warmup, 3), None)
+            hbm_points.append({"workload": name, "config": workload_config(hp, name, args.l2),
+                               "ms_per_launch": hms, "tflops": hp.flops / (hms * 1e-3) / 1e12,
+                               "steps": max(args.steps, 50), "plan": hplan,
+                               "roofline": roofline(hp, hms, name, peaks)})
+            del hsets
 
     if rank != 0:
         _finish(world)
         return
-    peaks = measured_peaks()
-    bound = "hbm" if p.M <= 128 else "tensor"
-    if bound == "tensor":
-        # FP8 dense peak = measured BF16 burst x the nominal FP8/BF16 ratio (4.5 / 2.25)
-        peak = peaks["bf16_tflops"] * 2.0
-        achieved = p.flops / (ms * 1e-3) / 1e12
-        roof = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
-                "frac": achieved / peak, "traffic": profiled_traffic(args.workload),
-                "peak_source": f"{peaks['source']} bf16 burst x 2 (FP8/BF16 nominal ratio)",
-                "frac_of_nominal_4500": achieved / 4500.0}
-    else:
-        bytes_ = algorithmic_bytes(p)
-        peak = peaks["hbm_gbs"]
-        achieved = bytes_ / (ms * 1e-3) / 1e9
-        roof = {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
-                "frac": achieved / peak, "traffic": profiled_traffic(args.workload), "peak_source": f"{peaks['source']} hbm copy",
-                "algorithmic_bytes_per_launch": bytes_}
     line = {
         "metric": METRIC, "value": job_tflops(p.flops, world, ms_max), "unit": "TFLOP/s",
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_max,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "fp8_e4m3",
-        "data": "synthetic", "config": workload_config(p, args.workload) | {"parallelism": f"replicas{world}",
-                                                                              "plan": plan},
-        "roofline": roof, "e2e": e2e, "gpu_launches": args.steps * plan["kernels"],
-        "clocks": clk.summary(), "wall_s_timed_region": t_wall,
-        "min_ms": min(times_ms), "median_ms": statistics.median(times_ms),
+        "data": "synthetic", "config": workload_config(p, args.workload, args.l2),
+        "parallelism": f"replicas{world}", "plan": plan, "input_sets": len(sets),
+        "input_set_bytes": per_set,
+        "step": ("quantise A (BF16 -> E4M3 + block scales) + GEMM" if args.quantize_a else "GEMM"),
+        "roofline": roofline(p, ms, args.workload, peaks), "e2e": e2e,
+        "gpu_launches": args.steps * (plan["kernels"] + (1 if args.quantize_a else 0)), "clocks": clocks,
+        "hbm_bound": hbm_points,
     }
+    if per:
+        line["min_ms"] = min(per)
+        line["median_ms"] = statistics.median(per)
     if not args.no_cpu_baseline and world == 1:
         line["cpu_baseline"] = cpu_baseline(p, args.cpu_seconds)
     else:
@@ -425,7 +553,7 @@ def run_reference(args):
         "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": statistics.mean(r["seconds"] for r in per) * 1e3,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-        "data": "synthetic", "config": workload_config(p, args.workload),
+        "data": "synthetic", "config": workload_config(p, args.workload, args.l2),
         "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": oracle.num_threads(), "kind": "oracle",
                          "sample": per[-1]["sample"] + " per step"},
         "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
