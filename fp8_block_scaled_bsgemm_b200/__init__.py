@@ -64,7 +64,7 @@ EXPORTS = ("bsgemm_fp8_nt", "bsgemm_fp8_tn", "bsgemm_fp8_nn", "bsgemm_fp8_tt", "
            "bsgemm_fp8_gemm_fmt", "bsgemm_fp8_gemm_fused", "bsgemm_fp8_grouped_nt",
            "bsgemm_make_plan", "bsgemm_status_string", "bsgemm_get_last_device_status",
            "bsgemm_last_device_status_detail", "bsgemm_diag_wait_timeout", "bsgemm_version",
-           "bsgemm_fp8_nt_noalloc", "bsgemm_quantize_fp8")
+           "bsgemm_fp8_nt_noalloc", "bsgemm_quantize_fp8", "bsgemm_release_workspaces")
 
 
 def lib():
@@ -79,7 +79,7 @@ def lib():
             p, i64, i32 = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int
             gemm_args = [p, p, p, p, p, i64, i64, i64, i32, p]
             for name in ("bsgemm_fp8_nt", "bsgemm_fp8_tn", "bsgemm_fp8_nn", "bsgemm_fp8_tt",
-                         "bsgemm_fp8_nt_noalloc", "bsgemm_quantize_fp8"):
+                         "bsgemm_fp8_nt_noalloc", "bsgemm_quantize_fp8", "bsgemm_release_workspaces"):
                 getattr(L, name).argtypes = gemm_args
                 getattr(L, name).restype = i32
             L.bsgemm_fp8_gemm_ex.argtypes = [i32, p, p, p, p, p, i64, i64, i64, i32,
@@ -106,6 +106,8 @@ def lib():
             L.bsgemm_diag_wait_timeout.restype = i32
             L.bsgemm_quantize_fp8.argtypes = [i32, i32, p, i64, i64, i32, p, p, p]
             L.bsgemm_quantize_fp8.restype = i32
+            L.bsgemm_release_workspaces.argtypes = []
+            L.bsgemm_release_workspaces.restype = i32
             L.bsgemm_version.argtypes = []
             L.bsgemm_version.restype = i32
             _lib = L
@@ -335,6 +337,11 @@ def make_plan(M, N, K, gran=128, layout="nt", num_sms=148, tuning=None) -> dict:
 
 def get_last_device_status(stream=None) -> int:
     return int(lib().bsgemm_get_last_device_status(_stream_handle(stream)))
+
+
+def release_workspaces() -> int:
+    """Free the library's split-K workspaces on the current device (waits for the device)."""
+    return int(lib().bsgemm_release_workspaces())
 
 
 def diag_wait_timeout(timeout_ns: int, stream=None) -> int:

@@ -8,6 +8,7 @@
 #include <cstdint>
 #include <cstdlib>
 #include <cstring>
+#include <iterator>
 #include <map>
 #include <mutex>
 #include <utility>
@@ -58,10 +59,23 @@ bool make_map_2d(CUtensorMap* m, const void* base, CUtensorMapDataType dt, uint6
   return r == CUDA_SUCCESS;
 }
 
+bool make_out_map(CUtensorMap* m, void* out, int M, int N, bool f32) {
+  if (f32)
+    return make_map_2d(m, out, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, N, M, static_cast<uint64_t>(N) * 4, 32, 32);
+  return make_map_2d(m, out, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, N, M, static_cast<uint64_t>(N) * 2, 64, 32);
+}
+
 // ------------------------------------------------------------------ per-device state
 std::mutex g_mu;
 std::map<int, DeviceInfo> g_dev;
-std::map<std::pair<int, uintptr_t>, Workspace> g_ws;
+// Split-K workspaces, keyed by (device, the stream's process-unique id from
+// cudaStreamGetId).  Ids are never reused, so a stream created later with the
+// same handle value gets a workspace of its own.  cudaStreamGetId is not
+// called on a stream that is being captured (that would invalidate the
+// capture); there the id comes from g_ids, the last id an uncaptured call saw
+// for the (device, handle).
+std::map<std::pair<int, unsigned long long>, Workspace> g_ws;
+std::map<std::pair<int, uintptr_t>, unsigned long long> g_ids;
 
 bsgemm_status device_info(DeviceInfo& out) {
   int dev = 0;
@@ -89,29 +103,53 @@ bsgemm_status device_info(DeviceInfo& out) {
 }
 
 // Workspace of at least `ws_bytes` and `n_counters` zeroed counters for
-// (current device, stream). Growing frees the old buffers (cudaFree waits for
-// the device, so no launch still uses them). New counters are zeroed on the
-// call's own stream: a memset on the legacy default stream would not be
-// ordered before the kernel when the caller's stream is non-blocking.
+// (current device, stream).  Growing is stream-ordered on the call's own
+// stream: the old buffers are released with cudaFreeAsync after the stream's
+// earlier launches and the new ones come from cudaMallocAsync, so a growing
+// call never waits for the device or for other streams.  New counters are
+// zeroed on the same stream.  A call being captured into a CUDA graph can
+// only use the workspace an uncaptured call on the same stream already made
+// big enough (the graph would otherwise own the new memory); otherwise it
+// fails with BSGEMM_ERR_CUDA before anything is captured.
 bsgemm_status get_workspace(cudaStream_t stream, size_t ws_bytes, size_t n_counters, Workspace& out) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return BSGEMM_ERR_CUDA;
+  cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+  if (cudaStreamIsCapturing(stream, &cs) != cudaSuccess) return BSGEMM_ERR_CUDA;
+  const bool capturing = cs != cudaStreamCaptureStatusNone;
+  unsigned long long sid = 0;
+  if (!capturing && cudaStreamGetId(stream, &sid) != cudaSuccess) return BSGEMM_ERR_CUDA;
   std::lock_guard<std::mutex> lk(g_mu);
-  Workspace& w = g_ws[{dev, reinterpret_cast<uintptr_t>(stream)}];
+  const std::pair<int, uintptr_t> hkey{dev, reinterpret_cast<uintptr_t>(stream)};
+  if (capturing) {
+    auto id = g_ids.find(hkey);
+    if (id == g_ids.end()) return BSGEMM_ERR_CUDA;  // the stream has no workspace yet
+    sid = id->second;
+  } else {
+    g_ids[hkey] = sid;
+  }
+  Workspace& w = g_ws[{dev, sid}];
+  if (w.ws_bytes < ws_bytes || w.n_counters < n_counters) {
+    if (capturing) return BSGEMM_ERR_CUDA;
+  }
   if (w.ws_bytes < ws_bytes) {
-    if (w.ws) cudaFree(w.ws);
+    if (w.ws && cudaFreeAsync(w.ws, stream) != cudaSuccess) return BSGEMM_ERR_CUDA;
     w.ws = nullptr;
     w.ws_bytes = 0;
     size_t want = ws_bytes + ws_bytes / 4;
-    if (cudaMalloc(&w.ws, want) != cudaSuccess) return BSGEMM_ERR_CUDA;
+    void* p = nullptr;
+    if (cudaMallocAsync(&p, want, stream) != cudaSuccess) return BSGEMM_ERR_CUDA;
+    w.ws = static_cast<float*>(p);
     w.ws_bytes = want;
   }
   if (w.n_counters < n_counters) {
-    if (w.counters) cudaFree(w.counters);
+    if (w.counters && cudaFreeAsync(w.counters, stream) != cudaSuccess) return BSGEMM_ERR_CUDA;
     w.counters = nullptr;
     w.n_counters = 0;
     size_t want = n_counters < 1024 ? 1024 : n_counters * 2;
-    if (cudaMalloc(&w.counters, want * sizeof(int)) != cudaSuccess) return BSGEMM_ERR_CUDA;
+    void* p = nullptr;
+    if (cudaMallocAsync(&p, want * sizeof(int), stream) != cudaSuccess) return BSGEMM_ERR_CUDA;
+    w.counters = static_cast<int*>(p);
     if (cudaMemsetAsync(w.counters, 0, want * sizeof(int), stream) != cudaSuccess) return BSGEMM_ERR_CUDA;
     w.n_counters = want;
   }
@@ -454,9 +492,12 @@ extern "C" bsgemm_status bsgemm_get_last_device_status(bsgemm_stream_t stream) {
   if (v == 0) return BSGEMM_OK;
   const int zero = 0;
   if (cudaMemcpyToSymbol(g_device_status, &zero, sizeof zero) != cudaSuccess) return BSGEMM_ERR_CUDA;
-  // an aborted split-K launch may have left tile counters raised: clear them
+  // an aborted split-K launch may have left tile counters raised: clear them,
+  // once no stream of the device still runs (workspaces are stream-ordered
+  // allocations of their own streams)
   int cur = 0;
   cudaGetDevice(&cur);
+  if (cudaDeviceSynchronize() != cudaSuccess) return BSGEMM_ERR_CUDA;
   {
     std::lock_guard<std::mutex> lk(bsg_host::g_mu);
     for (auto& kv : bsg_host::g_ws)
@@ -465,6 +506,27 @@ extern "C" bsgemm_status bsgemm_get_last_device_status(bsgemm_stream_t stream) {
   }
   if (cudaDeviceSynchronize() != cudaSuccess) return BSGEMM_ERR_CUDA;
   return static_cast<bsgemm_status>(v & 0xFF);
+}
+
+extern "C" bsgemm_status bsgemm_release_workspaces(void) {
+  int cur = 0;
+  if (cudaGetDevice(&cur) != cudaSuccess) return BSGEMM_ERR_CUDA;
+  // no launch may still use the buffers
+  if (cudaDeviceSynchronize() != cudaSuccess) return BSGEMM_ERR_CUDA;
+  std::lock_guard<std::mutex> lk(bsg_host::g_mu);
+  bsgemm_status st = BSGEMM_OK;
+  for (auto it = bsg_host::g_ws.begin(); it != bsg_host::g_ws.end();) {
+    if (it->first.first != cur) {
+      ++it;
+      continue;
+    }
+    if (it->second.ws && cudaFree(it->second.ws) != cudaSuccess) st = BSGEMM_ERR_CUDA;
+    if (it->second.counters && cudaFree(it->second.counters) != cudaSuccess) st = BSGEMM_ERR_CUDA;
+    it = bsg_host::g_ws.erase(it);
+  }
+  for (auto it = bsg_host::g_ids.begin(); it != bsg_host::g_ids.end();)
+    it = it->first.first == cur ? bsg_host::g_ids.erase(it) : std::next(it);
+  return st;
 }
 
 extern "C" int bsgemm_last_device_status_detail(void) {

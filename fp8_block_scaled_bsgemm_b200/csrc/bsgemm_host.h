@@ -46,6 +46,11 @@ struct Workspace {
 bool make_map_2d(CUtensorMap* m, const void* base, CUtensorMapDataType dt, uint64_t inner,
                  uint64_t outer, uint64_t row_stride_bytes, uint32_t box_inner, uint32_t box_outer);
 
+// Tensor map of the [M, N] row-major output for the TMA-store epilogue: BF16
+// boxes of 32 rows x 64 columns, or FP32 boxes of 32 x 32 (128 bytes a row,
+// 128-byte swizzle).
+bool make_out_map(CUtensorMap* m, void* out, int M, int N, bool f32);
+
 // Split-K workspace of at least `ws_bytes` bytes and `n_counters` zeroed
 // counters for (current device, stream).
 bsgemm_status get_workspace(cudaStream_t stream, size_t ws_bytes, size_t n_counters, Workspace& out);

@@ -37,7 +37,7 @@ template <int BNQ, int GRAN, bool SWAP, bool P_MN, bool Q_MN, bool SPLIT, bool G
 bsgemm_status launch(const bsgemm_plan& plan, const void* a, const void* b, const float* sa,
                      const float* sb, void* out, int M, int N, int K, const CallOpts& opts,
                      cudaStream_t stream, const DeviceInfo& dev) {
-  using SC = bsg::StageCfg<BNQ, Q_MN, SWAP>;
+  using SC = bsg::StageCfg<BNQ, Q_MN, SWAP, GROUPED>;
   auto kern = bsg::bsgemm_kernel<BNQ, GRAN, SWAP, P_MN, Q_MN, SPLIT, GROUPED>;
 
   // P/Q operands: normally P = A (M rows), Q = B (N rows); swapped P = B, Q = A
@@ -52,6 +52,9 @@ bsgemm_status launch(const bsgemm_plan& plan, const void* a, const void* b, cons
   else      ok &= make_map_2d(&tm_p, p_ptr, CU_TENSOR_MAP_DATA_TYPE_UINT8, K, P, K, bsg::BK, bsg::BM);
   if (Q_MN) ok &= make_map_2d(&tm_q, q_ptr, CU_TENSOR_MAP_DATA_TYPE_UINT8, Q, K, Q, 128, bsg::BK);
   else      ok &= make_map_2d(&tm_q, q_ptr, CU_TENSOR_MAP_DATA_TYPE_UINT8, K, Q, K, bsg::BK, BNQ);
+  CUtensorMap tm_out;
+  std::memset(&tm_out, 0, sizeof tm_out);
+  if (SC::kTmaStore) ok &= make_out_map(&tm_out, out, M, N, (opts.epi & bsg::kEpiOutF32) != 0);
   if (!ok) return BSGEMM_ERR_CUDA;
 
   bsg::Params prm{};
@@ -105,7 +108,7 @@ bsgemm_status launch(const bsgemm_plan& plan, const void* a, const void* b, cons
     }
     setup.mark(dev.ordinal);
   }
-  kern<<<plan.grid, bsg::kNumThreads, SC::kSmemBytes, stream>>>(tm_p, tm_q, prm);
+  kern<<<plan.grid, bsg::kNumThreads, SC::kSmemBytes, stream>>>(tm_p, tm_q, tm_out, prm);
   return cudaGetLastError() == cudaSuccess ? BSGEMM_OK : BSGEMM_ERR_CUDA;
 }
 

@@ -21,7 +21,8 @@
 //   warps 4-11 promotion + epilogue: tcgen05.ld each K-block's partial,
 //            acc += (sP*sQ) * partial in FP32 registers (packed f32x2 FMAs),
 //            release the TMEM buffer, and at the end of a tile round to BF16
-//            and store it straight from registers.
+//            and store it: through shared memory and a TMA bulk tensor store
+//            for data-parallel tiles, straight from registers otherwise.
 // Work is split three ways:
 //   whole tiles (data-parallel), walked by the persistent CTAs in raster order;
 //   split-K: every tile's K-blocks cut into `splits` equal pieces;
@@ -109,10 +110,20 @@ struct Tiles {
   static constexpr int kQBytes = kQRows * BK;
 };
 
-template <int BNQ, bool Q_MN, bool SWAP>
+// Epilogue staging for the TMA store: each promotion warp owns one buffer of
+// 32 rows x 128 bytes (64 BF16 or 32 FP32 columns), in the 128-byte swizzled
+// layout of the output tensor map.
+constexpr int kEpiChunkBytes = 32 * 128;
+
+template <int BNQ, bool Q_MN, bool SWAP, bool GROUPED = false>
 struct StageCfg {
   static constexpr int kStageBytes = Tiles<BNQ, Q_MN>::kPBytes + Tiles<BNQ, Q_MN>::kQBytes;
-  static constexpr int kEpiBytes = 0;  // the epilogue stores straight from registers
+  // Data-parallel tiles store through TMA from a per-warp staging buffer.
+  // Swap-AB tiles (rows of the output are spread over the tile's columns)
+  // and grouped tiles (a tile may end inside the next group's rows) store
+  // straight from registers.
+  static constexpr bool kTmaStore = !SWAP && !GROUPED;
+  static constexpr int kEpiBytes = kTmaStore ? kNumEpiWarps * kEpiChunkBytes : 0;
   static constexpr int kBudget = 227 * 1024 - 1024 /*align slack*/ - 512 /*barriers*/;
   static constexpr int kStagesRaw = (kBudget - kEpiBytes) / kStageBytes;
   static constexpr int kStages = kStagesRaw > 8 ? 8 : kStagesRaw;
@@ -414,12 +425,10 @@ __device__ __forceinline__ float epi_act(float v, int act) {
   return v;
 }
 
-// One thread's run of columns [n0, n0 + 2 * NP) of row m: acc pairs in
-// column order. Applies the epilogue in place and stores BF16 (8 per 16-byte
-// store) or FP32 (4 per 16-byte store); N % 8 == 0, so a group of 8 columns
-// is wholly inside or outside the matrix.
+// out = act(acc + bias[n]) in place on one thread's run of columns
+// [n0, n0 + 2 * NP) (acc pairs in column order).
 template <int NP>
-__device__ __forceinline__ void store_row_run(const Params& p, int m, int n0, float2 (&acc)[NP]) {
+__device__ __forceinline__ void apply_epi(const Params& p, int n0, float2 (&acc)[NP]) {
   const int act = p.epi & 3;
   if (p.bias != nullptr || act != 0) {
 #pragma unroll
@@ -434,6 +443,82 @@ __device__ __forceinline__ void store_row_run(const Params& p, int m, int n0, fl
       acc[i].y = epi_act(acc[i].y + b1, act);
     }
   }
+}
+
+__device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t x, uint32_t y, uint32_t z, uint32_t w) {
+  asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(x), "r"(y), "r"(z), "r"(w)
+               : "memory");
+}
+
+// TMA-store epilogue of one promotion warp: lane l holds row m0 + l, columns
+// [n0, n0 + 2 * NP) (acc pairs in column order, epilogue already applied).
+// The warp's rows go out in chunks of 128 bytes per row (64 BF16 or 32 FP32
+// columns): every lane writes its row of the chunk into the warp's staging
+// buffer -- 16-byte piece u of row l at l * 128 + ((u ^ (l % 8)) * 16), the
+// tensor map's 128-byte swizzle, so a warp's store touches every bank evenly
+// -- then one lane issues the bulk tensor store.  The tensor map clips rows
+// past M and columns past N.  Before a buffer is rewritten, the store that
+// read it must have finished reading (cp.async.bulk.wait_group.read).
+template <int NP>
+__device__ __forceinline__ void store_tile_tma(const Params& p, const CUtensorMap* tm_out,
+                                               uint32_t buf, int m0, int n0, float2 (&acc)[NP],
+                                               uint32_t lane) {
+  const uint32_t row = buf + lane * 128;
+  const uint32_t sw = lane & 7;
+  if (m0 >= p.M) return;  // the warp's rows are all past the end
+  if (!(p.epi & kEpiOutF32)) {
+    static_assert((2 * NP) % 64 == 0, "BF16 chunks of 64 columns");
+#pragma unroll
+    for (int c = 0; c < 2 * NP / 64; ++c) {
+      if (n0 + c * 64 < p.N) {
+        if (lane == 0) bulk_wait_group_read0();
+        __syncwarp();
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          const int i = c * 32 + 4 * u;
+          st_shared_v4(row + ((u ^ sw) << 4), pack_bf16x2(acc[i].x, acc[i].y),
+                       pack_bf16x2(acc[i + 1].x, acc[i + 1].y), pack_bf16x2(acc[i + 2].x, acc[i + 2].y),
+                       pack_bf16x2(acc[i + 3].x, acc[i + 3].y));
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          tma_store_2d(tm_out, buf, n0 + c * 64, m0);
+          bulk_commit_group();
+        }
+      }
+    }
+  } else {
+    static_assert((2 * NP) % 32 == 0, "FP32 chunks of 32 columns");
+#pragma unroll
+    for (int c = 0; c < 2 * NP / 32; ++c) {
+      if (n0 + c * 32 < p.N) {
+        if (lane == 0) bulk_wait_group_read0();
+        __syncwarp();
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          const int i = c * 16 + 2 * u;
+          st_shared_v4(row + ((u ^ sw) << 4), __float_as_uint(acc[i].x), __float_as_uint(acc[i].y),
+                       __float_as_uint(acc[i + 1].x), __float_as_uint(acc[i + 1].y));
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          tma_store_2d(tm_out, buf, n0 + c * 32, m0);
+          bulk_commit_group();
+        }
+      }
+    }
+  }
+}
+
+// One thread's run of columns [n0, n0 + 2 * NP) of row m: acc pairs in
+// column order. Applies the epilogue in place and stores BF16 (8 per 16-byte
+// store) or FP32 (4 per 16-byte store); N % 8 == 0, so a group of 8 columns
+// is wholly inside or outside the matrix.
+template <int NP>
+__device__ __forceinline__ void store_row_run(const Params& p, int m, int n0, float2 (&acc)[NP]) {
+  apply_epi(p, n0, acc);
   if (p.epi & kEpiOutF32) {
     float* row = reinterpret_cast<float*>(p.out) + static_cast<size_t>(m) * p.N + n0;
 #pragma unroll
@@ -461,9 +546,9 @@ __device__ __forceinline__ void store_row_run(const Params& p, int m, int n0, fl
 template <int BNQ, int GRAN, bool SWAP, bool P_MN, bool Q_MN, bool SPLIT, bool GROUPED = false>
 __global__ void __launch_bounds__(kNumThreads, 1)
     bsgemm_kernel(const __grid_constant__ CUtensorMap tm_p, const __grid_constant__ CUtensorMap tm_q,
-                  const Params p) {
+                  const __grid_constant__ CUtensorMap tm_out, const Params p) {
   using TL = Tiles<BNQ, Q_MN>;
-  using SC = StageCfg<BNQ, Q_MN, SWAP>;
+  using SC = StageCfg<BNQ, Q_MN, SWAP, GROUPED>;
   constexpr int STAGES = SC::kStages;
   constexpr int kHalf = BNQ / 2;                      // columns per promotion warp
   constexpr int kNumGroups = (kHalf > GRAN) ? kHalf / GRAN : 1;  // scale groups per warp
@@ -484,7 +569,8 @@ __global__ void __launch_bounds__(kNumThreads, 1)
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* p_tiles = smem;
   uint8_t* q_tiles = smem + STAGES * TL::kPBytes;
-  Barriers* bars = reinterpret_cast<Barriers*>(q_tiles + STAGES * TL::kQBytes);
+  uint8_t* epi_bufs = q_tiles + STAGES * TL::kQBytes;  // 1024-aligned: stage sizes are multiples of 1 KB
+  Barriers* bars = reinterpret_cast<Barriers*>(epi_bufs + SC::kEpiBytes);
 
   const int warp = threadIdx.x / 32;
   const uint32_t lane = lane_id();
@@ -507,6 +593,7 @@ __global__ void __launch_bounds__(kNumThreads, 1)
   if (warp == kProducerWarp && lane == 0) {
     tma_prefetch_desc(&tm_p);
     tma_prefetch_desc(&tm_q);
+    if constexpr (SC::kTmaStore) tma_prefetch_desc(&tm_out);
   }
   if (warp == kMmaWarp) {
     tmem_alloc(smem_addr(&bars->tmem_base), kTmemCols);
@@ -769,11 +856,16 @@ __global__ void __launch_bounds__(kNumThreads, 1)
             __stcg(my_ws + (half * kHalf + 2 * i) * BM + row_in_tile, acc[i].x);
             __stcg(my_ws + (half * kHalf + 2 * i + 1) * BM + row_in_tile, acc[i].y);
           }
-          __threadfence();
-          // the partial now lives in the workspace; acc is dead until the sum below
+          // The partial now lives in the workspace; acc is dead until the sum
+          // below.  Publishing it takes one release: every promotion thread's
+          // stores come before the CTA barrier, the barrier before the
+          // leader's acq_rel add on the tile counter (GPU scope).  The last
+          // piece's leader acquires the other pieces' partials the same way,
+          // and its barrier hands them to the other threads, which read them
+          // from L2 (ld.global.cg).
           named_barrier_sync(1, kNumEpiThreads);
           if (ew == 0 && lane == 0) {
-            const int old = atomicAdd(p.counters + pcs.counter, 1);
+            const int old = atom_add_acq_rel_gpu(p.counters + pcs.counter, 1);
             bars->split_last = (old == pcs.pieces - 1) ? 1 : 0;
           }
           named_barrier_sync(1, kNumEpiThreads);
@@ -781,7 +873,6 @@ __global__ void __launch_bounds__(kNumThreads, 1)
           // nobody may overwrite split_last before every thread has read it
           named_barrier_sync(1, kNumEpiThreads);
           if (!last) continue;
-          __threadfence();
           // fixed order: the tile's pieces in K order, whoever arrived last
           const size_t col_off = static_cast<size_t>(half * kHalf) * BM + row_in_tile;
           {
@@ -821,6 +912,13 @@ __global__ void __launch_bounds__(kNumThreads, 1)
             }
           }
         }
+      } else if constexpr (SC::kTmaStore) {
+        // this thread owns row m0 + lane, columns [n0, n0 + kHalf); the warp
+        // stores its 32 rows through its staging buffer
+        const int n0 = w.tq * BNQ + half * kHalf;
+        apply_epi<kHalf / 2>(p, n0, acc);
+        store_tile_tma<kHalf / 2>(p, &tm_out, smem_addr(epi_bufs + ew * kEpiChunkBytes),
+                                  w.tp * BM + quad * 32, n0, acc, lane);
       } else {
         // this thread owns row m, columns [n0, n0 + kHalf)
         const int m_local = w.tp * BM + row_in_tile;
@@ -828,6 +926,11 @@ __global__ void __launch_bounds__(kNumThreads, 1)
         const int n0 = w.tq * BNQ + half * kHalf;
         if (m < p.M && (!GROUPED || m_local < w.g_rows)) store_row_run<kHalf / 2>(p, m, n0, acc);
       }
+    }
+    // every bulk store this warp issued has finished (reads of its staging
+    // buffer and writes to global memory) before the CTA exits
+    if constexpr (SC::kTmaStore) {
+      if (lane == 0) bulk_wait_group0();
     }
   }
   __syncwarp();

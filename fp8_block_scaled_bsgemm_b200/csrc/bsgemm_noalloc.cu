@@ -12,8 +12,10 @@
 // that is cut into pieces) is a fixed array in the library's own device
 // memory, declared below.
 // Every GPU that loads the library holds one copy of it until the process
-// exits.  Its size bounds what this entry point accepts: a problem whose plan
-// needs more scratch than the array holds is rejected with
+// exits.  Its size bounds the plans this entry point takes: where the regular
+// plan would need more scratch than the array holds, it takes the largest
+// split-K count whose partial tiles fit, down to no split at all, which needs
+// no scratch.  A launch whose plan still needed more would be refused with
 // BSGEMM_ERR_SCRATCH_LIMIT before anything is launched.
 //
 // All calls share the array, and it keeps whatever the last call left in it.
@@ -48,6 +50,7 @@ constexpr int kMaxDevices = 64;
 struct DeviceScratch {
   std::atomic<int> state{0};  // 0 not set up, 1 being set up, 2 ready
   unsigned char* base = nullptr;
+  int ordinal = 0;
   int num_sms = 0;
   int* status = nullptr;
 };
@@ -79,6 +82,7 @@ bsgemm_status setup_current_device(DeviceScratch*& out) {
         return BSGEMM_ERR_CUDA;
       }
       d.base = static_cast<unsigned char*>(p);
+      d.ordinal = dev;
       d.num_sms = sms;
       d.status = status;
       d.state.store(2, std::memory_order_release);
@@ -126,6 +130,9 @@ bsgemm_status launch_fixed(const bsgemm_plan& plan, const void* a, const void* b
   if (!bsg_host::make_map_2d(&tm_p, p_ptr, CU_TENSOR_MAP_DATA_TYPE_UINT8, K, P, K, bsg::BK, bsg::BM) ||
       !bsg_host::make_map_2d(&tm_q, q_ptr, CU_TENSOR_MAP_DATA_TYPE_UINT8, K, Q, K, bsg::BK, BNQ))
     return BSGEMM_ERR_CUDA;
+  CUtensorMap tm_out;
+  std::memset(&tm_out, 0, sizeof tm_out);
+  if (SC::kTmaStore && !bsg_host::make_out_map(&tm_out, out, M, N, false)) return BSGEMM_ERR_CUDA;
 
   bsg::Params prm{};
   prm.M = M; prm.N = N; prm.K = K;
@@ -160,14 +167,19 @@ bsgemm_status launch_fixed(const bsgemm_plan& plan, const void* a, const void* b
     if (cudaMemsetAsync(prm.counters, 0, counters * sizeof(int), stream) != cudaSuccess)
       return BSGEMM_ERR_CUDA;
   }
-  if (bsg::RegSplit<BNQ>::kEnabled) {
-    cudaFuncAttributes fa{};
-    if (cudaFuncGetAttributes(&fa, kern) != cudaSuccess || fa.numRegs != bsg::kLaunchRegs)
+  static bsg_host::PerDeviceOnce setup;  // once per instance and device
+  if (!setup.done(d.ordinal)) {
+    // the setmaxnreg split is only safe with exactly the planned launch registers
+    if (bsg::RegSplit<BNQ>::kEnabled) {
+      cudaFuncAttributes fa{};
+      if (cudaFuncGetAttributes(&fa, kern) != cudaSuccess || fa.numRegs != bsg::kLaunchRegs)
+        return BSGEMM_ERR_CUDA;
+    }
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SC::kSmemBytes) != cudaSuccess)
       return BSGEMM_ERR_CUDA;
+    setup.mark(d.ordinal);
   }
-  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SC::kSmemBytes) != cudaSuccess)
-    return BSGEMM_ERR_CUDA;
-  kern<<<plan.grid, bsg::kNumThreads, SC::kSmemBytes, stream>>>(tm_p, tm_q, prm);
+  kern<<<plan.grid, bsg::kNumThreads, SC::kSmemBytes, stream>>>(tm_p, tm_q, tm_out, prm);
   return cudaGetLastError() == cudaSuccess ? BSGEMM_OK : BSGEMM_ERR_CUDA;
 }
 
@@ -209,7 +221,10 @@ extern "C" bsgemm_status bsgemm_fp8_nt_noalloc(const void* a, const void* b, con
   DeviceScratch* d = nullptr;
   bsgemm_status st = setup_current_device(d);
   if (st != BSGEMM_OK) return st;
-  // the regular plan when its scratch fits; otherwise the plan without stream-K.
+  // The regular plan when its scratch fits.  Otherwise the same variant and
+  // tile width without stream-K, with the heuristic's split count lowered
+  // until its partial tiles fit the array; one split needs no scratch, so
+  // every problem the regular entry point runs, this one runs too.
   // This entry point launches single-CTA tiles only: where the regular plan
   // takes CTA pairs (large g = 256 problems), it takes 128-row data-parallel
   // tiles instead.
@@ -222,9 +237,15 @@ extern "C" bsgemm_status bsgemm_fp8_nt_noalloc(const void* a, const void* b, con
     if (st != BSGEMM_OK) return st;
   }
   if (!fits(pl)) {
-    const bsgemm_tuning no_sk = {0, 0, 0, -1};
+    const int variant = pl.swap_ab ? BSGEMM_VARIANT_SWAP_AB : BSGEMM_VARIANT_DATA_PARALLEL;
+    const bsgemm_tuning no_sk = {variant, pl.bnq, 0, -1};
     st = bsgemm_make_plan(BSGEMM_LAYOUT_NT, M, N, K, gran, d->num_sms, &no_sk, &pl);
     if (st != BSGEMM_OK) return st;
+    for (int s = pl.splits - 1; !fits(pl) && s >= 1; --s) {
+      const bsgemm_tuning capped = {variant, pl.bnq, s, -1};
+      st = bsgemm_make_plan(BSGEMM_LAYOUT_NT, M, N, K, gran, d->num_sms, &capped, &pl);
+      if (st != BSGEMM_OK) return st;
+    }
     if (!fits(pl)) return BSGEMM_ERR_SCRATCH_LIMIT;
   }
   cudaStream_t s = static_cast<cudaStream_t>(stream);

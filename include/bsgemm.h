@@ -39,8 +39,18 @@
  * Ownership: all pointers belong to the caller, who keeps them alive until
  * the stream has passed the call.  The library keeps no pointer beyond the
  * call.  It owns an internal split-K workspace per (device, stream), grown on
- * demand with cudaMalloc and never shrunk; two calls that run concurrently on
- * different streams never share it.
+ * demand and never shrunk; two calls that run concurrently on different
+ * streams never share it.  Growth is stream-ordered on the call's stream
+ * (cudaFreeAsync of the old buffer, cudaMallocAsync of the new one), so a
+ * growing call neither synchronises the device nor waits for other streams.
+ * Workspaces are keyed by the stream's process-unique id (cudaStreamGetId),
+ * so a stream created after another was destroyed never inherits its
+ * workspace, even with the same handle value; the destroyed stream's
+ * workspace stays allocated until bsgemm_release_workspaces() or process
+ * exit.  A call captured into a CUDA graph can only use the workspace that
+ * earlier uncaptured calls on the same stream made big enough; otherwise it
+ * fails with BSGEMM_ERR_CUDA before anything is captured, and the capture
+ * stays valid: run the same call once on that stream before capturing it.
  *
  * Alignment (TMA rules), checked on the host before any launch:
  *   a, b, out 16-byte aligned; scale_a, scale_b 4-byte aligned;
@@ -279,6 +289,12 @@ const char *bsgemm_status_string(bsgemm_status status);
  * synchronisation itself failed. */
 bsgemm_status bsgemm_get_last_device_status(bsgemm_stream_t stream);
 
+/* Frees every split-K workspace the library holds on the current device
+ * (those of destroyed streams included), after waiting for the device to
+ * finish its work.  Later calls allocate again as needed.  Returns
+ * BSGEMM_ERR_CUDA if the device wait or a free fails. */
+bsgemm_status bsgemm_release_workspaces(void);
+
 /* Raw device status word (0, or the timeout code in the low byte and the
  * place of the wait that gave up in bits 8..15), without clearing it. */
 int bsgemm_last_device_status_detail(void);
@@ -296,23 +312,26 @@ bsgemm_status bsgemm_diag_wait_timeout(unsigned long long timeout_ns, bsgemm_str
  * under a framework that owns every byte of device memory and hands the
  * library only the tensors of the call, or in a process that must not grow
  * its device footprint after start-up.  The entry points above create their
- * split-K workspace with cudaMalloc on first use; this one never allocates
+ * split-K workspace with cudaMallocAsync on first use; this one never allocates
  * (no cudaMalloc, cudaFree or allocating library call, torch's included).
  *
  * It computes exactly what bsgemm_fp8_nt computes, with the same arguments,
  * rules and errors, and with the same single-CTA kernels.  It takes the same
- * plan when that plan's scratch fits the array, otherwise the plan without
- * stream-K; where the regular plan pairs CTAs (large g = 256 problems) it
- * takes 128-row data-parallel tiles instead.
+ * plan when that plan's scratch fits the array; otherwise it keeps the plan's
+ * variant and tile width, drops stream-K and lowers the split-K count until
+ * the partial tiles fit (one split needs no scratch, so every problem
+ * bsgemm_fp8_nt accepts runs here too, possibly with fewer K splits).  Where
+ * the regular plan pairs CTAs (large g = 256 problems) it takes 128-row
+ * data-parallel tiles instead.
  * Its split-K / stream-K scratch is a fixed array inside the library's device
- * memory: each GPU that loads
- * the library holds BSGEMM_NOALLOC_SCRATCH_BYTES of FP32 partial tiles plus
- * BSGEMM_NOALLOC_MAX_TILES tile counters until the process exits.  A problem
- * whose plan needs more -- split-K: tiles x splits partial tiles; stream-K:
- * 2 x sk_ctas partial tiles; a partial tile is tile width x 128 x 4 bytes --
- * or more tile counters than it holds, even without stream-K, is rejected with
- * BSGEMM_ERR_SCRATCH_LIMIT before anything is launched.  Problems whose plan
- * neither splits K nor uses stream-K need no scratch at all.
+ * memory: each GPU that loads the library holds BSGEMM_NOALLOC_SCRATCH_BYTES
+ * of FP32 partial tiles plus BSGEMM_NOALLOC_MAX_TILES tile counters until the
+ * process exits.  A plan needs split-K: tiles x splits partial tiles and one
+ * counter per tile; stream-K: 2 x sk_ctas partial tiles and one counter per
+ * stream-K tile; a partial tile is tile width x 128 x 4 bytes.  A launch
+ * whose plan needed more than the array holds would be refused with
+ * BSGEMM_ERR_SCRATCH_LIMIT before anything is launched; the plan choice
+ * above keeps every plan within it.
  *
  * The first call on each device looks up the array's device address (once,
  * with that device current); make that first call before any stream capture.

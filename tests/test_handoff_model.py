@@ -33,11 +33,12 @@ import pytest
 
 BK = 128                       # K bytes per stage
 BUDGET = 227 * 1024 - 1024 - 512
+EPI_STAGING = 8 * 32 * 128     # per-warp TMA-store staging of the data-parallel tiles
 
 
-def stages(bnq: int, q_mn: bool) -> int:
+def stages(bnq: int, q_mn: bool, tma_store: bool = False) -> int:
     q_rows = 128 if (q_mn and bnq < 128) else bnq
-    return min(8, BUDGET // (BM_BYTES + q_rows * BK))
+    return min(8, (BUDGET - (EPI_STAGING if tma_store else 0)) // (BM_BYTES + q_rows * BK))
 
 
 BM_BYTES = 128 * BK
@@ -224,19 +225,31 @@ def simulate(S, B, gran, K, items, rng, mutation=None):
     return errors
 
 
-CONFIGS = [(bnq, q_mn) for bnq in (16, 32, 64, 128, 256) for q_mn in (False, True)]
+# (tile width, MN-major Q, TMA-store staging): swap-AB tiles (16..128 wide) keep
+# every stage, data-parallel tiles (128, 256) give 32 KB to the epilogue staging
+CONFIGS = ([(bnq, q_mn, False) for bnq in (16, 32, 64, 128) for q_mn in (False, True)] +
+           [(bnq, q_mn, True) for bnq in (128, 256) for q_mn in (False, True)])
 
 
 @pytest.mark.parametrize("gran", [64, 128, 256])
-@pytest.mark.parametrize("bnq,q_mn", CONFIGS)
-def test_handoff_never_aliases_or_deadlocks(bnq, q_mn, gran):
-    S, B = stages(bnq, q_mn), bufs(bnq)
-    rng = random.Random(1000 * bnq + 10 * gran + q_mn)
+@pytest.mark.parametrize("bnq,q_mn,tma_store", CONFIGS)
+def test_handoff_never_aliases_or_deadlocks(bnq, q_mn, tma_store, gran):
+    S, B = stages(bnq, q_mn, tma_store), bufs(bnq)
+    rng = random.Random(1000 * bnq + 10 * gran + q_mn + 5 * tma_store)
     for _ in range(60):
         K = rng.choice([BK, 2 * BK, 3 * BK, 5 * BK + 16, 7 * BK, 9 * BK + 64, 17 * BK])
         items = work_list(rng, gran, K)
         errors = simulate(S, B, gran, K, items, rng)
         assert not errors, (S, B, gran, K, items, errors[0])
+
+
+def test_stage_counts_match_the_kernel_budget():
+    """The 256-wide data-parallel tile keeps 4 stages beside its 32 KB of
+    epilogue staging; the 128-wide one 6; swap-AB 128 keeps 7; the narrow swap
+    tiles 8."""
+    assert stages(256, False, True) == 4 and stages(256, True, True) == 4
+    assert stages(128, False, True) == 6
+    assert stages(128, False, False) == 7 and stages(16, False, False) == 8
 
 
 MUTATIONS = [
@@ -254,7 +267,7 @@ def test_model_catches_planted_protocol_mistakes(mutation):
     wrong phase, or a stage or buffer used out of turn."""
     rng = random.Random(hash(mutation) & 0xFFFF)
     for bnq, q_mn, gran in ((256, False, 128), (128, True, 64), (64, False, 256)):
-        S, B = stages(bnq, q_mn), bufs(bnq)
+        S, B = stages(bnq, q_mn, bnq >= 128), bufs(bnq)
         caught = False
         for _ in range(300):
             K = rng.choice([5 * BK, 9 * BK, 17 * BK])
