@@ -44,25 +44,36 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
 
 }  // namespace
 
-// 2D tensor map with 128-byte swizzle. `inner` is the contiguous extent.
-bool make_map_2d(CUtensorMap* m, const void* base, CUtensorMapDataType dt, uint64_t inner,
-                 uint64_t outer, uint64_t row_stride_bytes, uint32_t box_inner, uint32_t box_outer) {
+namespace {
+bool encode_2d(CUtensorMap* m, const void* base, CUtensorMapDataType dt, uint64_t inner, uint64_t outer,
+               uint64_t row_stride_bytes, uint32_t box_inner, uint32_t box_outer, CUtensorMapSwizzle swz) {
   auto fn = encode_fn();
   if (!fn) return false;
   cuuint64_t dims[2] = {inner, outer};
   cuuint64_t strides[1] = {row_stride_bytes};
   cuuint32_t box[2] = {box_inner, box_outer};
   cuuint32_t estr[2] = {1, 1};
-  CUresult r = fn(m, dt, 2, const_cast<void*>(base), dims, strides, box, estr,
-                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  CUresult r = fn(m, dt, 2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                  swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
+}
+}  // namespace
+
+// 2D tensor map with 128-byte swizzle. `inner` is the contiguous extent.
+bool make_map_2d(CUtensorMap* m, const void* base, CUtensorMapDataType dt, uint64_t inner,
+                 uint64_t outer, uint64_t row_stride_bytes, uint32_t box_inner, uint32_t box_outer) {
+  return encode_2d(m, base, dt, inner, outer, row_stride_bytes, box_inner, box_outer, CU_TENSOR_MAP_SWIZZLE_128B);
 }
 
 bool make_out_map(CUtensorMap* m, void* out, int M, int N, bool f32) {
   if (f32)
     return make_map_2d(m, out, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, N, M, static_cast<uint64_t>(N) * 4, 32, 32);
   return make_map_2d(m, out, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, N, M, static_cast<uint64_t>(N) * 2, 64, 32);
+}
+
+bool make_swap_out_map(CUtensorMap* m, void* out, int M, int N, int bnq) {
+  return encode_2d(m, out, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, N, M, static_cast<uint64_t>(N) * 2, bsg::BM,
+                   static_cast<uint32_t>(bnq), CU_TENSOR_MAP_SWIZZLE_NONE);
 }
 
 // ------------------------------------------------------------------ per-device state
@@ -287,13 +298,13 @@ extern "C" bsgemm_status bsgemm_make_plan(int layout, int64_t M, int64_t N, int6
     // waves stay whole tiles and the remaining tiles' units are shared out
     // evenly. Compared on the busiest CTA's units, with a partial tile written
     // and re-read counted as (1 + width/128) units.  Measured on B200, the
-    // ranges only pay off when a tile has many units (K >= 64 K-blocks of
-    // 128) or, with fewer tiles than SMs, when the tiles are at least 64
-    // wide; below that whole tiles (or split-K) win, so the heuristic keeps
-    // to those cases.  stream_k = 1 forces it wherever a wave is ragged.
+    // ranges pay off with fewer tiles than SMs (the decode shapes: 5-11 %
+    // over split-K at every tile width) and, with more, only when a tile has
+    // many units (K >= 64 K-blocks of 128); on short-K problems whole tiles
+    // win.  stream_k = 1 forces it wherever a wave is ragged.
     const int64_t full = (tiles / num_sms) * num_sms;
     const int64_t rem = tiles - full;
-    const bool sk_pays = tiles < num_sms ? bnq >= 64 : U * unit_kb * gran >= 64 * 128;
+    const bool sk_pays = tiles < num_sms ? true : U * unit_kb * gran >= 64 * 128;
     bool use_sk = false;
     if (rem > 0 && sk_req >= 0 && (sk_req > 0 || sk_pays)) {
       const int64_t R = rem * U;

@@ -51,6 +51,10 @@ bool make_map_2d(CUtensorMap* m, const void* base, CUtensorMapDataType dt, uint6
 // 128-byte swizzle).
 bool make_out_map(CUtensorMap* m, void* out, int M, int N, bool f32);
 
+// Tensor map of the BF16 [M, N] output for swap-AB tiles: boxes of BNQ rows
+// (m) x 128 columns (n), no swizzle (the staging tile is [BNQ][128] BF16).
+bool make_swap_out_map(CUtensorMap* m, void* out, int M, int N, int bnq);
+
 // Split-K workspace of at least `ws_bytes` bytes and `n_counters` zeroed
 // counters for (current device, stream).
 bsgemm_status get_workspace(cudaStream_t stream, size_t ws_bytes, size_t n_counters, Workspace& out);

@@ -55,6 +55,7 @@ bsgemm_status launch(const bsgemm_plan& plan, const void* a, const void* b, cons
   CUtensorMap tm_out;
   std::memset(&tm_out, 0, sizeof tm_out);
   if (SC::kTmaStore) ok &= make_out_map(&tm_out, out, M, N, (opts.epi & bsg::kEpiOutF32) != 0);
+  if (SC::kSwapTmaStore && !(opts.epi & bsg::kEpiOutF32)) ok &= make_swap_out_map(&tm_out, out, M, N, BNQ);
   if (!ok) return BSGEMM_ERR_CUDA;
 
   bsg::Params prm{};
@@ -108,7 +109,20 @@ bsgemm_status launch(const bsgemm_plan& plan, const void* a, const void* b, cons
     }
     setup.mark(dev.ordinal);
   }
-  kern<<<plan.grid, bsg::kNumThreads, SC::kSmemBytes, stream>>>(tm_p, tm_q, tm_out, prm);
+  // programmatic dependent launch: the kernel's set-up may overlap the tail
+  // of the previous grid on the stream; it waits for that grid before any
+  // global memory access (grid_dependency_wait)
+  cudaLaunchConfig_t cfg{};
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.gridDim = dim3(plan.grid, 1, 1);
+  cfg.blockDim = dim3(bsg::kNumThreads, 1, 1);
+  cfg.dynamicSmemBytes = SC::kSmemBytes;
+  cfg.stream = stream;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, kern, tm_p, tm_q, tm_out, prm) != cudaSuccess) return BSGEMM_ERR_CUDA;
   return cudaGetLastError() == cudaSuccess ? BSGEMM_OK : BSGEMM_ERR_CUDA;
 }
 
@@ -148,16 +162,18 @@ bsgemm_status launch_pair(const bsgemm_plan& plan, const void* a, const void* b,
   prm.timeout_ns = wait_timeout_ns();
 
   cudaLaunchConfig_t cfg{};
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = 2;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;  // see launch()
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.blockDim = dim3(bsg::kNumThreads, 1, 1);
   cfg.dynamicSmemBytes = PC::kSmemBytes;
   cfg.stream = stream;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = 2;
 
   // co-resident CTA pairs, found once per instance and device
   static PerDeviceOnce setup;
@@ -172,8 +188,10 @@ bsgemm_status launch_pair(const bsgemm_plan& plan, const void* a, const void* b,
     if (cudaFuncGetAttributes(&fa, kern) != cudaSuccess || fa.numRegs != bsg::kLaunchRegs)
       return BSGEMM_ERR_CUDA;
     cfg.gridDim = dim3(plan.grid, 1, 1);
+    cfg.numAttrs = 1;  // the cluster shape alone decides residency
     int n = 0;
     if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) != cudaSuccess || n < 1) return BSGEMM_ERR_CUDA;
+    cfg.numAttrs = 2;
     max_pairs = n;
     if (slot >= 0) {
       resident_pairs[slot].store(n, std::memory_order_relaxed);

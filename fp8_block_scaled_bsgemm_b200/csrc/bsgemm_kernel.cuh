@@ -96,7 +96,7 @@ struct Params {
   const float* sP;       // [Pb][Kb]
   const float* sQ;       // [Qb][Kb]
   __nv_bfloat16* out;    // [M][N] row-major, BF16 (FP32 when epi bit 2 is set)
-  float* ws;             // partial tiles [slot][BNQ][BM]: split-K slot tile*splits+split,
+  float* ws;             // partial tiles [slot][BNQ/4][BM][4]: split-K slot tile*splits+split,
                          // stream-K slot 2*cta + (0: the CTA's first tile, 1: its last)
   int* counters;         // one per split or stream-K tile, zero between launches
   int* status;           // device status word
@@ -119,11 +119,13 @@ template <int BNQ, bool Q_MN, bool SWAP, bool GROUPED = false>
 struct StageCfg {
   static constexpr int kStageBytes = Tiles<BNQ, Q_MN>::kPBytes + Tiles<BNQ, Q_MN>::kQBytes;
   // Data-parallel tiles store through TMA from a per-warp staging buffer.
-  // Swap-AB tiles (rows of the output are spread over the tile's columns)
-  // and grouped tiles (a tile may end inside the next group's rows) store
-  // straight from registers.
+  // Swap-AB tiles stage the whole BF16 tile, transposed to the output's
+  // [M][N] order ([BNQ][128] BF16), and store it with one TMA copy (their FP32
+  // output stores from registers).  Grouped tiles (a tile may end inside the
+  // next group's rows) store straight from registers.
   static constexpr bool kTmaStore = !SWAP && !GROUPED;
-  static constexpr int kEpiBytes = kTmaStore ? kNumEpiWarps * kEpiChunkBytes : 0;
+  static constexpr bool kSwapTmaStore = SWAP;
+  static constexpr int kEpiBytes = kTmaStore ? kNumEpiWarps * kEpiChunkBytes : (SWAP ? BNQ * BM * 2 : 0);
   static constexpr int kBudget = 227 * 1024 - 1024 /*align slack*/ - 512 /*barriers*/;
   static constexpr int kStagesRaw = (kBudget - kEpiBytes) / kStageBytes;
   static constexpr int kStages = kStagesRaw > 8 ? 8 : kStagesRaw;
@@ -170,6 +172,28 @@ __device__ __forceinline__ bool bounded_wait(uint32_t bar, uint32_t parity, cons
     if (!ignore_abort && *reinterpret_cast<volatile int*>(&bars->abort_flag)) return false;
     if (globaltimer_ns() - t0 > p.timeout_ns) {
       if (!ignore_abort) record_timeout(p, bars, where);
+      return false;
+    }
+  }
+}
+
+// Bounded wait of one thread until the counter at `ctr` reaches `target`,
+// with acquire semantics at GPU scope (the publishers' stores before their
+// release adds are visible afterwards).  Returns false on timeout (recorded)
+// or when another warp of the CTA raised the abort flag.
+__device__ __forceinline__ bool wait_counter_acquire(const Params& p, Barriers* bars, const int* ctr,
+                                                     int target, int where) {
+  if (ld_acquire_gpu(ctr) >= target) return true;
+  const uint64_t t0 = globaltimer_ns();
+  while (true) {
+#pragma unroll 1
+    for (int i = 0; i < 32; ++i) {
+      __nanosleep(64);
+      if (ld_acquire_gpu(ctr) >= target) return true;
+    }
+    if (*reinterpret_cast<volatile int*>(&bars->abort_flag)) return false;
+    if (globaltimer_ns() - t0 > p.timeout_ns) {
+      record_timeout(p, bars, where);
       return false;
     }
   }
@@ -445,6 +469,10 @@ __device__ __forceinline__ void apply_epi(const Params& p, int n0, float2 (&acc)
   }
 }
 
+__device__ __forceinline__ void st_shared_b16(uint32_t addr, unsigned short v) {
+  asm volatile("st.shared.b16 [%0], %1;" ::"r"(addr), "h"(v) : "memory");
+}
+
 __device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t x, uint32_t y, uint32_t z, uint32_t w) {
   asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(x), "r"(y), "r"(z), "r"(w)
                : "memory");
@@ -593,7 +621,11 @@ __global__ void __launch_bounds__(kNumThreads, 1)
   if (warp == kProducerWarp && lane == 0) {
     tma_prefetch_desc(&tm_p);
     tma_prefetch_desc(&tm_q);
+    // the output map exists for data-parallel tiles and for BF16 swap-AB tiles
     if constexpr (SC::kTmaStore) tma_prefetch_desc(&tm_out);
+    if constexpr (SC::kSwapTmaStore) {
+      if (!(p.epi & kEpiOutF32)) tma_prefetch_desc(&tm_out);
+    }
   }
   if (warp == kMmaWarp) {
     tmem_alloc(smem_addr(&bars->tmem_base), kTmemCols);
@@ -603,6 +635,14 @@ __global__ void __launch_bounds__(kNumThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = bars->tmem_base;
+  // Programmatic dependent launch: everything above (barriers, TMEM, the
+  // tensor-map prefetch) and the producer's first work item touch no global
+  // memory, so they may overlap the previous grid's last CTAs.  The producer
+  // and the promotion warps -- the only roles that read or write global
+  // memory (operands, scales, workspace, output) -- wait for that grid
+  // (grid_dependency_wait) first; the MMA warp touches only shared memory and
+  // TMEM.  The next grid may start its own set-up as soon as SMs free up.
+  if (threadIdx.x == 0) grid_launch_dependents();
 
   if (warp < kFirstEpiWarp) {
     // warpgroup 0: producer, MMA issuer and two idle warps
@@ -613,8 +653,13 @@ __global__ void __launch_bounds__(kNumThreads, 1)
       uint32_t it = 0;  // stage-slot uses so far
       bool ok = true;
       WorkIter wit;
+      // the grouped work list reads the group sizes from global memory
+      if constexpr (GROUPED) grid_dependency_wait();
       work_begin<SPLIT, GROUPED>(p, wit);
-      for (Work w; ok && work_next<GRAN, SPLIT, GROUPED>(p, wit, w);) {
+      Work w;
+      bool more = work_next<GRAN, SPLIT, GROUPED>(p, wit, w);
+      if constexpr (!GROUPED) grid_dependency_wait();
+      for (; ok && more; more = work_next<GRAN, SPLIT, GROUPED>(p, wit, w)) {
         int st0, st1;
         stage_range<GRAN>(p, w, st0, st1);
         for (int st = st0; st < st1; ++st, ++it) {
@@ -670,6 +715,8 @@ __global__ void __launch_bounds__(kNumThreads, 1)
       uint32_t b = 0, bph = 0;    // TMEM buffer and its phase
       bool ok = true;
       WorkIter wit;
+      // the grouped work list reads the group sizes from global memory
+      if constexpr (GROUPED) grid_dependency_wait();
       work_begin<SPLIT, GROUPED>(p, wit);
       for (Work w; ok && work_next<GRAN, SPLIT, GROUPED>(p, wit, w);) {
         for (int kb = w.kb0; kb < w.kb1; ++kb) {
@@ -736,6 +783,7 @@ __global__ void __launch_bounds__(kNumThreads, 1)
   } else {
     // ============================================================ promotion + epilogue
     if constexpr (RegSplit<BNQ>::kEnabled) set_max_regs_inc<kPromoteRegs>();
+    grid_dependency_wait();
     const int ew = warp - kFirstEpiWarp;   // 0..7
     const int quad = warp & 3;             // TMEM lane quadrant this warp may access
     const int half = ew >> 2;              // which half of the BNQ columns
@@ -849,46 +897,80 @@ __global__ void __launch_bounds__(kNumThreads, 1)
           pcs.slot0 = d[3]; pcs.slot_base = d[4]; pcs.slot_step = d[5];
         }
         if (pcs.pieces > 1) {
-          // partial tile, column-major [BNQ][BM]: a warp writes 128 contiguous bytes per column
-          float* my_ws = p.ws + static_cast<size_t>(pcs.slot) * (BNQ * BM);
+          // Stream-K: the piece that starts the tile (kb0 == 0) is the last
+          // segment of its CTA's range, so it ends after the tile's other
+          // pieces, which each start a CTA's range.  It keeps its partial in
+          // registers, waits for the others and adds them in K order.
+          // Split-K pieces all end at about the same time; there the last to
+          // arrive adds all of them.  Either way the sum is piece 0 + piece 1
+          // + ... in FP32, in that order, every run.
+          const bool reducer = p.sk_ctas > 0 && w.tile >= p.sk_first_tile && w.kb0 == 0;
+          const size_t chunk_off = static_cast<size_t>(half * kHalf / 4) * BM + row_in_tile;
+          if (!reducer) {
+            // partial tile as 16-byte chunks [BNQ / 4][BM][4]: each thread writes
+            // its row's kHalf / 4 chunks, and a warp (32 consecutive rows) writes
+            // 512 contiguous bytes per chunk
+            float4* my_ws = reinterpret_cast<float4*>(p.ws + static_cast<size_t>(pcs.slot) * (BNQ * BM)) +
+                            (half * kHalf / 4) * BM + row_in_tile;
 #pragma unroll
-          for (int i = 0; i < kHalf / 2; ++i) {
-            __stcg(my_ws + (half * kHalf + 2 * i) * BM + row_in_tile, acc[i].x);
-            __stcg(my_ws + (half * kHalf + 2 * i + 1) * BM + row_in_tile, acc[i].y);
-          }
-          // The partial now lives in the workspace; acc is dead until the sum
-          // below.  Publishing it takes one release: every promotion thread's
-          // stores come before the CTA barrier, the barrier before the
-          // leader's acq_rel add on the tile counter (GPU scope).  The last
-          // piece's leader acquires the other pieces' partials the same way,
-          // and its barrier hands them to the other threads, which read them
-          // from L2 (ld.global.cg).
-          named_barrier_sync(1, kNumEpiThreads);
-          if (ew == 0 && lane == 0) {
-            const int old = atom_add_acq_rel_gpu(p.counters + pcs.counter, 1);
-            bars->split_last = (old == pcs.pieces - 1) ? 1 : 0;
-          }
-          named_barrier_sync(1, kNumEpiThreads);
-          const bool last = *reinterpret_cast<volatile int*>(&bars->split_last) != 0;
-          // nobody may overwrite split_last before every thread has read it
-          named_barrier_sync(1, kNumEpiThreads);
-          if (!last) continue;
-          // fixed order: the tile's pieces in K order, whoever arrived last
-          const size_t col_off = static_cast<size_t>(half * kHalf) * BM + row_in_tile;
-          {
-            const float* src = p.ws + static_cast<size_t>(piece_slot(pcs, 0)) * (BNQ * BM) + col_off;
-#pragma unroll
-            for (int i = 0; i < kHalf / 2; ++i) {
-              acc[i].x = __ldcg(src + (2 * i) * BM);
-              acc[i].y = __ldcg(src + (2 * i + 1) * BM);
+            for (int c = 0; c < kHalf / 4; ++c)
+              __stcg(my_ws + c * BM, make_float4(acc[2 * c].x, acc[2 * c].y, acc[2 * c + 1].x, acc[2 * c + 1].y));
+            // The partial now lives in the workspace; acc is dead until the
+            // sum below.  Publishing it takes one release: every promotion
+            // thread's stores come before the CTA barrier, the barrier before
+            // the leader's release add on the tile counter (GPU scope).  A
+            // split-K leader's add also acquires the earlier pieces (acq_rel)
+            // and tells whether this piece arrived last.
+            named_barrier_sync(1, kNumEpiThreads);
+            if (ew == 0 && lane == 0) {
+              int is_last = 0;
+              if (p.sk_ctas > 0 && w.tile >= p.sk_first_tile) {
+                red_add_release_gpu(p.counters + pcs.counter, 1);
+              } else {
+                is_last = atom_add_acq_rel_gpu(p.counters + pcs.counter, 1) == pcs.pieces - 1;
+              }
+              bars->split_last = is_last;
             }
-          }
-          for (int j = 1; j < pcs.pieces; ++j) {
-            const float* src = p.ws + static_cast<size_t>(piece_slot(pcs, j)) * (BNQ * BM) + col_off;
+            named_barrier_sync(1, kNumEpiThreads);
+            const bool last = *reinterpret_cast<volatile int*>(&bars->split_last) != 0;
+            // nobody may overwrite split_last before every thread has read it
+            named_barrier_sync(1, kNumEpiThreads);
+            if (!last) continue;
+            // split-K, last to arrive: piece 0 from the workspace first
+            const float4* src =
+                reinterpret_cast<const float4*>(p.ws + static_cast<size_t>(piece_slot(pcs, 0)) * (BNQ * BM)) + chunk_off;
 #pragma unroll
-            for (int i = 0; i < kHalf / 2; ++i) {
-              acc[i].x += __ldcg(src + (2 * i) * BM);
-              acc[i].y += __ldcg(src + (2 * i + 1) * BM);
+            for (int c = 0; c < kHalf / 4; ++c) {
+              const float4 v = __ldcg(src + c * BM);
+              acc[2 * c] = make_float2(v.x, v.y);
+              acc[2 * c + 1] = make_float2(v.z, v.w);
+            }
+          } else {
+            // stream-K reducer: the leader waits (bounded) until the other
+            // pieces - 1 pieces have published (acquire), and the barrier
+            // hands them to the other threads
+            if (ew == 0 && lane == 0)
+              bars->split_last = wait_counter_acquire(p, bars, p.counters + pcs.counter, pcs.pieces - 1, 5) ? 1 : 0;
+            named_barrier_sync(1, kNumEpiThreads);
+            const bool got = *reinterpret_cast<volatile int*>(&bars->split_last) != 0;
+            named_barrier_sync(1, kNumEpiThreads);
+            if (!got) { ok = false; break; }
+          }
+          // piece 0 is in acc; the others follow in K order.  A piece's
+          // kHalf / 4 chunk loads are independent, so they are all in flight
+          // together
+          for (int j = 1; j < pcs.pieces; ++j) {
+            const float4* src =
+                reinterpret_cast<const float4*>(p.ws + static_cast<size_t>(piece_slot(pcs, j)) * (BNQ * BM)) + chunk_off;
+            float4 v[kHalf / 4];
+#pragma unroll
+            for (int c = 0; c < kHalf / 4; ++c) v[c] = __ldcg(src + c * BM);
+#pragma unroll
+            for (int c = 0; c < kHalf / 4; ++c) {
+              acc[2 * c].x += v[c].x;
+              acc[2 * c].y += v[c].y;
+              acc[2 * c + 1].x += v[c].z;
+              acc[2 * c + 1].y += v[c].w;
             }
           }
           if (ew == 0 && lane == 0) p.counters[pcs.counter] = 0;  // ready for the next launch
@@ -899,7 +981,29 @@ __global__ void __launch_bounds__(kNumThreads, 1)
       if constexpr (SWAP) {
         // tile rows are N, tile columns are M: out[m][n]
         const int n = w.tp * BM + row_in_tile;
-        if (n < p.N) {
+        if (!(p.epi & kEpiOutF32)) {
+          // BF16: the whole tile goes through the staging buffer, [BNQ][128]
+          // in the output's order: for each m, the warp's 32 lanes write 32
+          // consecutive n (64 bytes); then one TMA copy stores the tile (rows
+          // past M and columns past N are clipped by the tensor map)
+          const uint32_t stage = smem_addr(epi_bufs);
+          const int act = p.epi & 3;
+          const float bn = (p.bias != nullptr && n < p.N) ? __ldg(p.bias + n) : 0.f;
+          // the previous tile's store must have finished reading the buffer
+          if (ew == 0 && lane == 0) bulk_wait_group_read0();
+          named_barrier_sync(2, kNumEpiThreads);
+#pragma unroll
+          for (int i = 0; i < kHalf; ++i) {
+            const float v = epi_act(((i & 1) ? acc[i / 2].y : acc[i / 2].x) + bn, act);
+            st_shared_b16(stage + ((half * kHalf + i) * BM + row_in_tile) * 2, __bfloat16_as_ushort(__float2bfloat16_rn(v)));
+          }
+          fence_proxy_async_smem();
+          named_barrier_sync(2, kNumEpiThreads);
+          if (ew == 0 && lane == 0) {
+            tma_store_2d(&tm_out, stage, w.tp * BM, w.tq * BNQ);
+            bulk_commit_group();
+          }
+        } else if (n < p.N) {
           const int act = p.epi & 3;
           const float bn = p.bias != nullptr ? __ldg(p.bias + n) : 0.f;
 #pragma unroll
@@ -929,7 +1033,7 @@ __global__ void __launch_bounds__(kNumThreads, 1)
     }
     // every bulk store this warp issued has finished (reads of its staging
     // buffer and writes to global memory) before the CTA exits
-    if constexpr (SC::kTmaStore) {
+    if constexpr (SC::kTmaStore || SC::kSwapTmaStore) {
       if (lane == 0) bulk_wait_group0();
     }
   }

@@ -133,6 +133,7 @@ bsgemm_status launch_fixed(const bsgemm_plan& plan, const void* a, const void* b
   CUtensorMap tm_out;
   std::memset(&tm_out, 0, sizeof tm_out);
   if (SC::kTmaStore && !bsg_host::make_out_map(&tm_out, out, M, N, false)) return BSGEMM_ERR_CUDA;
+  if (SC::kSwapTmaStore && !bsg_host::make_swap_out_map(&tm_out, out, M, N, BNQ)) return BSGEMM_ERR_CUDA;
 
   bsg::Params prm{};
   prm.M = M; prm.N = N; prm.K = K;

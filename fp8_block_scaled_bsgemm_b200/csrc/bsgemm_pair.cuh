@@ -108,6 +108,10 @@ __global__ void __launch_bounds__(kNumThreads, 1)
   cluster_sync_all();
   tc_fence_after();
   const uint32_t tmem_base = bars->tmem_base;
+  // global memory is touched only after the grids this one depends on are
+  // complete (programmatic dependent launch; see bsgemm_kernel)
+  grid_dependency_wait();
+  if (threadIdx.x == 0) grid_launch_dependents();
 
   if (warp < kFirstEpiWarp) {
     set_max_regs_dec<kProducerRegs>();

@@ -67,6 +67,14 @@
  *
  * Results are deterministic: the same inputs give bit-identical outputs
  * (split-K partials are added in a fixed order).
+ *
+ * Launches use programmatic dependent launch: a GEMM kernel may start its
+ * set-up (barriers, TMEM, descriptor prefetch) while the previous kernel on
+ * the stream is finishing, and waits for that kernel to complete, with its
+ * memory visible, before it reads or writes any global memory.  Stream
+ * order is therefore unchanged for the caller.  A later kernel that the
+ * caller launches with programmatic serialisation of its own must likewise
+ * wait (griddepcontrol.wait) before it reads this call's output.
  */
 #ifndef BSGEMM_H
 #define BSGEMM_H

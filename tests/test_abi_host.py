@@ -78,9 +78,12 @@ def test_plan_uses_stream_k_for_a_ragged_last_wave():
     assert bsg.make_plan(4096, 4096, 4096, 128, "nt", 148)["sk_ctas"] == 0
     forced = bsg.make_plan(4096, 4096, 4096, 128, "nt", 148, {"stream_k": 1})
     assert forced["sk_first_tile"] == 444 and forced["sk_ctas"] == 148
-    # fewer tiles than SMs: stream-K for tiles at least 64 wide, split-K below
+    # fewer tiles than SMs: stream-K, whatever the tile width; split-K when
+    # stream-K is turned off
     assert bsg.make_plan(128, 7168, 7168, 128, "nt", 148)["sk_ctas"] == 148
-    small = bsg.make_plan(16, 7168, 7168, 128, "nt", 148)
+    assert bsg.make_plan(16, 7168, 7168, 128, "nt", 148)["sk_ctas"] == 148
+    assert bsg.make_plan(1, 7168, 7168, 128, "nt", 148)["sk_ctas"] == 148
+    small = bsg.make_plan(16, 7168, 7168, 128, "nt", 148, {"stream_k": -1})
     assert small["sk_ctas"] == 0 and small["splits"] > 1
     # an exact number of full waves needs no stream-K
     assert bsg.make_plan(128 * 148, 256, 1024, 128, "nt", 148, {"stream_k": 1})["sk_ctas"] == 0
@@ -144,6 +147,14 @@ def test_stream_k_partition_covers_each_tile_once_in_k_order(tiles_sk, U, G):
                 assert p[3] == 2 * c + (0 if start(c) // U == t else 1)
                 assert p[3] not in used
                 used.add(p[3])
+            # The reducer is piece 0's CTA, and piece 0 is the last segment of
+            # its CTA's range; every later piece is the first segment of its
+            # CTA's range.  So a reducer waits only on pieces their CTAs reach
+            # before any wait of their own: no cycle of waits.
+            c0 = ps[0][0]
+            assert ps[0][1] == 0 and start(c0 + 1) == t * U + ps[0][2]
+            for p in ps[1:]:
+                assert start(p[0]) == t * U + p[1]
 
 
 def test_plan_rejects_bad_tuning():

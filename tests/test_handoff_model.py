@@ -37,8 +37,11 @@ EPI_STAGING = 8 * 32 * 128     # per-warp TMA-store staging of the data-parallel
 
 
 def stages(bnq: int, q_mn: bool, tma_store: bool = False) -> int:
+    """Pipeline stages beside the epilogue staging: 32 KB for data-parallel
+    tiles (tma_store), the BF16 [bnq][128] tile for swap-AB tiles."""
     q_rows = 128 if (q_mn and bnq < 128) else bnq
-    return min(8, (BUDGET - (EPI_STAGING if tma_store else 0)) // (BM_BYTES + q_rows * BK))
+    staging = EPI_STAGING if tma_store else bnq * 128 * 2
+    return min(8, (BUDGET - staging) // (BM_BYTES + q_rows * BK))
 
 
 BM_BYTES = 128 * BK
@@ -245,11 +248,12 @@ def test_handoff_never_aliases_or_deadlocks(bnq, q_mn, tma_store, gran):
 
 def test_stage_counts_match_the_kernel_budget():
     """The 256-wide data-parallel tile keeps 4 stages beside its 32 KB of
-    epilogue staging; the 128-wide one 6; swap-AB 128 keeps 7; the narrow swap
-    tiles 8."""
+    epilogue staging; the 128-wide one 6; swap-AB 128 keeps 6 beside its 32 KB
+    BF16 tile; the narrow swap tiles 8."""
     assert stages(256, False, True) == 4 and stages(256, True, True) == 4
     assert stages(128, False, True) == 6
-    assert stages(128, False, False) == 7 and stages(16, False, False) == 8
+    assert stages(128, False, False) == 6 and stages(64, False, False) == 8
+    assert stages(16, False, False) == 8 and stages(16, True, False) == 6   # MN-major Q: 128-wide atoms
 
 
 MUTATIONS = [
