@@ -232,12 +232,16 @@ extern "C" bsgemm_status bsgemm_make_plan(int layout, int64_t M, int64_t N, int6
   if (variant == BSGEMM_VARIANT_AUTO) {
     variant = (M <= 128) ? BSGEMM_VARIANT_SWAP_AB : BSGEMM_VARIANT_DATA_PARALLEL;
     // CTA pairs halve each SM's operand traffic and double its pipeline
-    // depth; measured on B200 that pays where the promotion hand-off is rare
-    // (g = 256: one per two stages) and there is at least a full wave of
-    // 256 x 256 tiles (long_k g = 256: 219 vs 234 us), not at g = 128.
+    // depth.  Measured on B200 (same box) that pays, given at least a full
+    // wave of 256 x 256 tiles, where the promotion hand-off is rare (g = 256:
+    // one per two stages; long_k 2048 x 4096 x 32768: 223 us) or where a tile
+    // streams a long K (g = 128, K = 32768: 260 against 284 us), not on
+    // short K at g = 128 (4096^3: 78.7 against 70.7 us; FFN: 486 against
+    // 459 us) nor at g = 64.
     const bool tuned = t && (t->bnq != 0 || t->splits != 0 || t->stream_k != 0);
     const int64_t pair_tiles = ((M + 255) / 256) * ((N + 255) / 256);
-    if (!tuned && gran == 256 && M > 128 && num_sms >= 2 && pair_tiles >= num_sms / 2)
+    const bool pair_pays = gran == 256 || (gran == 128 && K >= 16384);
+    if (!tuned && pair_pays && M > 128 && num_sms >= 2 && pair_tiles >= num_sms / 2)
       variant = BSGEMM_VARIANT_CTA_PAIR;
   }
   if (variant == BSGEMM_VARIANT_CTA_PAIR) {
@@ -345,7 +349,13 @@ extern "C" bsgemm_status bsgemm_make_plan(int layout, int64_t M, int64_t N, int6
   if (work > (1 << 30)) return BSGEMM_ERR_INVALID_ARG;  // work items are counted in 32 bits
   if (work < pl.sk_ctas) work = pl.sk_ctas;
   pl.grid = static_cast<int>(work < num_sms ? work : num_sms);
-  pl.group_p = 16;
+  // Raster: the persistent CTAs walk group_p row (P) tiles down, then across
+  // the Q tiles.  DRAM reads are about P-operand + Q-operand x (tiles_p /
+  // group_p): each Q panel is read once per group.  When the whole P operand
+  // fits comfortably in L2 (<= 48 MB of the 126 MB), one group spans all the
+  // row tiles, P stays resident and every Q panel is read once (FFN
+  // 8192 x 14336 x 4096: 265 MB of DRAM reads with groups of 16).
+  pl.group_p = (P * K <= (int64_t(48) << 20)) ? pl.tiles_p : 16;
   pl.layout = layout;
   pl.gran = gran;
   pl.kernels = 1;

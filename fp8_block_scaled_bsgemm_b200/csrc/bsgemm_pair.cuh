@@ -279,7 +279,9 @@ __global__ void __launch_bounds__(kNumThreads, 1)
           s2[j] = make_float2(sv, sv);
         }
         const uint32_t buf = pc % kBufs;
-        if (!warp_wait(smem_addr(&bars->tmem_full[buf]), (pc / kBufs) & 1, p, bars, 4)) { ok = false; break; }
+        // every lane waits on the barrier itself: they all wake together when
+        // the commit lands (a lane-0 wait plus a shuffle measured ~5 % slower)
+        if (!warp_wait_all(smem_addr(&bars->tmem_full[buf]), (pc / kBufs) & 1, p, bars, 4)) { ok = false; break; }
         const uint32_t taddr = tmem_base + t_lane + buf * BNQ + half * kHalf;
         {
           // 64-column chunks; the buffer is released (to the even CTA's

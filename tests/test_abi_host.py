@@ -69,9 +69,11 @@ def test_plan_fills_the_machine_for_small_m():
 
 
 def test_plan_uses_stream_k_for_a_ragged_last_wave():
-    # long K: 256 tiles = 1 wave + 108, whose units are shared out
-    pl = bsg.make_plan(2048, 4096, 32768, 128, "nt", 148)
+    # long K, single-CTA tiles: 256 tiles = 1 wave + 108, whose units are shared out
+    dp = {"variant": "data_parallel"}
+    pl = bsg.make_plan(2048, 4096, 32768, 128, "nt", 148, dp)
     assert pl["sk_first_tile"] == 148 and pl["sk_ctas"] == 148
+    assert bsg.make_plan(2048, 4096, 32768, 64, "nt", 148)["sk_ctas"] == 148
     assert bsg.make_plan(2048, 4096, 32768, 128, "nt", 148, {"stream_k": -1})["sk_ctas"] == 0
     assert bsg.make_plan(2048, 4096, 32768, 128, "nt", 148, {"splits": 2})["sk_ctas"] == 0
     # short K (32 K-blocks): whole tiles unless forced
@@ -100,9 +102,12 @@ def test_plan_for_cta_pairs():
         with pytest.raises(bsg.BsgemmError):
             bsg.make_plan(4096, 4096, 4096, 128, "nt", 148, bad)
     assert bsg.make_plan(4096, 4096, 4096, 128, "nt", 148)["cta_pair"] == 0
-    # the heuristic takes CTA pairs only at g = 256 with a full wave of 256 x 256 tiles
+    # the heuristic takes CTA pairs at g = 256, and at g = 128 for long K, with a
+    # full wave of 256 x 256 tiles
     assert bsg.make_plan(2048, 4096, 32768, 256, "nt", 148)["cta_pair"] == 1
-    assert bsg.make_plan(2048, 4096, 32768, 128, "nt", 148)["cta_pair"] == 0
+    assert bsg.make_plan(2048, 4096, 32768, 128, "nt", 148)["cta_pair"] == 1
+    assert bsg.make_plan(2048, 4096, 32768, 64, "nt", 148)["cta_pair"] == 0
+    assert bsg.make_plan(8192, 14336, 4096, 128, "nt", 148)["cta_pair"] == 0
     assert bsg.make_plan(512, 512, 4096, 256, "nt", 148)["cta_pair"] == 0          # 4 pair tiles
     assert bsg.make_plan(2048, 4096, 32768, 256, "nt", 148, {"stream_k": -1})["cta_pair"] == 0
 
@@ -274,8 +279,10 @@ def test_plan_rejects_sizes_past_its_32_bit_counts():
     with pytest.raises(bsg.BsgemmError):
         bsg.make_plan(1 << 20, 1 << 15, 1 << 20, 64, "nt", 148, {"splits": 1 << 14})
     # the largest sizes themselves still plan
-    pl = bsg.make_plan(1 << 30, 256, 1 << 30, 128, "nt", 148)
+    pl = bsg.make_plan(1 << 30, 256, 1 << 30, 128, "nt", 148, {"variant": "data_parallel"})
     assert pl["tiles_p"] == (1 << 23) and pl["tiles_q"] == 1 and pl["splits"] == 1
+    pl = bsg.make_plan(1 << 30, 256, 1 << 30, 128, "nt", 148)     # long K: CTA pairs
+    assert pl["cta_pair"] == 1 and pl["tiles_p"] == (1 << 22) and pl["tiles_q"] == 1
 
 
 def test_allocation_free_plan_never_pairs_ctas():
