@@ -592,7 +592,11 @@ __global__ void __launch_bounds__(kNumThreads, 1)
   const uint32_t lane = lane_id();
 
   // -------------------------------------------------------------- setup
-  if (threadIdx.x == 0) {
+  // Warp 2 (otherwise idle) initialises the barriers and warp 1 allocates
+  // TMEM, while the producer prefetches the tensor maps and works out its
+  // first work item (integer divisions: ~1000 cycles of one thread), so its
+  // first TMA load issues right after the set-up barrier.
+  if (warp == 2 && lane == 0) {
     for (int s = 0; s < STAGES; ++s) {
       mbar_init(smem_addr(&bars->full[s]), 1);
       mbar_init(smem_addr(&bars->empty[s]), 1);
@@ -606,6 +610,9 @@ __global__ void __launch_bounds__(kNumThreads, 1)
     bars->split_last = 0;
     fence_barrier_init();
   }
+  WorkIter pwit;        // the producer's work cursor and first item
+  Work pw;
+  bool pmore = false;
   if (warp == kProducerWarp && lane == 0) {
     tma_prefetch_desc(&tm_p);
     tma_prefetch_desc(&tm_q);
@@ -613,6 +620,11 @@ __global__ void __launch_bounds__(kNumThreads, 1)
     if constexpr (SC::kTmaStore) tma_prefetch_desc(&tm_out);
     if constexpr (SC::kSwapTmaStore) {
       if (!(p.epi & kEpiOutF32)) tma_prefetch_desc(&tm_out);
+    }
+    if constexpr (!GROUPED) {
+      // from the launch parameters alone: no global memory
+      work_begin<SPLIT, GROUPED>(p, pwit);
+      pmore = work_next<GRAN, SPLIT, GROUPED>(p, pwit, pw);
     }
   }
   if (warp == kMmaWarp) {
@@ -640,13 +652,19 @@ __global__ void __launch_bounds__(kNumThreads, 1)
     if (lane == 0) {
       uint32_t it = 0;  // stage-slot uses so far
       bool ok = true;
-      WorkIter wit;
-      // the grouped work list reads the group sizes from global memory
-      if constexpr (GROUPED) grid_dependency_wait();
-      work_begin<SPLIT, GROUPED>(p, wit);
-      Work w;
-      bool more = work_next<GRAN, SPLIT, GROUPED>(p, wit, w);
-      if constexpr (!GROUPED) grid_dependency_wait();
+      WorkIter gwit;      // grouped: the cursor starts after the wait
+      Work gw;
+      WorkIter& wit = GROUPED ? gwit : pwit;
+      Work& w = GROUPED ? gw : pw;
+      bool more = pmore;
+      if constexpr (GROUPED) {
+        // the grouped work list reads the group sizes from global memory
+        grid_dependency_wait();
+        work_begin<SPLIT, GROUPED>(p, wit);
+        more = work_next<GRAN, SPLIT, GROUPED>(p, wit, w);
+      } else {
+        grid_dependency_wait();
+      }
       for (; ok && more; more = work_next<GRAN, SPLIT, GROUPED>(p, wit, w)) {
         int st0, st1;
         stage_range<GRAN>(p, w, st0, st1);
