@@ -437,6 +437,29 @@ __device__ __forceinline__ float epi_act(float v, int act) {
   return v;
 }
 
+template <int ACT>
+__device__ __forceinline__ float epi_act_t(float v) {
+  if constexpr (ACT == kEpiRelu) return fmaxf(v, 0.f);
+  if constexpr (ACT == kEpiGelu) return 0.5f * v * (1.0f + erff(v * 0.70710678118654752f));
+  return v;
+}
+
+template <int V>
+struct ActTag {
+  static constexpr int value = V;
+};
+
+// Calls f(ActTag<ACT>{}) for the run-time activation code, so loops over
+// elements are instantiated per activation and never carry the other
+// activations' code (evaluated per element, the erf path cost ~90 cycles a
+// value even when the activation was none).
+template <typename F>
+__device__ __forceinline__ void with_act(int act, F&& f) {
+  if (act == kEpiGelu) f(ActTag<kEpiGelu>{});
+  else if (act == kEpiRelu) f(ActTag<kEpiRelu>{});
+  else f(ActTag<0>{});
+}
+
 // out = act(acc + bias[n]) in place on one thread's run of columns
 // [n0, n0 + 2 * NP) (acc pairs in column order).
 template <int NP>
@@ -1000,10 +1023,25 @@ __global__ void __launch_bounds__(kNumThreads, 1)
           // the previous tile's store must have finished reading the buffer
           if (ew == 0 && lane == 0) bulk_wait_group_read0();
           named_barrier_sync(2, kNumEpiThreads);
+          const uint32_t col0 = stage + (half * kHalf * BM + row_in_tile) * 2;  // m = half * kHalf
+          if (p.bias == nullptr && act == 0) {
+            // the plain BF16 output: no activation code in the loop (evaluated
+            // per element, the erf branch cost ~90 cycles a value)
 #pragma unroll
-          for (int i = 0; i < kHalf; ++i) {
-            const float v = epi_act(((i & 1) ? acc[i / 2].y : acc[i / 2].x) + bn, act);
-            st_shared_b16(stage + ((half * kHalf + i) * BM + row_in_tile) * 2, __bfloat16_as_ushort(__float2bfloat16_rn(v)));
+            for (int i = 0; i < kHalf / 2; ++i) {
+              const __nv_bfloat162 h = __float22bfloat162_rn(acc[i]);
+              st_shared_b16(col0 + (2 * i) * BM * 2, __bfloat16_as_ushort(h.x));
+              st_shared_b16(col0 + (2 * i + 1) * BM * 2, __bfloat16_as_ushort(h.y));
+            }
+          } else {
+            with_act(act, [&](auto tag) {
+              constexpr int ACT = decltype(tag)::value;
+#pragma unroll
+              for (int i = 0; i < kHalf; ++i) {
+                const float v = epi_act_t<ACT>(((i & 1) ? acc[i / 2].y : acc[i / 2].x) + bn);
+                st_shared_b16(col0 + i * BM * 2, __bfloat16_as_ushort(__float2bfloat16_rn(v)));
+              }
+            });
           }
           fence_proxy_async_smem();
           named_barrier_sync(2, kNumEpiThreads);
@@ -1014,15 +1052,15 @@ __global__ void __launch_bounds__(kNumThreads, 1)
         } else if (n < p.N) {
           const int act = p.epi & 3;
           const float bn = p.bias != nullptr ? __ldg(p.bias + n) : 0.f;
+          with_act(act, [&](auto tag) {
+            constexpr int ACT = decltype(tag)::value;
 #pragma unroll
-          for (int i = 0; i < kHalf; ++i) {
-            const int m = w.tq * BNQ + half * kHalf + i;
-            const float v = epi_act(((i & 1) ? acc[i / 2].y : acc[i / 2].x) + bn, act);
-            if (m < p.M) {
-              if (p.epi & kEpiOutF32) reinterpret_cast<float*>(p.out)[static_cast<size_t>(m) * p.N + n] = v;
-              else p.out[static_cast<size_t>(m) * p.N + n] = __float2bfloat16_rn(v);
+            for (int i = 0; i < kHalf; ++i) {
+              const int m = w.tq * BNQ + half * kHalf + i;
+              const float v = epi_act_t<ACT>(((i & 1) ? acc[i / 2].y : acc[i / 2].x) + bn);
+              if (m < p.M) reinterpret_cast<float*>(p.out)[static_cast<size_t>(m) * p.N + n] = v;
             }
-          }
+          });
         }
       } else if constexpr (SC::kTmaStore) {
         // this thread owns row m0 + lane, columns [n0, n0 + kHalf); the warp
