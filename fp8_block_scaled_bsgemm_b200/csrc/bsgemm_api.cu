@@ -231,13 +231,15 @@ extern "C" bsgemm_status bsgemm_make_plan(int layout, int64_t M, int64_t N, int6
   int variant = t ? t->variant : BSGEMM_VARIANT_AUTO;
   if (variant == BSGEMM_VARIANT_AUTO) {
     variant = (M <= 128) ? BSGEMM_VARIANT_SWAP_AB : BSGEMM_VARIANT_DATA_PARALLEL;
-    // CTA pairs halve each SM's operand traffic and double its pipeline
-    // depth.  Measured on B200 (same box) that pays, given at least a full
-    // wave of 256 x 256 tiles, where the promotion hand-off is rare (g = 256:
-    // one per two stages; long_k 2048 x 4096 x 32768: 223 us) or where a tile
-    // streams a long K (g = 128, K = 32768: 260 against 284 us), not on
-    // short K at g = 128 (4096^3: 78.7 against 70.7 us; FFN: 486 against
-    // 459 us) nor at g = 64.
+    // CTA pairs halve each SM's operand traffic and deepen its pipeline
+    // (six stages instead of four).  Measured on B200 (same box, back to
+    // back) that pays, given at least a full wave of 256 x 256 tiles, where
+    // the promotion hand-off is rare (g = 256: one per two stages;
+    // 2048 x 4096 x 32768: 224 against 255 us) or where a tile streams a long
+    // K (g = 128, K = 32768: 265 against 288 us).  On short K at g = 128 the
+    // two are within run-to-run noise of each other (4096^3: 71.6-74.9
+    // against 71.9-72.1 us; 6144^2 x 4096: 158 against 145 us), and single
+    // CTAs keep stream-K for ragged waves; at g = 64 pairs lose.
     const bool tuned = t && (t->bnq != 0 || t->splits != 0 || t->stream_k != 0);
     const int64_t pair_tiles = ((M + 255) / 256) * ((N + 255) / 256);
     const bool pair_pays = gran == 256 || (gran == 128 && K >= 16384);

@@ -139,6 +139,8 @@ bsgemm_status launch_pair(const bsgemm_plan& plan, const void* a, const void* b,
   else      ok &= make_map_2d(&tm_p, a, CU_TENSOR_MAP_DATA_TYPE_UINT8, K, M, K, bsg::BK, bsg::BM);
   if (Q_MN) ok &= make_map_2d(&tm_q, b, CU_TENSOR_MAP_DATA_TYPE_UINT8, N, K, N, 128, bsg::BK);
   else      ok &= make_map_2d(&tm_q, b, CU_TENSOR_MAP_DATA_TYPE_UINT8, K, N, K, bsg::BK, bsg::kPairQRows);
+  CUtensorMap tm_out;
+  ok &= make_out_map(&tm_out, out, M, N, (opts.epi & bsg::kEpiOutF32) != 0);
   if (!ok) return BSGEMM_ERR_CUDA;
 
   bsg::Params prm{};
@@ -203,7 +205,7 @@ bsgemm_status launch_pair(const bsgemm_plan& plan, const void* a, const void* b,
   if (pairs > max_pairs) pairs = max_pairs;
   if (pairs < 1) return BSGEMM_ERR_INVALID_ARG;
   cfg.gridDim = dim3(2 * pairs, 1, 1);
-  if (cudaLaunchKernelEx(&cfg, kern, tm_p, tm_q, prm) != cudaSuccess) return BSGEMM_ERR_CUDA;
+  if (cudaLaunchKernelEx(&cfg, kern, tm_p, tm_q, tm_out, prm) != cudaSuccess) return BSGEMM_ERR_CUDA;
   return cudaGetLastError() == cudaSuccess ? BSGEMM_OK : BSGEMM_ERR_CUDA;
 }
 

@@ -9,8 +9,12 @@
 //   N = 256, K = 32), which reads A and B from both CTAs' shared memory and
 //   writes rows 128 r .. 128 r + 127 of the partial into CTA r's TMEM.
 // Each SM therefore streams 32 KB of operands per 128-deep stage for the same
-// tensor work that costs 48 KB with a 128 x 256 tile per CTA, and seven
-// stages fit in shared memory instead of four.
+// tensor work that costs 48 KB with a 128 x 256 tile per CTA, and six stages
+// fit in shared memory beside the 32 KB of epilogue staging, instead of four.
+// The epilogue is the single-CTA kernel's: each promotion warp stages its 32
+// rows x 128 columns in 128-byte-swizzled chunks and one lane issues bulk
+// tensor stores, so a tile's output leaves while the next tile's first
+// K-blocks are promoted.
 //
 // Synchronisation (all mbarrier waits bounded, as in bsgemm_kernel):
 //   full[s]        even CTA only: the even CTA's producer expects both CTAs'
@@ -36,10 +40,11 @@ struct PairCfg {
   static constexpr int kPBytes = BM * BK;          // 16 KB
   static constexpr int kQBytes = kPairQRows * BK;  // 16 KB
   static constexpr int kStageBytes = kPBytes + kQBytes;
+  static constexpr int kEpiBytes = kNumEpiWarps * kEpiChunkBytes;  // 32 KB of store staging
   static constexpr int kBudget = 227 * 1024 - 1024 /*align slack*/ - 512 /*barriers*/;
-  static constexpr int kStagesRaw = kBudget / kStageBytes;
+  static constexpr int kStagesRaw = (kBudget - kEpiBytes) / kStageBytes;
   static constexpr int kStages = kStagesRaw > 8 ? 8 : kStagesRaw;
-  static constexpr int kSmemBytes = 1024 + kStages * kStageBytes + 512;
+  static constexpr int kSmemBytes = 1024 + kStages * kStageBytes + kEpiBytes + 512;
 };
 
 template <bool P_MN, bool Q_MN>
@@ -56,7 +61,7 @@ __device__ __forceinline__ constexpr uint32_t instr_desc_pair() {
 template <int GRAN, bool P_MN, bool Q_MN>
 __global__ void __launch_bounds__(kNumThreads, 1)
     bsgemm_pair_kernel(const __grid_constant__ CUtensorMap tm_p, const __grid_constant__ CUtensorMap tm_q,
-                       const Params p) {
+                       const __grid_constant__ CUtensorMap tm_out, const Params p) {
   using PC = PairCfg;
   constexpr int STAGES = PC::kStages;
   constexpr int BNQ = kPairN;
@@ -73,7 +78,8 @@ __global__ void __launch_bounds__(kNumThreads, 1)
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* p_tiles = smem;
   uint8_t* q_tiles = smem + STAGES * PC::kPBytes;
-  Barriers* bars = reinterpret_cast<Barriers*>(q_tiles + STAGES * PC::kQBytes);
+  uint8_t* epi_bufs = q_tiles + STAGES * PC::kQBytes;  // 1024-aligned: stage sizes are multiples of 1 KB
+  Barriers* bars = reinterpret_cast<Barriers*>(epi_bufs + PC::kEpiBytes);
 
   const int warp = threadIdx.x / 32;
   const uint32_t lane = lane_id();
@@ -99,6 +105,7 @@ __global__ void __launch_bounds__(kNumThreads, 1)
   if (warp == kProducerWarp && lane == 0) {
     tma_prefetch_desc(&tm_p);
     tma_prefetch_desc(&tm_q);
+    tma_prefetch_desc(&tm_out);
   }
   if (warp == kMmaWarp) {
     tmem_alloc_pair(smem_addr(&bars->tmem_base), kTmemCols);
@@ -310,10 +317,15 @@ __global__ void __launch_bounds__(kNumThreads, 1)
       if (!ok) break;
 
       // ---------------------------------------------------------- epilogue + store
-      const int m = prow0 + row_in_tile;
+      // this thread owns row prow0 + row_in_tile, columns [n0, n0 + kHalf);
+      // the warp stores its 32 rows through its staging buffer
       const int n0 = tq * kPairN + half * kHalf;
-      if (m < p.M) store_row_run<kHalf / 2>(p, m, n0, acc);
+      apply_epi<kHalf / 2>(p, n0, acc);
+      store_tile_tma<kHalf / 2>(p, &tm_out, smem_addr(epi_bufs + ew * kEpiChunkBytes), prow0 + quad * 32, n0,
+                                acc, lane);
     }
+    // every bulk store this warp issued has finished before the CTA exits
+    if (lane == 0) bulk_wait_group0();
   }
   __syncwarp();
 
