@@ -598,6 +598,26 @@ __global__ void __launch_bounds__(kNumThreads, 1)
   constexpr uint32_t kTmemCols = (kBufs * BNQ <= 32) ? 32 : (kBufs * BNQ <= 64) ? 64
                                 : (kBufs * BNQ <= 128) ? 128 : (kBufs * BNQ <= 256) ? 256 : 512;
   static_assert(kBufs * BNQ <= 512, "TMEM holds 512 columns");
+  // Two MMA-issuing warps take the K-blocks in turn (issuer x % 2 takes the
+  // CTA's K-block x, counted over all its work items).  One warp issues a
+  // tcgen05.mma about every 80 cycles whatever its N (measured on B200), and
+  // each barrier wait and commit adds to that, so one warp alone leaves the
+  // tensor core idle between narrow instructions.  Parity waits are only
+  // sound when a waiter observes every phase of its barrier in turn, so:
+  // - every TMEM buffer belongs to one issuer (kBufs even, x % kBufs);
+  // - at g = 128 a K-block is one stage, so with an even number of stages
+  //   every stage belongs to one issuer, which alone releases it;
+  // - otherwise stages change hands (g = 64: a stage holds blocks x and
+  //   x + 1; g = 256: a block is two stages, or one at the K tail; an odd
+  //   ring, as in the grouped 128-wide tiles' seven stages), and both
+  //   issuers wait for every stage and release it: the owner after its MMAs,
+  //   the other by a commit of no MMAs.  Having waited for the stage's fill,
+  //   whose phase the previous release completed, neither release can land
+  //   in an earlier phase.
+  constexpr int kIssuers = 2;
+  constexpr bool kSharedStages = (GRAN != BK) || (STAGES % kIssuers != 0);
+  constexpr int kStageUsers = kSharedStages ? 2 : 1;
+  static_assert(kBufs % kIssuers == 0, "TMEM buffers split evenly between the issuers");
   constexpr uint32_t kTxBytes = TL::kPBytes + TL::kQBytes;
   static_assert(BNQ % 16 == 0 && BNQ >= 16 && BNQ <= 256, "MMA N must be a multiple of 16 in [16, 256]");
   static_assert(GRAN == 64 || GRAN == 128 || GRAN == 256, "granularity");
@@ -622,13 +642,13 @@ __global__ void __launch_bounds__(kNumThreads, 1)
   if (warp == 2 && lane == 0) {
     for (int s = 0; s < STAGES; ++s) {
       mbar_init(smem_addr(&bars->full[s]), 1);
-      mbar_init(smem_addr(&bars->empty[s]), 1);
+      mbar_init(smem_addr(&bars->empty[s]), kStageUsers);
     }
     for (int b = 0; b < kBufs; ++b) {
       mbar_init(smem_addr(&bars->tmem_full[b]), 1);
       mbar_init(smem_addr(&bars->tmem_empty[b]), kNumEpiWarps);
     }
-    mbar_init(smem_addr(&bars->mma_done), 1);
+    mbar_init(smem_addr(&bars->mma_done), kIssuers);
     bars->abort_flag = 0;
     bars->split_last = 0;
     fence_barrier_init();
@@ -721,17 +741,22 @@ __global__ void __launch_bounds__(kNumThreads, 1)
           bounded_wait(smem_addr(&bars->full[j % STAGES]), (j / STAGES) & 1, p, bars, 9, true);
       }
     }
-  } else if (warp == kMmaWarp) {
-    // ============================================================ MMA issuer
-    // Per K-block the issuer claims a TMEM buffer, issues the block's MMAs
+  } else if (warp == kMmaWarp || warp == kMmaWarp + 1) {
+    // ============================================================ MMA issuers
+    // Issuer i (warp kMmaWarp + i) takes the K-blocks of parity i, in K
+    // order: it claims the block's TMEM buffer, issues the block's MMAs
     // (K = 32 each) stage by stage -- waiting for a stage at its first k-step,
     // releasing it after its last -- and commits the buffer to the promotion
-    // warps as soon as the block's last MMA is issued (the promotion of block
-    // kb gates the MMAs of block kb + kBufs). The whole warp runs the loop,
-    // converged: every lane polls the barriers, descriptors are warp-uniform,
-    // and each tcgen05 instruction is predicated on elect.sync, so one lane
-    // (always the same) issues it without the warp ever diverging.
+    // warps after the block's last MMA (the promotion of block x gates the
+    // MMAs of block x + kBufs).  Both issuers walk every work item and stage,
+    // so the stage ring and the K-block counter (buffer x % kBufs) agree
+    // between them, the producer and the promotion warps.  A commit tracks
+    // the MMAs of its own thread only, so the issuers' commits are
+    // independent.  Each warp runs converged: every lane polls the barriers,
+    // descriptors are warp-uniform, and each tcgen05 instruction is
+    // predicated on elect.sync, so one lane (always the same) issues it.
     {
+      const uint32_t issuer = static_cast<uint32_t>(warp - kMmaWarp);
       const uint32_t idesc = instr_desc<BNQ, P_MN, Q_MN>() | p.fmt_bits;
       // descriptor steps: per k-step of 32 (K-major +32 B, MN-major +32 rows
       // of 128 B) and per pipeline stage, in the descriptor's 16-byte units
@@ -741,70 +766,90 @@ __global__ void __launch_bounds__(kNumThreads, 1)
       const uint64_t ad0 = smem_desc_sw128(smem_addr(p_tiles), P_MN ? 128 * BK : 16);
       const uint64_t bd0 = smem_desc_sw128(smem_addr(q_tiles), Q_MN ? 128 * BK : 16);
       uint32_t s = 0, ph = 0;     // pipeline stage and its phase
-      uint32_t b = 0, bph = 0;    // TMEM buffer and its phase
+      uint32_t x = 0;             // K-blocks so far
       bool ok = true;
       WorkIter wit;
       // the grouped work list reads the group sizes from global memory
       if constexpr (GROUPED) grid_dependency_wait();
       work_begin<SPLIT, GROUPED>(p, wit);
       for (Work w; ok && work_next<GRAN, SPLIT, GROUPED>(p, wit, w);) {
-        for (int kb = w.kb0; kb < w.kb1; ++kb) {
+        for (int kb = w.kb0; kb < w.kb1; ++kb, ++x) {
           // Order of the waits: the stage's operands first (normally already
-          // loaded, so that wait is cheap and happens while the tensor pipe
-          // still works on the previous block), then the TMEM buffer, which
-          // gates the MMAs; the promotion warps arrive on tmem_empty only
-          // after tcgen05.wait::ld, so their reads of the buffer are complete
+          // loaded, so that wait is cheap), then the TMEM buffer, which gates
+          // the MMAs; the promotion warps arrive on tmem_empty only after
+          // tcgen05.wait::ld, so their reads of the buffer are complete
           // before it is overwritten.  Commits: tmem_full first (the
           // promotion warps wait on it), then the stage release.
+          const uint32_t b = x % kBufs, bph = (x / kBufs) & 1;
           const uint32_t d_tmem = tmem_base + b * BNQ;
           if constexpr (GRAN >= BK) {
             // whole stages: GRAN / 128 of them, 4 k-steps each (fewer at the K tail)
+            const bool mine = (x & 1) == issuer;
 #pragma unroll
             for (int j = 0; j < GRAN / BK; ++j) {
               const int k0 = kb * GRAN + j * BK;
               if (k0 >= p.K) break;
-              // TMA writes and MMA reads are async-proxy accesses ordered by this barrier
-              if (!warp_wait_all(smem_addr(&bars->full[s]), ph, p, bars, 2)) { ok = false; break; }
-              if (j == 0 && !warp_wait_all(smem_addr(&bars->tmem_empty[b]), bph ^ 1, p, bars, 3)) {
-                ok = false;
-                break;
+              if (!mine && kSharedStages) {
+                // the other issuer's stage: observe its fill and release it
+                // (a commit of no MMAs: it follows this issuer's own MMAs)
+                if (!warp_wait_all(smem_addr(&bars->full[s]), ph, p, bars, 2)) { ok = false; break; }
+                mma_commit_elect(smem_addr(&bars->empty[s]));
               }
-              const uint64_t ad = ad0 + s * kPStage, bd = bd0 + s * kQStage;
-              if (k0 + BK <= p.K) {
+              if (mine) {
+                // TMA writes and MMA reads are async-proxy accesses ordered by this barrier
+                if (!warp_wait_all(smem_addr(&bars->full[s]), ph, p, bars, 2)) { ok = false; break; }
+                if (j == 0 && !warp_wait_all(smem_addr(&bars->tmem_empty[b]), bph ^ 1, p, bars, 3)) {
+                  ok = false;
+                  break;
+                }
+                const uint64_t ad = ad0 + s * kPStage, bd = bd0 + s * kQStage;
+                if (k0 + BK <= p.K) {
 #pragma unroll
-                for (int t = 0; t < BK / kMmaK; ++t)
-                  mma_f8f6f4_elect(d_tmem, ad + t * kPStep, bd + t * kQStep, idesc, (j > 0 || t > 0) ? 1u : 0u);
-              } else {
-                const int nsteps = (p.K - k0 + kMmaK - 1) / kMmaK;
-                for (int t = 0; t < nsteps; ++t)
-                  mma_f8f6f4_elect(d_tmem, ad + t * kPStep, bd + t * kQStep, idesc, (j > 0 || t > 0) ? 1u : 0u);
+                  for (int t = 0; t < BK / kMmaK; ++t)
+                    mma_f8f6f4_elect(d_tmem, ad + t * kPStep, bd + t * kQStep, idesc, (j > 0 || t > 0) ? 1u : 0u);
+                } else {
+                  const int nsteps = (p.K - k0 + kMmaK - 1) / kMmaK;
+                  for (int t = 0; t < nsteps; ++t)
+                    mma_f8f6f4_elect(d_tmem, ad + t * kPStep, bd + t * kQStep, idesc, (j > 0 || t > 0) ? 1u : 0u);
+                }
+                if (j == GRAN / BK - 1 || k0 + BK >= p.K) mma_commit_elect(smem_addr(&bars->tmem_full[b]));
+                mma_commit_elect(smem_addr(&bars->empty[s]));  // stage free once these MMAs finish
               }
-              if (j == GRAN / BK - 1 || k0 + BK >= p.K) mma_commit_elect(smem_addr(&bars->tmem_full[b]));
-              mma_commit_elect(smem_addr(&bars->empty[s]));  // stage free once these MMAs finish
               if (++s == STAGES) { s = 0; ph ^= 1; }
             }
             if (!ok) break;
           } else {
-            // GRAN == 64: a K-block is half a stage; even blocks open the
-            // stage, odd blocks (or the K tail) release it
+            // GRAN == 64: a K-block is half a stage (work items start on even
+            // K-blocks, so a stage holds consecutive blocks x and x + 1, one
+            // per issuer) and each issuer releases the stage after its half.
+            // Where the K tail leaves a stage without its second half, the
+            // other issuer waits for it and releases it all the same.
             const int k0 = kb * GRAN;
             const int t0 = (kb & 1) * 2;
-            if (t0 == 0 && !warp_wait_all(smem_addr(&bars->full[s]), ph, p, bars, 2)) { ok = false; break; }
-            if (!warp_wait_all(smem_addr(&bars->tmem_empty[b]), bph ^ 1, p, bars, 3)) { ok = false; break; }
-            const uint64_t ad = ad0 + s * kPStage, bd = bd0 + s * kQStage;
-            const int nsteps = (p.K - k0 >= GRAN) ? 2 : (p.K - k0 + kMmaK - 1) / kMmaK;
-            for (int t = 0; t < nsteps; ++t)
-              mma_f8f6f4_elect(d_tmem, ad + (t0 + t) * kPStep, bd + (t0 + t) * kQStep, idesc, t > 0 ? 1u : 0u);
-            mma_commit_elect(smem_addr(&bars->tmem_full[b]));
-            if (t0 == 2 || k0 + GRAN >= p.K) {
+            const bool last_in_stage = (t0 == 2 || k0 + GRAN >= p.K);
+            if ((x & 1) == issuer) {
+              // (a stage's two halves belong to different issuers, so each
+              // issuer waits for every stage once)
+              if (!warp_wait_all(smem_addr(&bars->full[s]), ph, p, bars, 2)) { ok = false; break; }
+              if (!warp_wait_all(smem_addr(&bars->tmem_empty[b]), bph ^ 1, p, bars, 3)) { ok = false; break; }
+              const uint64_t ad = ad0 + s * kPStage, bd = bd0 + s * kQStage;
+              const int nsteps = (p.K - k0 >= GRAN) ? 2 : (p.K - k0 + kMmaK - 1) / kMmaK;
+              for (int t = 0; t < nsteps; ++t)
+                mma_f8f6f4_elect(d_tmem, ad + (t0 + t) * kPStep, bd + (t0 + t) * kQStep, idesc, t > 0 ? 1u : 0u);
+              mma_commit_elect(smem_addr(&bars->tmem_full[b]));
               mma_commit_elect(smem_addr(&bars->empty[s]));
+            } else if (t0 == 0 && last_in_stage) {
+              // the stage has no second half: wait for it all the same
+              if (!warp_wait_all(smem_addr(&bars->full[s]), ph, p, bars, 2)) { ok = false; break; }
+              mma_commit_elect(smem_addr(&bars->empty[s]));
+            }
+            if (last_in_stage) {
               if (++s == STAGES) { s = 0; ph ^= 1; }
             }
           }
-          if (++b == kBufs) { b = 0; bph ^= 1; }
         }
       }
-      // all MMAs issued by the elected lane complete before TMEM is freed
+      // all MMAs issued by both issuers complete before TMEM is freed
       mma_commit_elect(smem_addr(&bars->mma_done));
       warp_wait_all(smem_addr(&bars->mma_done), 0, p, bars, 8, true);
     }

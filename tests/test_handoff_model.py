@@ -1,24 +1,30 @@
 """Model check of the single-CTA GEMM kernel's K-block hand-off (CPU only).
 
-Three roles share two barrier rings in ``csrc/bsgemm_kernel.cuh``:
+Four roles share two barrier rings in ``csrc/bsgemm_kernel.cuh``:
 - the TMA producer fills stage s and completes ``full[s]``; before refilling it,
   it waits for ``empty[s]``;
-- the MMA warp waits for ``full[s]`` and then for TMEM buffer b (``tmem_empty[b]``).
-  It issues the K-block's MMAs and commits ``tmem_full[b]`` after the block's last
-  stage and ``empty[s]`` after each stage. At g = 64 a stage holds two K-blocks;
-  at g = 256 a K-block spans two stages;
+- two MMA issuers take the K-blocks in turn (issuer i the blocks of parity i).
+  Each walks every stage and, for its own blocks, waits for ``full[s]`` and then
+  for TMEM buffer b (``tmem_empty[b]``), issues the MMAs, commits
+  ``tmem_full[b]`` after the block's last stage and ``empty[s]`` after each
+  stage. At g = 64 a stage holds two K-blocks, one per issuer, so ``empty[s]``
+  needs both issuers' commits; where the K tail leaves a stage without its
+  second half, issuer 1 commits without MMAs. At g = 256 a K-block spans two
+  stages;
 - the promotion warps wait for ``tmem_full[b]``, read the partial and arrive on
   ``tmem_empty[b]``.
 
 Every wait is a parity wait: waiting for phase k passes when the barrier's
 completed-phase count c has (c & 1) != (k & 1). That answer is only right when
 c == k + 1. A barrier one phase behind (c == k - 1) or two ahead (c == k + 2)
-gives the same answer, which is aliasing. The model runs the three roles with
-these barriers as counters. The MMA completions are asynchronous, in issue
-order, and the TMA completions come in any order. Random schedules are run
-over random work lists: whole tiles, split-K pieces and stream-K ranges, with
-a partial last K-block. The checks:
-- no wait passes at a count other than k + 1, and the roles never deadlock;
+gives the same answer, which is aliasing. The model runs the roles with these
+barriers as counters. A commit completes once its issuer's earlier MMAs have
+(each issuer's commits in order, the two issuers' in any order), and the TMA
+completions come in any order. Random schedules are run over random work
+lists: whole tiles, split-K pieces and stream-K ranges, with a partial last
+K-block. The checks:
+- no wait passes at a count other than k + 1, no arrival lands in another
+  phase than the one it is meant for, and the roles never deadlock;
 - no stage is overwritten while MMAs read it or before they have used it;
 - no TMEM buffer is rewritten before the promotion has read it;
 - no MMA reads a stage before its copy landed, and no promotion reads an
@@ -83,9 +89,75 @@ class Bar:
         return (self.c & 1) != (k & 1)
 
 
+class CountBar(Bar):
+    """A barrier whose phase completes after `need` arrivals; an arrival meant
+    for another phase than the current one is an error."""
+    __slots__ = ("need", "got")
+
+    def __init__(self, need):
+        super().__init__()
+        self.need, self.got = need, 0
+
+    def add(self, phase, errors, what):
+        if phase != self.c:
+            errors.append(f"{what}: arrival for phase {phase} landed during phase {self.c}")
+            return
+        self.got += 1
+        if self.got == self.need:
+            self.c += 1
+            self.got = 0
+
+
+def programs(gran, K, items, S, mutation=None):
+    """The producer's stage slots and each issuer's steps, as the kernel runs
+    them. A step: (slot, wait_full, wait_block, mma, commit_block, commit_slot);
+    wait_block / commit_block name the K-block whose TMEM buffer is claimed /
+    committed, or None. Issuer x % 2 takes K-block x."""
+    shared = (gran != BK or S % 2 == 1) and mutation != "skip_foreign_stage_wait"
+    by_kb = mutation == "issuer_by_kb"
+    nst = -(-K // BK)
+    nslots = 0
+    steps = ([], [])
+    x = 0
+    for kb0, kb1 in items:
+        if gran >= BK:
+            st0, st1 = kb0 * (gran // BK), kb1 * (gran // BK)
+        else:
+            st0, st1 = kb0 // 2, (kb1 + 1) // 2
+        nslots += min(st1, nst) - st0
+    slot = 0
+    for kb0, kb1 in items:
+        for kb in range(kb0, kb1):
+            owner = (kb if by_kb else x) & 1
+            if gran >= BK:
+                for j in range(gran // BK):
+                    k0 = kb * gran + j * BK
+                    if k0 >= K:
+                        break
+                    last = j == gran // BK - 1 or k0 + BK >= K
+                    steps[owner].append((slot, True, x if j == 0 else None, True, x if last else None, slot))
+                    if shared:
+                        steps[1 - owner].append((slot, True, None, False, None, slot))
+                    slot += 1
+            else:
+                k0 = kb * gran
+                t0 = kb & 1
+                last_in_stage = t0 == 1 or k0 + gran >= K
+                steps[owner].append((slot, True, x, True, x, slot))
+                if t0 == 0 and last_in_stage and mutation != "tail_no_release":
+                    steps[1 - owner].append((slot, True, None, False, None, slot))
+                if last_in_stage:
+                    slot += 1
+            x += 1
+    assert slot == nslots
+    return nslots, steps, x
+
+
 def simulate(S, B, gran, K, items, rng, mutation=None):
+    shared = (gran != BK or S % 2 == 1) and mutation != "skip_foreign_stage_wait"
+    stage_users = 1 if (mutation == "one_stage_user" or not shared) else 2
     full = [Bar() for _ in range(S)]
-    empty = [Bar() for _ in range(S)]
+    empty = [CountBar(stage_users) for _ in range(S)]
     tfull = [Bar() for _ in range(B)]
     tempty = [Bar() for _ in range(B)]
     errors = []
@@ -94,136 +166,116 @@ def simulate(S, B, gran, K, items, rng, mutation=None):
         if bar.c != k + 1:
             errors.append(f"{what}: waited for phase {k}, count was {bar.c}")
 
-    nst = -(-K // BK)
+    nslots, steps, nblocks = programs(gran, K, items, S, mutation)
+    readers = [0] * nslots          # MMA groups that read each slot
+    for prog in steps:
+        for st in prog:
+            if st[3]:
+                readers[st[0]] += 1
+    reads_done = [0] * nslots       # ... of which completed
 
-    # producer program: the stage slots it fills, in order
-    prod = []
-    for kb0, kb1 in items:
-        if gran >= BK:
-            st0, st1 = kb0 * (gran // BK), kb1 * (gran // BK)
-        else:
-            st0, st1 = kb0 // 2, (kb1 + 1) // 2
-        prod += [None] * (min(st1, nst) - st0)
-
-    # MMA program: a list of steps (wait_full, wait_tmem, commit_tmem_full, commit_empty)
-    mma = []
-    for kb0, kb1 in items:
-        for kb in range(kb0, kb1):
-            if gran >= BK:
-                for j in range(gran // BK):
-                    k0 = kb * gran + j * BK
-                    if k0 >= K:
-                        break
-                    last = j == gran // BK - 1 or k0 + BK >= K
-                    mma.append((True, j == 0, last, True))
-            else:
-                k0 = kb * gran
-                t0 = kb & 1
-                mma.append((t0 == 0, True, True, t0 == 1 or k0 + gran >= K))
-    nblocks = sum(kb1 - kb0 for kb0, kb1 in items)
-
-    p_it = 0                       # producer: stage slots filled
-    landing = []                   # TMA copies in flight (stage indices)
-    m_i = 0                        # MMA: next step
-    m_st = 0                       # MMA: stage slots consumed
-    m_blk = 0                      # MMA: K-blocks started
-    m_sub = 0                      # MMA: 0 = before its waits, 1 = full passed
-    inflight = []                  # MMA commits not yet complete, in issue order
+    p_it = 0                        # producer: stage slots filled
+    landing = []                    # TMA copies in flight (slots)
+    landed = set()
+    m_i = [0, 0]                    # each issuer: next step
+    m_sub = [0, 0]                  # 0 = before its waits, 1 = full passed
+    inflight = ([], [])             # each issuer's commits not yet complete, in issue order
     promo = 0
-    reading = [0] * S              # MMA groups in flight that read each stage
-    stage_done = 0                 # stage slots whose reads are complete
-    blocks_done = 0                # K-blocks whose MMAs are complete
-    landed = set()                 # stage slots whose copies landed
-    # adversarial pacing: some roles run far slower than the others in this run
-    slow = {r for r in ("prod", "land", "mma", "m_done", "promo") if rng.random() < 0.3}
+    blocks_done = set()
+    slow = {r for r in ("prod", "land", "mma0", "mma1", "done0", "done1", "promo") if rng.random() < 0.3}
     guard = 0
-    while promo < nblocks and not errors:
+    def running():
+        return (promo < nblocks or p_it < nslots or landing or inflight[0] or inflight[1] or
+                m_i != [len(steps[0]), len(steps[1])])
+
+    while running() and not errors:
         guard += 1
-        if guard > 200000:
+        if guard > 300000:
             errors.append("no progress")
             break
         acts = []
-        if p_it < len(prod):
+        if p_it < nslots:
             k = p_it // S - (0 if mutation == "producer_phase" else 1)
             if k < 0 or empty[p_it % S].passes(k):
-                acts.append("prod")
+                acts.append(("prod",))
         if landing:
-            acts.append("land")
-        if m_i < len(mma):
-            wf, wt, _, _ = mma[m_i]
-            s = m_st % S
-            if m_sub == 0 and wf:
-                if full[s].passes(m_st // S):
-                    acts.append("m_full")
-            else:
-                b, k = m_blk % B, m_blk // B - (0 if mutation == "tmem_phase" else 1)
-                if not wt or k < 0 or mutation == "skip_tmem_wait" or tempty[b].passes(k):
-                    acts.append("m_issue")
-        if inflight:
-            acts.append("m_done")
-        b, k = promo % B, promo // B - (1 if mutation == "promo_phase" else 0)
-        if k < 0 or tfull[b].passes(k):
-            acts.append("promo")
+            acts.append(("land",))
+        for i in (0, 1):
+            if m_i[i] < len(steps[i]):
+                slot, wf, wb, _, _, _ = steps[i][m_i[i]]
+                if m_sub[i] == 0 and wf:
+                    if full[slot % S].passes(slot // S):
+                        acts.append(("m_full", i))
+                else:
+                    ok = True
+                    if wb is not None and mutation != "skip_tmem_wait":
+                        k = wb // B - (0 if mutation == "tmem_phase" else 1)
+                        ok = k < 0 or tempty[wb % B].passes(k)
+                    if ok:
+                        acts.append(("m_issue", i))
+            if inflight[i]:
+                acts.append(("m_done", i))
+        k = promo // B - (1 if mutation == "promo_phase" else 0)
+        if promo < nblocks and (k < 0 or tfull[promo % B].passes(k)):
+            acts.append(("promo",))
         if not acts:
-            errors.append(f"deadlock: producer {p_it}/{len(prod)}, mma {m_i}/{len(mma)}, promotion {promo}")
+            errors.append(f"deadlock: producer {p_it}/{nslots}, issuers {m_i}, promotion {promo}/{nblocks}")
             break
-        role = {"m_full": "mma", "m_issue": "mma"}
-        weights = [0.03 if role.get(x, x) in slow else 1.0 for x in acts]
-        a = rng.choices(acts, weights)[0]
-        if a == "prod":
+
+        def role(a):
+            return {"m_full": f"mma{a[-1]}", "m_issue": f"mma{a[-1]}", "m_done": f"done{a[-1]}"}.get(a[0], a[0])
+        a = rng.choices(acts, [0.03 if role(x) in slow else 1.0 for x in acts])[0]
+        if a[0] == "prod":
             if p_it // S - 1 >= 0 and mutation is None:
                 check(empty[p_it % S], p_it // S - 1, f"producer slot {p_it}")
-            if reading[p_it % S] or stage_done < p_it - S + 1:
-                errors.append(f"producer slot {p_it}: stage {p_it % S} overwritten while in use")
+            old = p_it - S
+            if old >= 0 and reads_done[old] < readers[old]:
+                errors.append(f"producer slot {p_it}: stage {p_it % S} overwritten while slot {old} is read")
             landing.append(p_it)
             p_it += 1
-        elif a == "land":
+        elif a[0] == "land":
             slot = landing.pop(rng.randrange(len(landing)))
             landed.add(slot)
             full[slot % S].c += 1
-        elif a == "m_full":
-            check(full[m_st % S], m_st // S, f"mma step {m_i} (full)")
-            m_sub = 1
-        elif a == "m_issue":
-            wf, wt, ctf, cem = mma[m_i]
-            if wt and m_blk // B - 1 >= 0 and mutation is None:
-                check(tempty[m_blk % B], m_blk // B - 1, f"mma step {m_i} (tmem_empty)")
-            if m_st not in landed:
-                errors.append(f"mma step {m_i}: stage slot {m_st} read before its copy landed")
-            if wt and promo < m_blk - B + 1:
-                errors.append(f"mma step {m_i}: buffer {m_blk % B} rewritten before block "
-                              f"{m_blk - B} was promoted")
-            reading[m_st % S] += 1
-            if mutation == "early_release" and cem:
-                empty[m_st % S].c += 1
-                stage_done += 1
-                cem_late = False
-            else:
-                cem_late = cem
-            inflight.append((m_blk % B if ctf else None, m_st % S if cem_late else None, m_st % S))
-            if ctf:
-                m_blk += 1
-            if cem:
-                m_st += 1
-            m_i += 1
-            m_sub = 0
-        elif a == "m_done":
-            tb, es, rs = inflight.pop(0)
-            reading[rs] -= 1
-            if tb is not None:
-                tfull[tb].c += 1
-                blocks_done += 1
-            if es is not None:
-                empty[es].c += 1
-                stage_done += 1
+        elif a[0] == "m_full":
+            i = a[1]
+            slot = steps[i][m_i[i]][0]
+            check(full[slot % S], slot // S, f"issuer {i} step {m_i[i]} (full)")
+            m_sub[i] = 1
+        elif a[0] == "m_issue":
+            i = a[1]
+            slot, wf, wb, mma, cb, cs = steps[i][m_i[i]]
+            if wb is not None:
+                if wb // B - 1 >= 0 and mutation is None:
+                    check(tempty[wb % B], wb // B - 1, f"issuer {i} step {m_i[i]} (tmem_empty)")
+                if promo < wb - B + 1:
+                    errors.append(f"issuer {i}: buffer {wb % B} rewritten before block {wb - B} was promoted")
+            if mma and slot not in landed:
+                errors.append(f"issuer {i}: stage slot {slot} read before its copy landed")
+            if mutation == "early_release" and cs is not None and mma:
+                empty[cs % S].add(cs // S, errors, f"issuer {i} early release, slot {cs}")
+                cs = None
+            inflight[i].append((slot if mma else None, cb, cs))
+            m_i[i] += 1
+            m_sub[i] = 0
+        elif a[0] == "m_done":
+            i = a[1]
+            rs, cb, cs = inflight[i].pop(0)
+            if rs is not None:
+                reads_done[rs] += 1
+            if cb is not None:
+                tfull[cb % B].c += 1
+                blocks_done.add(cb)
+            if cs is not None:
+                empty[cs % S].add(cs // S, errors, f"issuer {i} commit, slot {cs}")
         else:
             if mutation is None:
                 check(tfull[promo % B], promo // B, f"promotion block {promo}")
-            if blocks_done < promo + 1:
+            if promo not in blocks_done:
                 errors.append(f"promotion block {promo}: read an unfinished partial")
             tempty[promo % B].c += 1
             promo += 1
-    if not errors and (m_i != len(mma) or p_it != len(prod)):
+    if not errors and (m_i != [len(steps[0]), len(steps[1])] or p_it != nslots):
         errors.append("roles finished out of step")
     return errors
 
@@ -232,6 +284,19 @@ def simulate(S, B, gran, K, items, rng, mutation=None):
 # every stage, data-parallel tiles (128, 256) give 32 KB to the epilogue staging
 CONFIGS = ([(bnq, q_mn, False) for bnq in (16, 32, 64, 128) for q_mn in (False, True)] +
            [(bnq, q_mn, True) for bnq in (128, 256) for q_mn in (False, True)])
+
+
+def test_odd_ring_shares_its_stages():
+    """The grouped 128-wide tiles have no staging and 7 stages, an odd ring: at
+    g = 128 both issuers then wait for and release every stage."""
+    S = min(8, BUDGET // (BM_BYTES + 128 * BK))
+    assert S == 7
+    rng = random.Random(7)
+    for _ in range(80):
+        K = rng.choice([BK, 3 * BK, 9 * BK + 64, 17 * BK])
+        items = work_list(rng, 128, K)
+        errors = simulate(S, bufs(128), 128, K, items, rng)
+        assert not errors, (S, K, items, errors[0])
 
 
 @pytest.mark.parametrize("gran", [64, 128, 256])
@@ -258,23 +323,37 @@ def test_stage_counts_match_the_kernel_budget():
 
 MUTATIONS = [
     "producer_phase",   # the producer waits for the stage's current phase, not the previous one
-    "tmem_phase",       # the MMA waits for the buffer's current phase
-    "skip_tmem_wait",   # the MMA does not wait for the promotion to free the buffer
+    "tmem_phase",       # an issuer waits for the buffer's current phase
+    "skip_tmem_wait",   # an issuer does not wait for the promotion to free the buffer
     "early_release",    # the stage is released when the MMAs are issued, not when they finish
     "promo_phase",      # the promotion waits for the previous phase of tmem_full
+    "one_stage_user",   # g != 128: a stage is released by one issuer's commit, not both
+    "tail_no_release",  # g = 64: the other issuer does not release a stage the K tail left half empty
+    "issuer_by_kb",     # the issuer is picked by the K-block's parity within its work item
+    "skip_foreign_stage_wait",  # g != 128: an issuer skips the stages of the other's blocks
 ]
+
+# (tile width, MN-major Q, g) where each mistake can show: the issuer and
+# stage-sharing mistakes need g != 128, and a buffer that changes owner
+# aliases soonest with two buffers
+MUTATION_CONFIGS = {
+    "one_stage_user": ((256, False, 64), (128, False, 256)),
+    "tail_no_release": ((256, False, 64), (16, True, 64)),
+    "issuer_by_kb": ((256, False, 64),),
+    "skip_foreign_stage_wait": ((128, False, 256), (256, False, 64)),
+}
 
 
 @pytest.mark.parametrize("mutation", MUTATIONS)
 def test_model_catches_planted_protocol_mistakes(mutation):
     """Each planted mistake is caught: as a deadlock, a wait passing at the
     wrong phase, or a stage or buffer used out of turn."""
-    rng = random.Random(hash(mutation) & 0xFFFF)
-    for bnq, q_mn, gran in ((256, False, 128), (128, True, 64), (64, False, 256)):
+    rng = random.Random(sum(map(ord, mutation)))
+    for bnq, q_mn, gran in MUTATION_CONFIGS.get(mutation, ((256, False, 128), (128, True, 64), (64, False, 256))):
         S, B = stages(bnq, q_mn, bnq >= 128), bufs(bnq)
         caught = False
         for _ in range(300):
-            K = rng.choice([5 * BK, 9 * BK, 17 * BK])
+            K = rng.choice([5 * BK, 9 * BK, 17 * BK, 9 * BK + 64])
             items = work_list(rng, gran, K)
             if simulate(S, B, gran, K, items, rng, mutation):
                 caught = True
@@ -290,7 +369,7 @@ def test_model_catches_planted_protocol_mistakes(mutation):
 # and commits to both CTAs' tmem_full[b] and empty[s]. Each CTA's promotion warps
 # wait their own tmem_full[b] and arrive on the even CTA's tmem_empty[b], whose
 # phase needs both CTAs' arrivals.
-PAIR_STAGES = min(8, BUDGET // (2 * 128 * BK))   # 16 KB of A and 16 KB of B per stage: 7
+PAIR_STAGES = min(8, (BUDGET - EPI_STAGING) // (2 * 128 * BK))   # 32 KB per stage beside the staging: 6
 PAIR_BUFS = 2
 
 
