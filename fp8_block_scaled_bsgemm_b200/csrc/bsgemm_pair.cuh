@@ -73,6 +73,14 @@ __global__ void __launch_bounds__(kNumThreads, 1)
   constexpr uint32_t kTxBytes = 2 * PC::kStageBytes;  // both CTAs' loads of a stage
   static_assert(GRAN == 64 || GRAN == 128 || GRAN == 256, "granularity");
   static_assert(STAGES >= 4, "stages");
+  // Two MMA-issuing warps of the even CTA take the K-blocks in turn, under
+  // the single-CTA kernel's rules: buffers (2, even) belong to one issuer;
+  // at g = 128 with an even ring every stage belongs to one issuer, else both
+  // wait for every stage and release it (the other by a commit of no MMAs).
+  constexpr int kIssuers = 2;
+  constexpr bool kSharedStages = (GRAN != BK) || (STAGES % kIssuers != 0);
+  constexpr int kStageUsers = kSharedStages ? 2 : 1;
+  static_assert(kBufs % kIssuers == 0, "TMEM buffers split evenly between the issuers");
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -91,13 +99,13 @@ __global__ void __launch_bounds__(kNumThreads, 1)
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
       mbar_init(smem_addr(&bars->full[s]), 1);
-      mbar_init(smem_addr(&bars->empty[s]), 1);
+      mbar_init(smem_addr(&bars->empty[s]), kStageUsers);
     }
     for (int b = 0; b < kBufs; ++b) {
       mbar_init(smem_addr(&bars->tmem_full[b]), 1);
       mbar_init(smem_addr(&bars->tmem_empty[b]), 2 * kNumEpiWarps);
     }
-    mbar_init(smem_addr(&bars->mma_done), 1);
+    mbar_init(smem_addr(&bars->mma_done), kIssuers);
     bars->abort_flag = 0;
     bars->split_last = 0;
     fence_barrier_init();
@@ -164,11 +172,13 @@ __global__ void __launch_bounds__(kNumThreads, 1)
         }
       }
     }
-  } else if (warp == kMmaWarp) {
-    // ============================================================ MMA issuer (even CTA)
-    // the whole warp, converged; each tcgen05 instruction is predicated on
-    // elect.sync, so one lane (always the same) issues without divergence
+  } else if (warp == kMmaWarp || warp == kMmaWarp + 1) {
+    // ============================================================ MMA issuers (even CTA)
+    // Issuer i (warp kMmaWarp + i) takes the K-blocks x with x % 2 == i,
+    // counted over the pair's tiles; both walk every stage.  Each warp runs
+    // converged and predicates its tcgen05 instructions on elect.sync.
     if (rank == 0) {
+      const uint32_t issuer = static_cast<uint32_t>(warp - kMmaWarp);
       const uint32_t idesc = instr_desc_pair<P_MN, Q_MN>() | p.fmt_bits;
       constexpr uint64_t kPStep = P_MN ? (kMmaK * 128) >> 4 : kMmaK >> 4;
       constexpr uint64_t kQStep = Q_MN ? (kMmaK * 128) >> 4 : kMmaK >> 4;
@@ -177,58 +187,78 @@ __global__ void __launch_bounds__(kNumThreads, 1)
       const uint64_t ad0 = smem_desc_sw128(smem_addr(p_tiles), P_MN ? 128 * BK : 16);
       const uint64_t bd0 = smem_desc_sw128(smem_addr(q_tiles), Q_MN ? 128 * BK : 16);
       uint32_t s = 0, ph = 0;
-      uint32_t b = 0, bph = 0;
+      uint32_t x = 0;             // K-blocks so far
       bool ok = true;
       for (int t = cluster; t < p.num_work && ok; t += num_clusters) {
-        for (int kb = 0; kb < p.Kb; ++kb) {
+        for (int kb = 0; kb < p.Kb; ++kb, ++x) {
           // operands first (normally already there), then the TMEM buffer;
           // tmem_full is committed before the stage release
+          const uint32_t b = x % kBufs, bph = (x / kBufs) & 1;
           const uint32_t d_tmem = tmem_base + b * BNQ;
           if constexpr (GRAN >= BK) {
+            const bool mine = (x & 1) == issuer;
 #pragma unroll
             for (int j = 0; j < GRAN / BK; ++j) {
               const int k0 = kb * GRAN + j * BK;
               if (k0 >= p.K) break;
-              if (!warp_wait_all(smem_addr(&bars->full[s]), ph, p, bars, 2)) { ok = false; break; }
-              if (j == 0 && !warp_wait_all(smem_addr(&bars->tmem_empty[b]), bph ^ 1, p, bars, 3)) {
-                ok = false;
-                break;
+              if (!mine && kSharedStages) {
+                // the other issuer's stage: observe its fill and release it
+                if (!warp_wait_all(smem_addr(&bars->full[s]), ph, p, bars, 2)) { ok = false; break; }
+                mma_commit_pair_elect(smem_addr(&bars->empty[s]), kBoth);
               }
-              const uint64_t ad = ad0 + s * kPStage, bd = bd0 + s * kQStage;
-              if (k0 + BK <= p.K) {
+              if (mine) {
+                if (!warp_wait_all(smem_addr(&bars->full[s]), ph, p, bars, 2)) { ok = false; break; }
+                if (j == 0 && !warp_wait_all(smem_addr(&bars->tmem_empty[b]), bph ^ 1, p, bars, 3)) {
+                  ok = false;
+                  break;
+                }
+                const uint64_t ad = ad0 + s * kPStage, bd = bd0 + s * kQStage;
+                if (k0 + BK <= p.K) {
 #pragma unroll
-                for (int u = 0; u < BK / kMmaK; ++u)
-                  mma_f8f6f4_pair_elect(d_tmem, ad + u * kPStep, bd + u * kQStep, idesc, (j > 0 || u > 0) ? 1u : 0u);
-              } else {
-                const int nsteps = (p.K - k0 + kMmaK - 1) / kMmaK;
-                for (int u = 0; u < nsteps; ++u)
-                  mma_f8f6f4_pair_elect(d_tmem, ad + u * kPStep, bd + u * kQStep, idesc, (j > 0 || u > 0) ? 1u : 0u);
+                  for (int u = 0; u < BK / kMmaK; ++u)
+                    mma_f8f6f4_pair_elect(d_tmem, ad + u * kPStep, bd + u * kQStep, idesc,
+                                          (j > 0 || u > 0) ? 1u : 0u);
+                } else {
+                  const int nsteps = (p.K - k0 + kMmaK - 1) / kMmaK;
+                  for (int u = 0; u < nsteps; ++u)
+                    mma_f8f6f4_pair_elect(d_tmem, ad + u * kPStep, bd + u * kQStep, idesc,
+                                          (j > 0 || u > 0) ? 1u : 0u);
+                }
+                if (j == GRAN / BK - 1 || k0 + BK >= p.K) mma_commit_pair_elect(smem_addr(&bars->tmem_full[b]), kBoth);
+                mma_commit_pair_elect(smem_addr(&bars->empty[s]), kBoth);
               }
-              if (j == GRAN / BK - 1 || k0 + BK >= p.K) mma_commit_pair_elect(smem_addr(&bars->tmem_full[b]), kBoth);
-              mma_commit_pair_elect(smem_addr(&bars->empty[s]), kBoth);
               if (++s == STAGES) { s = 0; ph ^= 1; }
             }
             if (!ok) break;
           } else {
-            // GRAN == 64: a K-block is half a stage
+            // GRAN == 64: a K-block is half a stage; a stage holds blocks x
+            // and x + 1, one per issuer, and each releases it after its half;
+            // at the K tail the other issuer waits for and releases a stage
+            // that has no second half
             const int k0 = kb * GRAN;
             const int t0 = (kb & 1) * 2;
-            if (t0 == 0 && !warp_wait_all(smem_addr(&bars->full[s]), ph, p, bars, 2)) { ok = false; break; }
-            if (!warp_wait_all(smem_addr(&bars->tmem_empty[b]), bph ^ 1, p, bars, 3)) { ok = false; break; }
-            const uint64_t ad = ad0 + s * kPStage, bd = bd0 + s * kQStage;
-            const int nsteps = (p.K - k0 >= GRAN) ? 2 : (p.K - k0 + kMmaK - 1) / kMmaK;
-            for (int u = 0; u < nsteps; ++u)
-              mma_f8f6f4_pair_elect(d_tmem, ad + (t0 + u) * kPStep, bd + (t0 + u) * kQStep, idesc, u > 0 ? 1u : 0u);
-            mma_commit_pair_elect(smem_addr(&bars->tmem_full[b]), kBoth);
-            if (t0 == 2 || k0 + GRAN >= p.K) {
+            const bool last_in_stage = (t0 == 2 || k0 + GRAN >= p.K);
+            if ((x & 1) == issuer) {
+              if (!warp_wait_all(smem_addr(&bars->full[s]), ph, p, bars, 2)) { ok = false; break; }
+              if (!warp_wait_all(smem_addr(&bars->tmem_empty[b]), bph ^ 1, p, bars, 3)) { ok = false; break; }
+              const uint64_t ad = ad0 + s * kPStage, bd = bd0 + s * kQStage;
+              const int nsteps = (p.K - k0 >= GRAN) ? 2 : (p.K - k0 + kMmaK - 1) / kMmaK;
+              for (int u = 0; u < nsteps; ++u)
+                mma_f8f6f4_pair_elect(d_tmem, ad + (t0 + u) * kPStep, bd + (t0 + u) * kQStep, idesc,
+                                      u > 0 ? 1u : 0u);
+              mma_commit_pair_elect(smem_addr(&bars->tmem_full[b]), kBoth);
               mma_commit_pair_elect(smem_addr(&bars->empty[s]), kBoth);
+            } else if (t0 == 0 && last_in_stage) {
+              if (!warp_wait_all(smem_addr(&bars->full[s]), ph, p, bars, 2)) { ok = false; break; }
+              mma_commit_pair_elect(smem_addr(&bars->empty[s]), kBoth);
+            }
+            if (last_in_stage) {
               if (++s == STAGES) { s = 0; ph ^= 1; }
             }
           }
-          if (++b == kBufs) { b = 0; bph ^= 1; }
         }
       }
-      // every pair MMA the elected lane issued completes before TMEM is freed
+      // every pair MMA both issuers issued completes before TMEM is freed
       mma_commit_pair_elect(smem_addr(&bars->mma_done), 0x1);
       warp_wait_all(smem_addr(&bars->mma_done), 0, p, bars, 8, true);
     }

@@ -365,10 +365,11 @@ def test_model_catches_planted_protocol_mistakes(mutation):
 # ``csrc/bsgemm_pair.cuh``: both CTAs' producers wait their own empty[s] and
 # load their halves of stage s; both copies complete on the even CTA's full[s],
 # whose phase also needs the even producer's arrive (with the byte count). The
-# even CTA's MMA warp waits full[s] and its tmem_empty[b], issues the pair MMAs
-# and commits to both CTAs' tmem_full[b] and empty[s]. Each CTA's promotion warps
-# wait their own tmem_full[b] and arrive on the even CTA's tmem_empty[b], whose
-# phase needs both CTAs' arrivals.
+# even CTA's two MMA issuers follow the single-CTA kernel's rules (issuer x % 2
+# takes K-block x; stages shared where they change hands) and commit to both
+# CTAs' tmem_full[b] and empty[s]. Each CTA's promotion warps wait their own
+# tmem_full[b] and arrive on the even CTA's tmem_empty[b], whose phase needs
+# both CTAs' arrivals.
 PAIR_STAGES = min(8, (BUDGET - EPI_STAGING) // (2 * 128 * BK))   # 32 KB per stage beside the staging: 6
 PAIR_BUFS = 2
 
@@ -402,80 +403,78 @@ def simulate_pair(gran, K, tiles, rng, mutation=None):
         if bar.c != k + 1:
             errors.append(f"{what}: waited for phase {k}, count was {bar.c}")
 
-    nst = -(-K // BK)
     Kb = -(-K // gran)
     items = [(0, Kb)] * tiles
+    nslots, steps, nblocks = programs(gran, K, items, S)
+    shared = gran != BK or S % 2 == 1
     full = [PhaseBar({"arrive", "land0", "land1"}) for _ in range(S)]
-    empty = [[Bar() for _ in range(S)] for _ in range(2)]
+    empty = [[CountBar(2 if shared else 1) for _ in range(S)] for _ in range(2)]
     tfull = [[Bar() for _ in range(B)] for _ in range(2)]
     tempty = [PhaseBar({0, 1} if mutation != "tmem_empty_one_cta" else {0}) for _ in range(B)]
-    mma = []
-    for kb0, kb1 in items:
-        for kb in range(kb0, kb1):
-            if gran >= BK:
-                for j in range(gran // BK):
-                    k0 = kb * gran + j * BK
-                    if k0 >= K:
-                        break
-                    mma.append((True, j == 0, j == gran // BK - 1 or k0 + BK >= K, True))
-            else:
-                k0 = kb * gran
-                mma.append(((kb & 1) == 0, True, True, (kb & 1) == 1 or k0 + gran >= K))
-    nprod = nst * tiles
-    nblocks = Kb * tiles
+    readers = [0] * nslots
+    for prog in steps:
+        for st in prog:
+            if st[3]:
+                readers[st[0]] += 1
+    reads_done = [0] * nslots
 
     p_it = [0, 0]
     landing = []
     landed = [set(), set()]
-    m_i = m_st = m_blk = m_sub = 0
-    inflight = []
+    m_i = [0, 0]
+    m_sub = [0, 0]
+    inflight = ([], [])
     promo = [0, 0]
-    reading = [0] * S
-    stage_done = 0
-    blocks_done = 0
-    slow = {r for r in ("prod0", "prod1", "land", "mma", "m_done", "promo0", "promo1") if rng.random() < 0.3}
+    blocks_done = set()
+    slow = {r for r in ("prod0", "prod1", "land", "mma0", "mma1", "done0", "done1", "promo0", "promo1")
+            if rng.random() < 0.3}
+
+    def running():
+        return (min(promo) < nblocks or p_it != [nslots, nslots] or landing or inflight[0] or inflight[1]
+                or m_i != [len(steps[0]), len(steps[1])])
+
     guard = 0
-    while min(promo) < nblocks and not errors:
+    while running() and not errors:
         guard += 1
         if guard > 400000:
             errors.append("no progress")
             break
         acts = []
         for r in (0, 1):
-            if p_it[r] < nprod:
+            if p_it[r] < nslots:
                 it = p_it[r]
                 k = it // S - 1
                 if k < 0 or (r == 1 and mutation == "odd_skips_stage_wait") or empty[r][it % S].passes(k):
                     acts.append(("prod", r))
         if landing:
             acts.append(("land",))
-        if m_i < len(mma):
-            wf, wt, _, _ = mma[m_i]
-            if m_sub == 0 and wf:
-                if full[m_st % S].passes(m_st // S):
-                    acts.append(("m_full",))
-            else:
-                b, k = m_blk % B, m_blk // B - 1
-                if not wt or k < 0 or tempty[b].passes(k):
-                    acts.append(("m_issue",))
-        if inflight:
-            acts.append(("m_done",))
+        for i in (0, 1):
+            if m_i[i] < len(steps[i]):
+                slot, wf, wb, _, _, _ = steps[i][m_i[i]]
+                if m_sub[i] == 0 and wf:
+                    if full[slot % S].passes(slot // S):
+                        acts.append(("m_full", i))
+                elif wb is None or wb // B - 1 < 0 or tempty[wb % B].passes(wb // B - 1):
+                    acts.append(("m_issue", i))
+            if inflight[i]:
+                acts.append(("m_done", i))
         for r in (0, 1):
             if promo[r] < nblocks and tfull[r][promo[r] % B].passes(promo[r] // B):
                 acts.append(("promo", r))
         if not acts:
-            errors.append(f"deadlock: producers {p_it}/{nprod}, mma {m_i}/{len(mma)}, promotion {promo}")
+            errors.append(f"deadlock: producers {p_it}/{nslots}, issuers {m_i}, promotion {promo}")
             break
 
         def role(a):
-            return {"prod": f"prod{a[1] if len(a) > 1 else ''}", "promo": f"promo{a[1] if len(a) > 1 else ''}",
-                    "m_full": "mma", "m_issue": "mma"}.get(a[0], a[0])
+            return {"prod": f"prod{a[-1]}", "promo": f"promo{a[-1]}", "m_full": f"mma{a[-1]}",
+                    "m_issue": f"mma{a[-1]}", "m_done": f"done{a[-1]}"}.get(a[0], a[0])
         a = rng.choices(acts, [0.03 if role(x) in slow else 1.0 for x in acts])[0]
         if a[0] == "prod":
             r = a[1]
             it = p_it[r]
-            if (reading[it % S] or stage_done < it - S + 1):
-                errors.append(f"producer {r} slot {it}: stage {it % S} overwritten while in use")
+            old = it - S
+            if old >= 0 and reads_done[old] < readers[old]:
+                errors.append(f"producer {r} slot {it}: stage {it % S} overwritten while slot {old} is read")
             if r == 0:
                 full[it % S].add("arrive", it // S, errors, f"even producer slot {it}")
             landing.append((r, it))
@@ -485,54 +484,51 @@ def simulate_pair(gran, K, tiles, rng, mutation=None):
             landed[r].add(it)
             full[it % S].add(f"land{r}", it // S, errors, f"copy of CTA {r} slot {it}")
         elif a[0] == "m_full":
-            check(full[m_st % S], m_st // S, f"mma step {m_i} (full)")
-            m_sub = 1
+            i = a[1]
+            slot = steps[i][m_i[i]][0]
+            check(full[slot % S], slot // S, f"issuer {i} step {m_i[i]} (full)")
+            m_sub[i] = 1
         elif a[0] == "m_issue":
-            wf, wt, ctf, cem = mma[m_i]
-            if wt and m_blk // B - 1 >= 0:
-                check(tempty[m_blk % B], m_blk // B - 1, f"mma step {m_i} (tmem_empty)")
-            if m_st not in landed[0] or m_st not in landed[1]:
-                errors.append(f"mma step {m_i}: stage slot {m_st} read before both copies landed")
-            if wt and min(promo) < m_blk - B + 1:
-                errors.append(f"mma step {m_i}: buffer {m_blk % B} rewritten before block "
-                              f"{m_blk - B} was promoted in both CTAs")
-            reading[m_st % S] += 1
-            if mutation == "early_release" and cem:
+            i = a[1]
+            slot, wf, wb, mma, cb, cs = steps[i][m_i[i]]
+            if wb is not None:
+                if wb // B - 1 >= 0:
+                    check(tempty[wb % B], wb // B - 1, f"issuer {i} step {m_i[i]} (tmem_empty)")
+                if min(promo) < wb - B + 1:
+                    errors.append(f"issuer {i}: buffer {wb % B} rewritten before block {wb - B} "
+                                  f"was promoted in both CTAs")
+            if mma and (slot not in landed[0] or slot not in landed[1]):
+                errors.append(f"issuer {i}: stage slot {slot} read before both copies landed")
+            if mutation == "early_release" and cs is not None and mma:
                 for r in (0, 1):
-                    empty[r][m_st % S].c += 1
-                stage_done += 1
-                cem = False
-            inflight.append((m_blk % B if ctf else None, m_st % S if cem else None, m_st % S))
-            if ctf:
-                m_blk += 1
-            if mma[m_i][3]:
-                m_st += 1
-            m_i += 1
-            m_sub = 0
+                    empty[r][cs % S].add(cs // S, errors, f"issuer {i} early release, slot {cs}")
+                cs = None
+            inflight[i].append((slot if mma else None, cb, cs))
+            m_i[i] += 1
+            m_sub[i] = 0
         elif a[0] == "m_done":
-            tb, es, rs = inflight.pop(0)
-            reading[rs] -= 1
-            if tb is not None:
+            i = a[1]
+            rs, cb, cs = inflight[i].pop(0)
+            if rs is not None:
+                reads_done[rs] += 1
+            if cb is not None:
                 for r in ((0,) if mutation == "tmem_full_even_only" else (0, 1)):
-                    tfull[r][tb].c += 1
-                blocks_done += 1
-            if es is not None:
+                    tfull[r][cb % B].c += 1
+                blocks_done.add(cb)
+            if cs is not None:
                 for r in (0, 1):
-                    empty[r][es].c += 1
-                stage_done += 1
+                    empty[r][cs % S].add(cs // S, errors, f"issuer {i} commit to CTA {r}, slot {cs}")
         else:
             r = a[1]
             blk = promo[r]
             check(tfull[r][blk % B], blk // B, f"promotion of CTA {r}, block {blk}")
-            if blocks_done < blk + 1:
+            if blk not in blocks_done:
                 errors.append(f"promotion of CTA {r}, block {blk}: read an unfinished partial")
             if mutation == "tmem_empty_one_cta" and r == 1:
                 pass            # the planted mistake: the odd CTA's arrival is not counted
             else:
                 tempty[blk % B].add(r, blk // B, errors, f"promotion of CTA {r}, block {blk}")
             promo[r] += 1
-    if not errors and (m_i != len(mma) or p_it != [nprod, nprod]):
-        errors.append("roles finished out of step")
     return errors
 
 
