@@ -706,6 +706,27 @@ __global__ void __launch_bounds__(kNumThreads, 1)
         work_begin<SPLIT, GROUPED>(p, wit);
         more = work_next<GRAN, SPLIT, GROUPED>(p, wit, w);
       } else {
+        // While the previous grid finishes, pull the first ring's worth of
+        // this CTA's operand tiles towards L2.  A prefetch returns nothing to
+        // the program and L2 is coherent, so the loads after the wait still
+        // read what the previous grid wrote; they find the bytes nearer.
+        if (more) {
+          int st0, st1;
+          stage_range<GRAN>(p, w, st0, st1);
+          const int stop = st1 < st0 + STAGES ? st1 : st0 + STAGES;
+          const int prow = w.tp * BM, qrow = w.tq * BNQ;
+          for (int st = st0; st < stop; ++st) {
+            const int k = st * BK;
+            if constexpr (P_MN) tma_prefetch_l2_2d(&tm_p, prow, k);
+            else                tma_prefetch_l2_2d(&tm_p, k, prow);
+            if constexpr (Q_MN) {
+#pragma unroll
+              for (int c = 0; c < TL::kQRows / 128; ++c) tma_prefetch_l2_2d(&tm_q, qrow + c * 128, k);
+            } else {
+              tma_prefetch_l2_2d(&tm_q, k, qrow);
+            }
+          }
+        }
         grid_dependency_wait();
       }
       for (; ok && more; more = work_next<GRAN, SPLIT, GROUPED>(p, wit, w)) {

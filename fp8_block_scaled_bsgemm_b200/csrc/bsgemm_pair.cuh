@@ -124,7 +124,24 @@ __global__ void __launch_bounds__(kNumThreads, 1)
   tc_fence_after();
   const uint32_t tmem_base = bars->tmem_base;
   // global memory is touched only after the grids this one depends on are
-  // complete (programmatic dependent launch; see bsgemm_kernel)
+  // complete (programmatic dependent launch; see bsgemm_kernel); before
+  // that, the producers pull their first tile's first stages towards L2
+  // (a prefetch returns nothing, and L2 is coherent)
+  if (warp == kProducerWarp && lane == 0 && cluster < p.num_work) {
+    int tp, tq;
+    tile_coords(p, cluster, tp, tq);
+    const int prow = tp * kPairM + static_cast<int>(rank) * BM;
+    const int qrow = tq * kPairN + static_cast<int>(rank) * kPairQRows;
+    const int nst = (p.K + BK - 1) / BK;
+    const int stop = nst < STAGES ? nst : STAGES;
+    for (int st = 0; st < stop; ++st) {
+      const int k = st * BK;
+      if constexpr (P_MN) tma_prefetch_l2_2d(&tm_p, prow, k);
+      else                tma_prefetch_l2_2d(&tm_p, k, prow);
+      if constexpr (Q_MN) tma_prefetch_l2_2d(&tm_q, qrow, k);
+      else                tma_prefetch_l2_2d(&tm_q, k, qrow);
+    }
+  }
   grid_dependency_wait();
   if (threadIdx.x == 0) grid_launch_dependents();
 
