@@ -139,6 +139,7 @@ struct __align__(8) Barriers {
   uint64_t tmem_full[8];
   uint64_t tmem_empty[8];
   uint64_t mma_done;
+  uint64_t publish;      // stream-K: the promotion warps' partial is written
   uint32_t tmem_base;
   int abort_flag;
   int split_last;
@@ -649,6 +650,7 @@ __global__ void __launch_bounds__(kNumThreads, 1)
       mbar_init(smem_addr(&bars->tmem_empty[b]), kNumEpiWarps);
     }
     mbar_init(smem_addr(&bars->mma_done), kIssuers);
+    mbar_init(smem_addr(&bars->publish), kNumEpiWarps);
     bars->abort_flag = 0;
     bars->split_last = 0;
     fence_barrier_init();
@@ -874,6 +876,31 @@ __global__ void __launch_bounds__(kNumThreads, 1)
       mma_commit_elect(smem_addr(&bars->mma_done));
       warp_wait_all(smem_addr(&bars->mma_done), 0, p, bars, 8, true);
     }
+  } else if (warp == 3) {
+    // ============================================================ stream-K publisher
+    // A CTA's stream-K range holds at most one piece that is not its tile's
+    // reducer: the range's first segment, when it starts inside a tile.  The
+    // promotion warps write that piece's partial, arrive on `publish`
+    // (release, CTA scope) and go straight on to their next item; this warp
+    // waits for them (acquire) and makes the partial visible to the
+    // reducer with one release add on the tile's counter (GPU scope), so the
+    // promotion warps never wait for that release to complete.
+    if constexpr (SPLIT) {
+      if (p.sk_ctas > 0) {
+        grid_dependency_wait();
+        WorkIter wit;
+        work_begin<SPLIT, GROUPED>(p, wit);
+        for (Work w; work_next<GRAN, SPLIT, GROUPED>(p, wit, w);) {
+          if (w.tile < p.sk_first_tile || w.kb0 == 0) continue;   // whole tile, or the reducer
+          const Pieces pq = pieces_of<GRAN>(p, w);
+          if (pq.pieces <= 1) continue;
+          if (!warp_wait_all(smem_addr(&bars->publish), 0, p, bars, 6)) break;
+          if (lane == 0) red_add_release_gpu(p.counters + pq.counter, 1);
+          __syncwarp();
+          break;
+        }
+      }
+    }
   }
   } else {
     // ============================================================ promotion + epilogue
@@ -1012,22 +1039,23 @@ __global__ void __launch_bounds__(kNumThreads, 1)
 #pragma unroll
             for (int c = 0; c < kHalf / 4; ++c)
               __stcg(my_ws + c * BM, make_float4(acc[2 * c].x, acc[2 * c].y, acc[2 * c + 1].x, acc[2 * c + 1].y));
-            // The partial now lives in the workspace; acc is dead until the
-            // sum below.  Publishing it takes one release: every promotion
-            // thread's stores come before the CTA barrier, the barrier before
-            // the leader's release add on the tile counter (GPU scope).  A
-            // split-K leader's add also acquires the earlier pieces (acq_rel)
-            // and tells whether this piece arrived last.
-            named_barrier_sync(1, kNumEpiThreads);
-            if (ew == 0 && lane == 0) {
-              int is_last = 0;
-              if (p.sk_ctas > 0 && w.tile >= p.sk_first_tile) {
-                red_add_release_gpu(p.counters + pcs.counter, 1);
-              } else {
-                is_last = atom_add_acq_rel_gpu(p.counters + pcs.counter, 1) == pcs.pieces - 1;
-              }
-              bars->split_last = is_last;
+            if (p.sk_ctas > 0 && w.tile >= p.sk_first_tile) {
+              // stream-K: the publisher warp releases the partial; this
+              // warp's stores come before its lane 0's arrive (the warp
+              // barrier orders them, the arrive is a CTA-scope release)
+              __syncwarp();
+              if (lane == 0) mbar_arrive(smem_addr(&bars->publish));
+              continue;
             }
+            // Split-K: the partial now lives in the workspace; acc is dead
+            // until the sum below.  Publishing it takes one release: every
+            // promotion thread's stores come before the CTA barrier, the
+            // barrier before the leader's acq_rel add on the tile counter
+            // (GPU scope), which also acquires the earlier pieces and tells
+            // whether this piece arrived last.
+            named_barrier_sync(1, kNumEpiThreads);
+            if (ew == 0 && lane == 0)
+              bars->split_last = atom_add_acq_rel_gpu(p.counters + pcs.counter, 1) == pcs.pieces - 1;
             named_barrier_sync(1, kNumEpiThreads);
             const bool last = *reinterpret_cast<volatile int*>(&bars->split_last) != 0;
             // nobody may overwrite split_last before every thread has read it
