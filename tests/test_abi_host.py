@@ -38,7 +38,7 @@ def test_status_strings_and_version():
 
 
 @pytest.mark.parametrize("M,N,K,gran,want_swap", [
-    (4096, 4096, 4096, 128, 0), (1, 7168, 7168, 128, 1), (128, 7168, 7168, 128, 1),
+    (4096, 4096, 4096, 128, 0), (1, 7168, 7168, 128, 1), (64, 7168, 7168, 128, 1), (128, 7168, 7168, 128, 0),
     (8192, 14336, 4096, 128, 0), (2048, 4096, 32768, 64, 0), (7, 1000, 656, 256, 1)])
 def test_plan_is_consistent(M, N, K, gran, want_swap):
     pl = bsg.make_plan(M, N, K, gran, "nt", 148)
@@ -402,3 +402,13 @@ def test_raster_maps_work_items_onto_the_tile_grid_one_to_one(group_p):
             (a0, b0), (a1, b1) = seen[t], seen[t + 1]
             if t // per_group == (t + 1) // per_group and a1 == a0 + 1:
                 assert b1 == b0              # next row of the same group: same B column
+
+
+@pytest.mark.parametrize("M,N,K,want_bnq", [
+    (4096, 4096, 4096, 256), (8192, 14336, 4096, 256),      # many tiles: 256 wide
+    (128, 7168, 7168, 128), (256, 4096, 7168, 128),          # few tiles, 128-wide ones fit one wave
+    (384, 7168, 7168, 256), (512, 7168, 7168, 256),          # 128-wide tiles would spill past a wave
+    (96, 100, 4096, 128)])                                    # N <= 128
+def test_data_parallel_width(M, N, K, want_bnq):
+    pl = bsg.make_plan(M, N, K, 128, "nt", 148, {"variant": "data_parallel"})
+    assert pl["bnq"] == want_bnq, pl

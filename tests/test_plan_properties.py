@@ -24,7 +24,7 @@ def expected_refusal(M, t, num_sms):
     if v == "cta_pair":
         return (bnq not in (0, 256)) or splits > 1 or sk > 0 or num_sms < 2
     if v == "auto":
-        v = "swap_ab" if M <= 128 else "data_parallel"   # a tuned plan never pairs automatically
+        v = "swap_ab" if M <= 64 else "data_parallel"   # a tuned plan never pairs automatically
     if v == "swap_ab":
         return bnq not in (0, 16, 32, 64, 128)
     return bnq not in (0, 128, 256)
