@@ -279,14 +279,23 @@ extern "C" bsgemm_status bsgemm_make_plan(int layout, int64_t M, int64_t N, int6
   int bnq = t ? t->bnq : 0;
   if (bnq == 0 && pl.swap_ab) bnq = pow2_at_least(static_cast<int>(Q < 128 ? Q : 128), 16);
   if (bnq == 0) {
-    // Data-parallel width: 256, except where 256-wide tiles are fewer than
-    // the SMs and 128-wide ones still fit in one wave -- there the narrower
-    // tiles halve each stream-K piece and the fix-up and measured 10-25 %
-    // faster (M = 128..256 with N = 4096..7168; same box).  With more 128-wide
-    // tiles than SMs, 256 stayed ahead (M = 320..512, N = 7168).
+    // Data-parallel width: 256, except
+    // - where 256-wide tiles are fewer than the SMs and 128-wide ones still
+    //   fit in one wave: the narrower tiles halve each stream-K piece and the
+    //   fix-up, measured 10-25 % faster (M = 128..256, N = 4096..7168; with
+    //   more 128-wide tiles than SMs 256 stayed ahead: M = 320..512);
+    // - with whole tiles (short K, no stream-K) where 128-wide tiles waste
+    //   less of the last wave: a 128-wide tile takes 0.62 of a 256-wide one
+    //   (the square workload: 7 waves of 128 against 4 of 256), and 2 waves
+    //   of 256 against 3 of 128 measured 2.5-9 % faster at 128 (seven shapes,
+    //   M = 384..2048).  Measured at g = 128 only, so applied there.
     const int64_t tp = (P + bsg::BM - 1) / bsg::BM;
     const int64_t t256 = tp * ((Q + 255) / 256), t128 = tp * ((Q + 127) / 128);
-    bnq = (Q <= 128 || (t256 < num_sms && t128 <= num_sms)) ? 128 : 256;
+    const int64_t w256 = (t256 + num_sms - 1) / num_sms, w128 = (t128 + num_sms - 1) / num_sms;
+    const bool whole = gran == 128 && static_cast<int64_t>(Kb) * gran < 64 * 128;   // no stream-K at 256
+    if (Q <= 128 || (t256 < num_sms && t128 <= num_sms)) bnq = 128;
+    else if (t256 >= num_sms && whole && 0.62 * static_cast<double>(w128) < 0.97 * static_cast<double>(w256)) bnq = 128;
+    else bnq = 256;
   }
   if (pl.swap_ab ? (bnq != 16 && bnq != 32 && bnq != 64 && bnq != 128) : (bnq != 128 && bnq != 256))
     return BSGEMM_ERR_INVALID_ARG;

@@ -408,6 +408,8 @@ def test_raster_maps_work_items_onto_the_tile_grid_one_to_one(group_p):
     (4096, 4096, 4096, 256), (8192, 14336, 4096, 256),      # many tiles: 256 wide
     (128, 7168, 7168, 128), (256, 4096, 7168, 128),          # few tiles, 128-wide ones fit one wave
     (384, 7168, 7168, 256), (512, 7168, 7168, 256),          # 128-wide tiles would spill past a wave
+    (768, 7168, 7168, 128), (1280, 4096, 2048, 128),         # whole tiles: 3 waves of 128 beat 2 of 256
+    (2048, 4096, 32768, 256),                                 # long K: stream-K evens the waves at 256
     (96, 100, 4096, 128)])                                    # N <= 128
 def test_data_parallel_width(M, N, K, want_bnq):
     pl = bsg.make_plan(M, N, K, 128, "nt", 148, {"variant": "data_parallel"})
