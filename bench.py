@@ -114,18 +114,39 @@ def algorithmic_bytes(p: workloads.Problem) -> int:
 KERNEL_FILES = ("bsgemm_kernel.cuh", "bsgemm_pair.cuh", "ptx.cuh")  # the device code
 
 
+def _code_only(text: str) -> str:
+    """C++ source without comments and blank lines (string literals kept as they are)."""
+    import re
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    out = []
+    for line in text.splitlines():
+        i, quoted = 0, False
+        while i < len(line):
+            c = line[i]
+            if c == '"' and (i == 0 or line[i - 1] != "\\"):
+                quoted = not quoted
+            elif not quoted and line.startswith("//", i):
+                line = line[:i]
+                break
+            i += 1
+        line = line.rstrip()
+        if line:
+            out.append(line)
+    return "\n".join(out)
+
+
 def kernel_source_hash() -> str:
     """Short hash of the device code of the GEMM kernels (ties ncu figures to a kernel version).
 
-    Host-side launch code (argument checks, caching of launch attributes)
-    does not change what a captured kernel did, so it is not part of it."""
+    Comments are left out, and so is host-side launch code (argument checks,
+    caching of launch attributes): neither changes what a captured kernel did."""
     import hashlib
     h = hashlib.sha256()
     for f in KERNEL_FILES:
         path = os.path.join(ROOT, "fp8_block_scaled_bsgemm_b200", "csrc", f)
         h.update(f.encode())
-        with open(path, "rb") as fh:
-            h.update(fh.read())
+        with open(path, encoding="utf-8") as fh:
+            h.update(_code_only(fh.read()).encode())
     return h.hexdigest()[:16]
 
 

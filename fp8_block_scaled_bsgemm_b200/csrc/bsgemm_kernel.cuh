@@ -14,10 +14,12 @@
 // One persistent CTA per SM, 12 warps (3 warpgroups):
 //   warp 0   TMA producer: P and Q tiles of 128 K-bytes into a STAGES-deep
 //            ring of 128B-swizzled shared-memory buffers (mbarrier full/empty);
-//   warp 1   TMEM owner and MMA issuer: for each K-block, tcgen05.mma
-//            (kind::f8f6f4, K = 32 per instruction) into one of 2..8 TMEM
-//            partial buffers, then tcgen05.commit to tell the promoters;
-//   warps 2-3 idle (they complete the first warpgroup);
+//   warps 1-2 MMA issuers (warp 1 also owns TMEM), taking the K-blocks in
+//            turn: tcgen05.mma (kind::f8f6f4, K = 32 per instruction) into
+//            one of 2..8 TMEM partial buffers, then tcgen05.commit to tell
+//            the promoters;
+//   warp 3   stream-K publisher: releases the CTA's one partial that another
+//            CTA reduces (idle otherwise);
 //   warps 4-11 promotion + epilogue: tcgen05.ld each K-block's partial,
 //            acc += (sP*sQ) * partial in FP32 registers (packed f32x2 FMAs),
 //            release the TMEM buffer, and at the end of a tile round to BF16
@@ -30,9 +32,10 @@
 //     K-blocks, laid end to end, are cut into equal contiguous ranges, one
 //     per CTA, so no SM idles in a ragged last wave.
 // A piece that is not a whole tile writes its FP32 partial tile to a
-// workspace slot; the last piece of a tile to arrive (per-tile counter) adds
-// all the tile's partials in K order -- the same order every run -- and
-// stores the BF16 tile.
+// workspace slot and arrives on a per-tile counter; the tile's reducer (for
+// split-K the last piece to arrive, for stream-K the piece that starts the
+// tile, which keeps its own partial in registers) adds all the tile's
+// partials in K order -- the same order every run -- and stores the BF16 tile.
 //
 // Every mbarrier wait is bounded by a %globaltimer deadline.  When one runs
 // out the kernel records BSGEMM_ERR_DEVICE_TIMEOUT in the status word, raises
@@ -685,12 +688,13 @@ __global__ void __launch_bounds__(kNumThreads, 1)
   // memory, so they may overlap the previous grid's last CTAs.  The producer
   // and the promotion warps -- the only roles that read or write global
   // memory (operands, scales, workspace, output) -- wait for that grid
-  // (grid_dependency_wait) first; the MMA warp touches only shared memory and
-  // TMEM.  The next grid may start its own set-up as soon as SMs free up.
+  // (grid_dependency_wait) first, and so does the stream-K publisher; the MMA
+  // issuers touch only shared memory and TMEM.  The next grid may start its
+  // own set-up as soon as SMs free up.
   if (threadIdx.x == 0) grid_launch_dependents();
 
   if (warp < kFirstEpiWarp) {
-    // warpgroup 0: producer, MMA issuer and two idle warps
+    // warpgroup 0: producer, two MMA issuers and the stream-K publisher
     if constexpr (RegSplit<BNQ>::kEnabled) set_max_regs_dec<kProducerRegs>();
   if (warp == kProducerWarp) {
     // ============================================================ TMA producer

@@ -19,8 +19,8 @@
 // Synchronisation (all mbarrier waits bounded, as in bsgemm_kernel):
 //   full[s]        even CTA only: the even CTA's producer expects both CTAs'
 //                  bytes; both producers' TMA loads complete on it;
-//   empty[s]       both CTAs: the MMA thread's commit arrives on both;
-//   tmem_full[b]   both CTAs: the MMA thread's commit arrives on both;
+//   empty[s]       both CTAs: the issuers' commits arrive on both;
+//   tmem_full[b]   both CTAs: the issuing thread's commit arrives on both;
 //   tmem_empty[b]  even CTA only: 16 arrivals, 8 promotion warps per CTA
 //                  (the odd CTA's arrive across the cluster);
 //   mma_done       even CTA only.

@@ -45,9 +45,14 @@ def test_traffic_is_reported_only_for_the_profiled_kernel_sources(fake_root):
     assert bench.profiled_traffic("square") == 34286848
     assert bench.profiled_traffic("ffn") is None            # taken on other sources
     assert bench.profiled_traffic("long_k:128") is None     # never profiled
-    # any change to the device code unties the figure
-    with open(os.path.join(fake_root, "fp8_block_scaled_bsgemm_b200", "csrc", "ptx.cuh"), "a") as f:
-        f.write("\n// edited\n")
+    # a comment does not change the device code, and keeps the figure
+    ptx = os.path.join(fake_root, "fp8_block_scaled_bsgemm_b200", "csrc", "ptx.cuh")
+    with open(ptx, "a") as f:
+        f.write("\n// edited\n/* a note\n   over two lines */\n")
+    assert bench.kernel_source_hash() == sha
+    # any change to the code itself unties it
+    with open(ptx, "a") as f:
+        f.write("\nnamespace bsg { constexpr int kEdited = 1; }\n")
     assert bench.kernel_source_hash() != sha
     assert bench.profiled_traffic("square") is None
 
