@@ -47,6 +47,28 @@ def test_quantiser_bf16_bit_exact(fmt, g):
     assert np.array_equal(q.cpu().numpy(), q_ref)
 
 
+@pytest.mark.parametrize("src", ["fp32", "bf16"])
+@pytest.mark.parametrize("g", [64, 128, 256])
+def test_quantiser_large_ragged(src, g):
+    """A large matrix: more blocks than the GPU holds CTAs at once (over eight
+    per SM), so blocks run in several waves. The last row block and the last
+    column block are ragged: 8208 columns leave a 16-column last block."""
+    rows, cols = (9300 if g == 256 else 6100), 8208
+    n_sms = torch.cuda.get_device_properties(0).multi_processor_count
+    assert (-(-rows // g)) * (-(-cols // g)) > 8 * n_sms
+    x32 = _source(rows, cols, 31 + g, scale=2.0)
+    if src == "bf16":
+        xt = torch.from_numpy(x32).to(torch.bfloat16)
+        x_ref = xt.float().numpy()                  # BF16 -> FP32 is exact
+    else:
+        xt = torch.from_numpy(x32)
+        x_ref = x32
+    q, s = bsg.quantize(xt.cuda(), g, "e4m3")
+    q_ref, s_ref = oracle.quantize_blocks(x_ref, g, "e4m3")
+    assert np.array_equal(s.cpu().numpy(), s_ref)
+    assert np.array_equal(q.cpu().numpy(), q_ref)
+
+
 def test_quantise_then_gemm_matches_oracle_pipeline():
     """Online activations: quantise A and B on the GPU, multiply on the GPU;
     the same steps in the oracle give the reference."""
