@@ -23,6 +23,7 @@
 #include <cuda_runtime.h>
 
 #include <cstdint>
+#include <type_traits>
 
 #include "bsgemm.h"
 
@@ -84,8 +85,41 @@ __device__ __forceinline__ uint32_t encode(float v) {
       __nv_cvt_float_to_fp8(v, __NV_SATFINITE, FMT == BSGEMM_FP8_E5M2 ? __NV_E5M2 : __NV_E4M3));
 }
 
+// x / s, correctly rounded in FP32.
+//
+// FAST = false: the division itself.
+// FAST = true: Markstein's correction step for division. From the correctly
+// rounded reciprocal rs = RN(1/s), take q0 = RN(x * rs), form the residual
+// x - q0 * s exactly with one fma, and correct q0 by residual * rs with a second
+// fma. The quotient's sign is copied from x, so -0 stays -0.
+//
+// The fast form is used only for BF16 input and only for s >= kFastMinScale.
+// There the residual is exact wherever the FP8 code depends on it.
+// tests/quant_division_model.c runs the same steps for every BF16 block amax
+// (s = RN(amax / FMAX)) and every BF16 x with |x| <= amax, for E4M3 and E5M2,
+// about 1.9e9 pairs. Where |x / s| >= 2^-18, q equals RN(x / s) bit for bit.
+// Below that, both are under 2^-17 with the same sign, so both give the code
+// +-0. FP32 input is not covered by that enumeration and keeps the division.
+constexpr float kFastMinScale = 0x1p-60f;
+
+template <bool FAST>
+__device__ __forceinline__ float quotient(float x, float s, float rs) {
+  if constexpr (FAST) {
+    const float q0 = __fmul_rn(x, rs);
+    return copysignf(__fmaf_rn(__fmaf_rn(-q0, s, x), rs, q0), x);
+  } else {
+    return __fdiv_rn(x, s);
+  }
+}
+
+// CTAs per SM each instance's registers are held to: g = 128 keeps its runs
+// in registers (BF16 at 64 registers, 4 CTAs; FP32 at 96, 2 CTAs); g = 64
+// runs 8 (BF16) or 6 (FP32), and g = 256 (which reads the block twice) 5.
+template <int G, bool BF16_IN>
+constexpr int kMinCtasPerSm = G == 128 ? (BF16_IN ? 4 : 2) : G == 64 ? (BF16_IN ? 8 : 6) : 5;
+
 template <int G, bool BF16_IN, int FMT>
-__global__ void __launch_bounds__(kThreads)
+__global__ void __launch_bounds__(kThreads, (kMinCtasPerSm<G, BF16_IN>))
     quant_kernel(const void* __restrict__ x, int64_t rows, int64_t cols, int64_t col_blocks,
                  uint8_t* __restrict__ q, float* __restrict__ scales) {
   constexpr int kRuns = G * G / kVec;   // runs of 8 columns in a full block
@@ -169,38 +203,48 @@ __global__ void __launch_bounds__(kThreads)
   __syncthreads();
   const float s = block_scale;
 
-  // ---- pass 2: encode
-  auto encode_run = [&](const float (&v)[kVec], int64_t r, int64_t c) {
-    uint32_t lo = 0, hi = 0;
+  // ---- pass 2: encode.  The quotient's form is chosen once per block.
+  auto encode_block = [&](auto fast_tag) {
+    constexpr bool kFast = decltype(fast_tag)::value;
+    const float rs = kFast ? __frcp_rn(s) : 0.f;
+    auto encode_run = [&](const float (&v)[kVec], int64_t r, int64_t c) {
+      uint32_t lo = 0, hi = 0;
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      lo |= encode<FMT>(__fdiv_rn(v[i], s)) << (8 * i);
-      hi |= encode<FMT>(__fdiv_rn(v[4 + i], s)) << (8 * i);
+      for (int i = 0; i < 4; ++i) {
+        lo |= encode<FMT>(quotient<kFast>(v[i], s, rs)) << (8 * i);
+        hi |= encode<FMT>(quotient<kFast>(v[4 + i], s, rs)) << (8 * i);
+      }
+      *reinterpret_cast<uint2*>(q + r * cols + c) = make_uint2(lo, hi);
+    };
+    if constexpr (kHeld > 0) {
+#pragma unroll
+      for (int j = 0; j < kHeld; ++j) {
+        const int run = threadIdx.x + j * kThreads;
+        const int64_t r = r0 + run / kRunsPerRow;
+        const int64_t c = c0 + (run % kRunsPerRow) * kVec;
+        if (r < rows && c < cols) {
+          float v[kVec];
+          widen<BF16_IN>(held[j], v);
+          encode_run(v, r, c);
+        }
+      }
+    } else {
+      for (int run = threadIdx.x; run < kRuns; run += kThreads) {
+        const int64_t r = r0 + run / kRunsPerRow;
+        const int64_t c = c0 + (run % kRunsPerRow) * kVec;
+        if (r < rows && c < cols) {
+          float v[kVec];
+          load8<BF16_IN>(x, r * cols + c, v);
+          encode_run(v, r, c);
+        }
+      }
     }
-    *reinterpret_cast<uint2*>(q + r * cols + c) = make_uint2(lo, hi);
   };
-  if constexpr (kHeld > 0) {
-#pragma unroll
-    for (int j = 0; j < kHeld; ++j) {
-      const int run = threadIdx.x + j * kThreads;
-      const int64_t r = r0 + run / kRunsPerRow;
-      const int64_t c = c0 + (run % kRunsPerRow) * kVec;
-      if (r < rows && c < cols) {
-        float v[kVec];
-        widen<BF16_IN>(held[j], v);
-        encode_run(v, r, c);
-      }
-    }
+  if constexpr (BF16_IN) {
+    if (s >= kFastMinScale) encode_block(std::true_type{});
+    else                    encode_block(std::false_type{});
   } else {
-    for (int run = threadIdx.x; run < kRuns; run += kThreads) {
-      const int64_t r = r0 + run / kRunsPerRow;
-      const int64_t c = c0 + (run % kRunsPerRow) * kVec;
-      if (r < rows && c < cols) {
-        float v[kVec];
-        load8<BF16_IN>(x, r * cols + c, v);
-        encode_run(v, r, c);
-      }
-    }
+    encode_block(std::false_type{});
   }
 }
 

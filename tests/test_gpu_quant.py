@@ -47,6 +47,44 @@ def test_quantiser_bf16_bit_exact(fmt, g):
     assert np.array_equal(q.cpu().numpy(), q_ref)
 
 
+# BF16 block maxima: denormals (their blocks keep the division), the smallest
+# normal, values around 1 and the formats' maxima, and the largest finite BF16
+AMAX_BITS = [0x0001, 0x0042, 0x0080, 0x0D00, 0x1C80, 0x2F3B, 0x3A01, 0x3F80, 0x3FC0,
+             0x41A5, 0x43E0, 0x4480, 0x4760, 0x5A5A, 0x6E11, 0x7F7F]
+
+
+def _every_bf16_up_to(amax_bits, g):
+    """Blocks of g x g BF16 values: for each amax, its value first and then
+    every BF16 bit pattern of either sign with |x| <= amax, over as many
+    blocks as that takes (each block starts with amax, so amax is its max)."""
+    per = g * g - 1
+    blocks = []
+    for ab in amax_bits:
+        mags = np.arange(0, ab + 1, dtype=np.uint32)
+        vals = np.concatenate([mags, mags | 0x8000]).astype(np.uint16)
+        for i in range(0, vals.size, per):
+            chunk = vals[i:i + per]
+            blk = np.full(g * g, ab, dtype=np.uint16)
+            blk[1:1 + chunk.size] = chunk
+            blocks.append(blk.reshape(g, g))
+    return np.concatenate(blocks, axis=0)          # [blocks * g, g]
+
+
+@pytest.mark.parametrize("fmt", ["e4m3", "e5m2"])
+@pytest.mark.parametrize("g", [64, 128])
+def test_quantiser_bf16_every_value_below_amax(fmt, g):
+    """The BF16 path's quotient (a corrected reciprocal product where the
+    block scale allows it) against the oracle's division, for every BF16 value
+    under each of several block maxima, from denormal to the largest finite."""
+    u16 = _every_bf16_up_to(AMAX_BITS, g)
+    xb = torch.from_numpy(u16.view(np.int16)).view(torch.bfloat16)
+    q, s = bsg.quantize(xb.cuda(), g, fmt)
+    q_ref, s_ref = oracle.quantize_blocks(xb.float().numpy(), g, fmt)   # BF16 -> FP32 is exact
+    assert np.array_equal(s.cpu().numpy(), s_ref)
+    got = q.cpu().numpy()
+    assert np.array_equal(got, q_ref), int(np.sum(got != q_ref))
+
+
 @pytest.mark.parametrize("src", ["fp32", "bf16"])
 @pytest.mark.parametrize("g", [64, 128, 256])
 def test_quantiser_large_ragged(src, g):
