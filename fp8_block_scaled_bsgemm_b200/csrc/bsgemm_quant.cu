@@ -29,7 +29,10 @@
 
 namespace bsgq {
 
-constexpr int kThreads = 256;
+// Threads per CTA: 512 at g = 128 from FP32 (each thread holds 4 runs), else
+// 256 (8 runs held at g = 128 from BF16).
+template <int G, bool BF16_IN>
+constexpr int kThreads = (G == 128 && !BF16_IN) ? 512 : 256;
 constexpr int kVec = 8;  // columns per run
 
 // One run of 8 source values as loaded: one 16-byte word of BF16 values, or
@@ -113,19 +116,21 @@ __device__ __forceinline__ float quotient(float x, float s, float rs) {
 }
 
 // CTAs per SM each instance's registers are held to: g = 128 keeps its runs
-// in registers (BF16 at 64 registers, 4 CTAs; FP32 at 96, 2 CTAs); g = 64
-// runs 8 (BF16) or 6 (FP32), and g = 256 (which reads the block twice) 5.
+// in registers (BF16: 256 threads at 64 registers, 4 CTAs; FP32: 512 threads
+// at 64 registers, 2 CTAs); g = 64 runs 8 (BF16) or 6 (FP32), and g = 256
+// (which reads the block twice) 5.
 template <int G, bool BF16_IN>
 constexpr int kMinCtasPerSm = G == 128 ? (BF16_IN ? 4 : 2) : G == 64 ? (BF16_IN ? 8 : 6) : 5;
 
 template <int G, bool BF16_IN, int FMT>
-__global__ void __launch_bounds__(kThreads, (kMinCtasPerSm<G, BF16_IN>))
+__global__ void __launch_bounds__((kThreads<G, BF16_IN>), (kMinCtasPerSm<G, BF16_IN>))
     quant_kernel(const void* __restrict__ x, int64_t rows, int64_t cols, int64_t col_blocks,
                  uint8_t* __restrict__ q, float* __restrict__ scales) {
+  constexpr int kT = kThreads<G, BF16_IN>;
   constexpr int kRuns = G * G / kVec;   // runs of 8 columns in a full block
   constexpr int kRunsPerRow = G / kVec;
   constexpr float kFmax = FMT == BSGEMM_FP8_E5M2 ? 57344.0f : 448.0f;
-  __shared__ float warp_max[kThreads / 32];
+  __shared__ float warp_max[kT / 32];
   __shared__ float block_scale;
 
   const int64_t blk = blockIdx.x;
@@ -133,7 +138,7 @@ __global__ void __launch_bounds__(kThreads, (kMinCtasPerSm<G, BF16_IN>))
   const int64_t c0 = (blk % col_blocks) * G;
   // g <= 128: the thread's runs stay in registers between the two passes
   // (at most 8 runs); g = 256 reads the block again from L2
-  constexpr int kHeld = kRuns / kThreads <= 8 ? kRuns / kThreads : 0;
+  constexpr int kHeld = kRuns / kT <= 8 ? kRuns / kT : 0;
   Run<BF16_IN> held[kHeld > 0 ? kHeld : 1];
 
   // ---- pass 1: amax over the block (elements outside the matrix are skipped)
@@ -141,7 +146,7 @@ __global__ void __launch_bounds__(kThreads, (kMinCtasPerSm<G, BF16_IN>))
   if constexpr (kHeld > 0) {
 #pragma unroll
     for (int j = 0; j < kHeld; ++j) {
-      const int run = threadIdx.x + j * kThreads;
+      const int run = threadIdx.x + j * kT;
       const int64_t r = r0 + run / kRunsPerRow;
       const int64_t c = c0 + (run % kRunsPerRow) * kVec;
       if (r < rows && c < cols) {  // cols % 8 == 0: a run is wholly in or out
@@ -177,7 +182,7 @@ __global__ void __launch_bounds__(kThreads, (kMinCtasPerSm<G, BF16_IN>))
       }
     }
   } else {
-    for (int run = threadIdx.x; run < kRuns; run += kThreads) {
+    for (int run = threadIdx.x; run < kRuns; run += kT) {
       const int64_t r = r0 + run / kRunsPerRow;
       const int64_t c = c0 + (run % kRunsPerRow) * kVec;
       if (r < rows && c < cols) {
@@ -195,7 +200,7 @@ __global__ void __launch_bounds__(kThreads, (kMinCtasPerSm<G, BF16_IN>))
   if (threadIdx.x == 0) {
     float m = warp_max[0];
 #pragma unroll
-    for (int w = 1; w < kThreads / 32; ++w) m = fmaxf(m, warp_max[w]);
+    for (int w = 1; w < kT / 32; ++w) m = fmaxf(m, warp_max[w]);
     const float s = m > 0.f ? __fdiv_rn(m, kFmax) : 1.0f;
     block_scale = s;
     scales[blk] = s;
@@ -219,7 +224,7 @@ __global__ void __launch_bounds__(kThreads, (kMinCtasPerSm<G, BF16_IN>))
     if constexpr (kHeld > 0) {
 #pragma unroll
       for (int j = 0; j < kHeld; ++j) {
-        const int run = threadIdx.x + j * kThreads;
+        const int run = threadIdx.x + j * kT;
         const int64_t r = r0 + run / kRunsPerRow;
         const int64_t c = c0 + (run % kRunsPerRow) * kVec;
         if (r < rows && c < cols) {
@@ -229,7 +234,7 @@ __global__ void __launch_bounds__(kThreads, (kMinCtasPerSm<G, BF16_IN>))
         }
       }
     } else {
-      for (int run = threadIdx.x; run < kRuns; run += kThreads) {
+      for (int run = threadIdx.x; run < kRuns; run += kT) {
         const int64_t r = r0 + run / kRunsPerRow;
         const int64_t c = c0 + (run % kRunsPerRow) * kVec;
         if (r < rows && c < cols) {
@@ -254,7 +259,7 @@ bsgemm_status launch(const void* x, int64_t rows, int64_t cols, uint8_t* q, floa
   const int64_t rb = (rows + G - 1) / G, cb = (cols + G - 1) / G;
   const int64_t blocks = rb * cb;
   if (blocks > 0x7FFFFFFFll) return BSGEMM_ERR_INVALID_ARG;
-  quant_kernel<G, BF16_IN, FMT><<<static_cast<unsigned>(blocks), kThreads, 0, stream>>>(
+  quant_kernel<G, BF16_IN, FMT><<<static_cast<unsigned>(blocks), kThreads<G, BF16_IN>, 0, stream>>>(
       x, rows, cols, cb, q, scales);
   return cudaGetLastError() == cudaSuccess ? BSGEMM_OK : BSGEMM_ERR_CUDA;
 }
