@@ -81,11 +81,12 @@ __device__ __forceinline__ void load8(const void* x, int64_t off, float (&v)[kVe
   widen<BF16_IN>(load_run<BF16_IN>(x, off), v);
 }
 
+// FP8 codes of a (low byte) and b (the byte above): round to nearest even,
+// saturating to the largest finite value; one conversion for the pair
 template <int FMT>
-__device__ __forceinline__ uint32_t encode(float v) {
-  // round to nearest even, saturating to the largest finite value
-  return static_cast<uint32_t>(
-      __nv_cvt_float_to_fp8(v, __NV_SATFINITE, FMT == BSGEMM_FP8_E5M2 ? __NV_E5M2 : __NV_E4M3));
+__device__ __forceinline__ uint32_t encode2(float a, float b) {
+  return static_cast<uint32_t>(__nv_cvt_float2_to_fp8x2(make_float2(a, b), __NV_SATFINITE,
+                                                        FMT == BSGEMM_FP8_E5M2 ? __NV_E5M2 : __NV_E4M3));
 }
 
 // x / s, correctly rounded in FP32.
@@ -93,8 +94,9 @@ __device__ __forceinline__ uint32_t encode(float v) {
 // FAST = false: the division itself.
 // FAST = true: Markstein's correction step for division. From the correctly
 // rounded reciprocal rs = RN(1/s), take q0 = RN(x * rs), form the residual
-// x - q0 * s exactly with one fma, and correct q0 by residual * rs with a second
-// fma. The quotient's sign is copied from x, so -0 stays -0.
+// negated, q0 * s - x, exactly with one fma, and subtract residual * rs from q0
+// with a second fma. Taking the residual negated keeps the sign of a zero x:
+// -0 gives -0.
 //
 // The fast form is used only for BF16 input and only for s >= kFastMinScale.
 // There the residual is exact wherever the FP8 code depends on it.
@@ -109,7 +111,7 @@ template <bool FAST>
 __device__ __forceinline__ float quotient(float x, float s, float rs) {
   if constexpr (FAST) {
     const float q0 = __fmul_rn(x, rs);
-    return copysignf(__fmaf_rn(__fmaf_rn(-q0, s, x), rs, q0), x);
+    return __fmaf_rn(-__fmaf_rn(q0, s, -x), rs, q0);
   } else {
     return __fdiv_rn(x, s);
   }
@@ -213,12 +215,11 @@ __global__ void __launch_bounds__((kThreads<G, BF16_IN>), (kMinCtasPerSm<G, BF16
     constexpr bool kFast = decltype(fast_tag)::value;
     const float rs = kFast ? __frcp_rn(s) : 0.f;
     auto encode_run = [&](const float (&v)[kVec], int64_t r, int64_t c) {
-      uint32_t lo = 0, hi = 0;
+      float d[kVec];
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        lo |= encode<FMT>(quotient<kFast>(v[i], s, rs)) << (8 * i);
-        hi |= encode<FMT>(quotient<kFast>(v[4 + i], s, rs)) << (8 * i);
-      }
+      for (int i = 0; i < kVec; ++i) d[i] = quotient<kFast>(v[i], s, rs);
+      const uint32_t lo = encode2<FMT>(d[0], d[1]) | (encode2<FMT>(d[2], d[3]) << 16);
+      const uint32_t hi = encode2<FMT>(d[4], d[5]) | (encode2<FMT>(d[6], d[7]) << 16);
       *reinterpret_cast<uint2*>(q + r * cols + c) = make_uint2(lo, hi);
     };
     if constexpr (kHeld > 0) {

@@ -3,8 +3,10 @@
  * The GPU quantiser divides every element x of a block by the block's scale
  * s = RN(amax / FMAX). For BF16 input with s >= 2^-60 it does not divide.
  * It applies Markstein's correction step to the correctly rounded
- * reciprocal rs = RN(1 / s):
- *     q0 = RN(x * rs);  e = RN(fma(-q0, s, x));  q = copysign(RN(fma(e, rs, q0)), x)
+ * reciprocal rs = RN(1 / s), with the residual taken negated:
+ *     q0 = RN(x * rs);  en = RN(fma(q0, s, -x));  q = RN(fma(-en, rs, q0))
+ * (en = q0 * s - x is exact where it matters; negated, the correction keeps
+ * the sign of a zero x: -0 gives -0)
  * This program runs those steps in IEEE single precision for every finite
  * BF16 amax >= 0 and every BF16 x of either sign with |x| <= amax, for E4M3
  * (FMAX 448) and E5M2 (FMAX 57344). It checks q against the correctly rounded
@@ -58,8 +60,8 @@ int main(void) {
           volatile float sv = s;
           const float want = x / sv;
           const float q0 = x * rs;
-          const float e = fmaf(-q0, s, x);
-          const float q = copysignf(fmaf(e, rs, q0), x);
+          const float en = fmaf(q0, s, -x);
+          const float q = fmaf(-en, rs, q0);
           pairs++;
           int same;
           if (fabsf(want) >= 0x1p-18f)
