@@ -63,11 +63,16 @@ def test_malformed_traffic_is_not_reported(fake_root):
 
 
 def test_committed_profiles_name_their_workload_and_sources():
-    """Each committed kernel summary (bsgemm_*.md) carries the three fields the
-    bench reads; other summaries (launch lists) at least the kernel sources."""
+    """Each committed GEMM kernel summary (bsgemm_*.md) carries the three fields
+    the bench reads; a quantiser summary (quantize_*.md) the hash of the
+    quantiser's code; other summaries (launch lists) the GEMM kernels' hash."""
     paths = [p for p in os.listdir(os.path.join(ROOT, "profiles")) if p.endswith(".md")]
     assert paths
     for p in paths:
+        if p.startswith("quantize_"):
+            text = open(os.path.join(ROOT, "profiles", p)).read()
+            assert "quantiser_source_sha256:" in text and "bench_workload:" not in text, p
+            continue
         if not p.startswith("bsgemm_"):
             assert "kernel_source_sha256:" in open(os.path.join(ROOT, "profiles", p)).read(), p
             continue
