@@ -12,12 +12,12 @@
 // to scales [ceil(rows/g), ceil(cols/g)] (row-major FP32): exactly the
 // operand and scale tensors the GEMM takes.
 //
-// One CTA of 256 threads per block. For g <= 128 each thread keeps its part
-// of the block in registers between the amax pass and the encode pass; for
-// g = 256 the block is read twice, the second time from L2. Each thread
-// handles runs of 8
-// consecutive columns: 32-byte (FP32) or 16-byte (BF16) loads, 8-byte stores
-// of 8 codes. This is HBM-bound work: no tensor cores.
+// One CTA per block for g <= 128; for g = 256 a cluster of four CTAs per
+// block, each taking 64 of its rows, which share their partial maxima through
+// distributed shared memory. Each thread keeps its part of the block in
+// registers between the amax pass and the encode pass. Each thread handles
+// runs of 8 consecutive columns: 32-byte (FP32) or 16-byte (BF16) loads,
+// 8-byte stores of 8 codes. This is HBM-bound work: no tensor cores.
 #include <cuda_bf16.h>
 #include <cuda_fp8.h>
 #include <cuda_runtime.h>
@@ -26,13 +26,19 @@
 #include <type_traits>
 
 #include "bsgemm.h"
+#include "ptx.cuh"
 
 namespace bsgq {
 
-// Threads per CTA: 512 at g = 128 from FP32 (each thread holds 4 runs), else
-// 256 (8 runs held at g = 128 from BF16).
+// CTAs per block: a g = 256 block is split by rows over a cluster of four, so
+// that every CTA holds 64 x 256 values, as many as a g = 128 block.
+template <int G>
+constexpr int kParts = G == 256 ? 4 : 1;
+
+// Threads per CTA: 512 from FP32 at g >= 128 (each thread holds 4 runs), else
+// 256 (8 runs held from BF16 at g >= 128; 2 at g = 64).
 template <int G, bool BF16_IN>
-constexpr int kThreads = (G == 128 && !BF16_IN) ? 512 : 256;
+constexpr int kThreads = (G >= 128 && !BF16_IN) ? 512 : 256;
 constexpr int kVec = 8;  // columns per run
 
 // One run of 8 source values as loaded: one 16-byte word of BF16 values, or
@@ -42,6 +48,13 @@ template <bool BF16_IN>
 struct Run {
   uint4 w[BF16_IN ? 1 : 2];
 };
+
+// A float in another CTA's shared memory (a shared::cluster address).
+__device__ __forceinline__ float ld_shared_cluster_f32(uint32_t addr) {
+  float v;
+  asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(addr) : "memory");
+  return v;
+}
 
 template <bool BF16_IN>
 __device__ __forceinline__ Run<BF16_IN> load_run(const void* x, int64_t off) {
@@ -117,29 +130,32 @@ __device__ __forceinline__ float quotient(float x, float s, float rs) {
   }
 }
 
-// CTAs per SM each instance's registers are held to: g = 128 keeps its runs
-// in registers (BF16: 256 threads at 64 registers, 4 CTAs; FP32: 512 threads
-// at 64 registers, 2 CTAs); g = 64 runs 8 (BF16) or 6 (FP32), and g = 256
-// (which reads the block twice) 5.
+// CTAs per SM each instance's registers are held to: at g >= 128 (BF16: 256
+// threads at 64 registers, 4 CTAs; FP32: 512 threads at 64 registers, 2 CTAs);
+// g = 64 runs 8 (BF16) or 6 (FP32).
 template <int G, bool BF16_IN>
-constexpr int kMinCtasPerSm = G == 128 ? (BF16_IN ? 4 : 2) : G == 64 ? (BF16_IN ? 8 : 6) : 5;
+constexpr int kMinCtasPerSm = G >= 128 ? (BF16_IN ? 4 : 2) : (BF16_IN ? 8 : 6);
 
 template <int G, bool BF16_IN, int FMT>
 __global__ void __launch_bounds__((kThreads<G, BF16_IN>), (kMinCtasPerSm<G, BF16_IN>))
     quant_kernel(const void* __restrict__ x, int64_t rows, int64_t cols, int64_t col_blocks,
                  uint8_t* __restrict__ q, float* __restrict__ scales) {
   constexpr int kT = kThreads<G, BF16_IN>;
-  constexpr int kRuns = G * G / kVec;   // runs of 8 columns in a full block
+  constexpr int kP = kParts<G>;
+  constexpr int kRuns = (G / kP) * G / kVec;   // runs of 8 columns in this CTA's rows of a full block
   constexpr int kRunsPerRow = G / kVec;
   constexpr float kFmax = FMT == BSGEMM_FP8_E5M2 ? 57344.0f : 448.0f;
   __shared__ float warp_max[kT / 32];
   __shared__ float block_scale;
+  __shared__ float part_max;   // this CTA's share of a split block's amax
 
-  const int64_t blk = blockIdx.x;
-  const int64_t r0 = (blk / col_blocks) * G;
+  // block blk; this CTA takes its rows [part * G / kP, (part + 1) * G / kP)
+  // (a cluster is kP consecutive CTAs of the grid, so part is the rank)
+  const int64_t blk = blockIdx.x / kP;
+  const int part = static_cast<int>(blockIdx.x % kP);
+  const int64_t r0 = (blk / col_blocks) * G + part * (G / kP);
   const int64_t c0 = (blk % col_blocks) * G;
-  // g <= 128: the thread's runs stay in registers between the two passes
-  // (at most 8 runs); g = 256 reads the block again from L2
+  // the thread's runs stay in registers between the two passes
   constexpr int kHeld = kRuns / kT <= 8 ? kRuns / kT : 0;
   Run<BF16_IN> held[kHeld > 0 ? kHeld : 1];
 
@@ -199,13 +215,29 @@ __global__ void __launch_bounds__((kThreads<G, BF16_IN>), (kMinCtasPerSm<G, BF16
   for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
   if ((threadIdx.x & 31) == 0) warp_max[threadIdx.x >> 5] = amax;
   __syncthreads();
+  float cta_max = 0.f;
   if (threadIdx.x == 0) {
-    float m = warp_max[0];
+    cta_max = warp_max[0];
 #pragma unroll
-    for (int w = 1; w < kT / 32; ++w) m = fmaxf(m, warp_max[w]);
-    const float s = m > 0.f ? __fdiv_rn(m, kFmax) : 1.0f;
+    for (int w = 1; w < kT / 32; ++w) cta_max = fmaxf(cta_max, warp_max[w]);
+  }
+  if constexpr (kP > 1) {
+    // the block's amax: every CTA of the cluster reads all kP shares (every
+    // thread passes both cluster barriers: the second keeps each share alive
+    // until all CTAs have read it)
+    if (threadIdx.x == 0) part_max = cta_max;
+    bsg::cluster_sync_all();
+    if (threadIdx.x == 0) {
+      const uint32_t mine = static_cast<uint32_t>(__cvta_generic_to_shared(&part_max));
+#pragma unroll
+      for (int r = 0; r < kP; ++r) cta_max = fmaxf(cta_max, ld_shared_cluster_f32(bsg::mapa_shared(mine, r)));
+    }
+    bsg::cluster_sync_all();
+  }
+  if (threadIdx.x == 0) {
+    const float s = cta_max > 0.f ? __fdiv_rn(cta_max, kFmax) : 1.0f;
     block_scale = s;
-    scales[blk] = s;
+    if (part == 0) scales[blk] = s;
   }
   __syncthreads();
   const float s = block_scale;
@@ -258,10 +290,28 @@ template <int G, bool BF16_IN, int FMT>
 bsgemm_status launch(const void* x, int64_t rows, int64_t cols, uint8_t* q, float* scales,
                      cudaStream_t stream) {
   const int64_t rb = (rows + G - 1) / G, cb = (cols + G - 1) / G;
-  const int64_t blocks = rb * cb;
-  if (blocks > 0x7FFFFFFFll) return BSGEMM_ERR_INVALID_ARG;
-  quant_kernel<G, BF16_IN, FMT><<<static_cast<unsigned>(blocks), kThreads<G, BF16_IN>, 0, stream>>>(
-      x, rows, cols, cb, q, scales);
+  const int64_t ctas = rb * cb * kParts<G>;
+  if (ctas > 0x7FFFFFFFll) return BSGEMM_ERR_INVALID_ARG;
+  if constexpr (kParts<G> == 1) {
+    quant_kernel<G, BF16_IN, FMT><<<static_cast<unsigned>(ctas), kThreads<G, BF16_IN>, 0, stream>>>(
+        x, rows, cols, cb, q, scales);
+  } else {
+    // a cluster of kParts CTAs per block
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(ctas), 1, 1);
+    cfg.blockDim = dim3(kThreads<G, BF16_IN>, 1, 1);
+    cfg.dynamicSmemBytes = 0;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = kParts<G>;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (cudaLaunchKernelEx(&cfg, quant_kernel<G, BF16_IN, FMT>, x, rows, cols, cb, q, scales) != cudaSuccess)
+      return BSGEMM_ERR_CUDA;
+  }
   return cudaGetLastError() == cudaSuccess ? BSGEMM_OK : BSGEMM_ERR_CUDA;
 }
 
