@@ -391,13 +391,7 @@ def roofline(p: workloads.Problem, ms: float, name: str, peaks: dict) -> dict:
     """Roofline of one launch: tensor-bound (FLOPs vs the FP8 peak) for
     M > 128, HBM-bound (algorithmic bytes vs the copy bandwidth) otherwise."""
     if p.M > 128:
-        # FP8 dense peak = measured BF16 burst x the nominal FP8/BF16 ratio (4.5 / 2.25)
-        peak = peaks["bf16_tflops"] * 2.0
-        achieved = p.flops / (ms * 1e-3) / 1e12
-        return {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
-                "frac": achieved / peak, "traffic": profiled_traffic(name),
-                "peak_source": f"{peaks['source']} bf16 burst x 2 (FP8/BF16 nominal ratio)",
-                "frac_of_nominal_4500": achieved / 4500.0}
+        return tensor_roofline(p.flops, ms, name, peaks)
     bytes_ = algorithmic_bytes(p)
     peak = peaks["hbm_gbs"]
     achieved = bytes_ / (ms * 1e-3) / 1e9
@@ -471,6 +465,89 @@ def run_e2e(p, dev, stream, tuning, args, world):
                     "double-buffered over a copy-in stream, the GEMM stream and a copy-out stream"}
 
 
+def clocks_under_load(call, n_sets: int, stream):
+    """SM clocks and throttle reasons under this load: the sampler covers
+    ~0.4 s of the same launches, eager and back to back, right after the timed
+    region (which itself is far shorter than nvidia-smi's sampling interval)."""
+    import torch
+    with ClockSampler(torch.cuda.current_device()) as clk:
+        t_soak = time.perf_counter()
+        with torch.cuda.stream(stream):
+            i = 0
+            while time.perf_counter() - t_soak < 0.4:
+                for _ in range(20):
+                    call(i % n_sets)
+                    i += 1
+                stream.synchronize()
+    clocks = clk.summary()
+    if clocks is not None:
+        clocks["window"] = "0.4 s of the benchmark's own launches, back to back, after the timed region"
+    return clocks
+
+
+def tensor_roofline(flops: int, ms: float, name: str, peaks: dict) -> dict:
+    # FP8 dense peak = measured BF16 burst x the nominal FP8/BF16 ratio (4.5 / 2.25)
+    peak = peaks["bf16_tflops"] * 2.0
+    achieved = flops / (ms * 1e-3) / 1e12
+    return {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+            "frac": achieved / peak, "traffic": profiled_traffic(name),
+            "peak_source": f"{peaks['source']} bf16 burst x 2 (FP8/BF16 nominal ratio)",
+            "frac_of_nominal_4500": achieved / 4500.0}
+
+
+def run_grouped(args, dev, stream, l2_bytes, peaks, world, rank):
+    """The grouped GEMM (one persistent launch over all experts) on the
+    seeded mixture-of-experts workload, timed like the plain GEMM: rotating
+    input sets, a CUDA graph of back-to-back launches, device events."""
+    import torch
+    import fp8_block_scaled_bsgemm_b200 as bsg
+    gp = workloads.grouped_moe()
+    rows = gp.a.shape[0]
+    base = [torch.from_numpy(x).to(dev) for x in (gp.a, gp.b, gp.sa, gp.sb)]
+    group_m = torch.tensor(gp.ms, dtype=torch.int32, device=dev)
+    per_set = sum(x.numel() * x.element_size() for x in base) + 2 * rows * gp.N
+    r = 1 if args.l2 == "flush" else max(3, -(-2 * l2_bytes // per_set))
+    sets = []
+    for i in range(r):
+        cp = base if i == 0 else [x.clone() for x in base]
+        sets.append(tuple(cp) + (torch.empty((rows, gp.N), dtype=torch.bfloat16, device=dev),))
+
+    def call(i):
+        a, b, sa, sb, out = sets[i]
+        bsg.grouped_gemm(a, b, sa, sb, group_m, out=out, gran=gp.gran, stream=stream)
+
+    with torch.cuda.stream(stream):
+        ms, per = time_device(call, len(sets), args.steps, args.warmup, stream, world, args.l2)
+    status = bsg.get_last_device_status(stream)
+    if status != 0:
+        raise SystemExit(f"device status {status} after the timed region of grouped")
+    ms_max = max_over_ranks(ms, world)
+    clocks = clocks_under_load(call, len(sets), stream)
+    if rank != 0:
+        _finish(world)
+        return
+    line = {
+        "metric": METRIC, "value": job_tflops(gp.flops, world, ms_max), "unit": "TFLOP/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_max,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "fp8_e4m3",
+        "data": "synthetic",
+        "config": {"workload": gp.name, "name": "grouped", "groups": len(gp.ms), "rows_per_group": gp.ms,
+                   "N": gp.N, "K": gp.K, "gran": gp.gran, "layout": "nt",
+                   "inputs": "E4M3 codes + FP32 block scales, seeded synthetic", "l2": l2_note(args.l2)},
+        "parallelism": f"replicas{world}", "input_sets": len(sets), "input_set_bytes": per_set,
+        "step": "grouped GEMM (one launch over all groups)",
+        "roofline": tensor_roofline(gp.flops, ms, "grouped", peaks),
+        "e2e": None, "gpu_launches": args.steps, "clocks": clocks, "hbm_bound": [],
+    }
+    if not args.no_cpu_baseline and world == 1:
+        largest = max(range(len(gp.ms)), key=lambda i: gp.ms[i])
+        line["cpu_baseline"] = cpu_baseline(gp.parts[largest], args.cpu_seconds)
+    else:
+        line["cpu_baseline"] = None
+    print(json.dumps(line), flush=True)
+    _finish(world)
+
+
 def run_ours(args):
     import torch
     import fp8_block_scaled_bsgemm_b200 as bsg
@@ -486,6 +563,9 @@ def run_ours(args):
     if args.variant != "auto" or args.bnq or args.splits or args.stream_k:
         tuning = {"variant": args.variant, "bnq": args.bnq, "splits": args.splits, "stream_k": args.stream_k}
     peaks = measured_peaks()
+    if args.workload == "grouped":
+        run_grouped(args, dev, stream, l2_bytes, peaks, world, rank)
+        return
 
     def measure(name, steps, warmup, tune, quantize_a=False):
         p = make_workload(name)
@@ -519,21 +599,7 @@ def run_ours(args):
                                                     args.quantize_a)
     ms_max = max_over_ranks(ms, world)
 
-    # clocks under this load: the sampler covers ~0.4 s of the same launches,
-    # eager and back to back, right after the timed region (which itself is
-    # far shorter than nvidia-smi's sampling interval)
-    with ClockSampler(torch.cuda.current_device()) as clk:
-        t_soak = time.perf_counter()
-        with torch.cuda.stream(stream):
-            i = 0
-            while time.perf_counter() - t_soak < 0.4:
-                for _ in range(20):
-                    call(i % len(sets))
-                    i += 1
-                stream.synchronize()
-    clocks = clk.summary()
-    if clocks is not None:
-        clocks["window"] = "0.4 s of the benchmark's own launches, back to back, after the timed region"
+    clocks = clocks_under_load(call, len(sets), stream)
 
     # ---- e2e through the public API from pinned host memory
     e2e = None
@@ -590,7 +656,15 @@ def run_reference(args):
     if rank != 0:
         return
     import oracle
-    p = make_workload(args.workload)
+    if args.workload == "grouped":
+        # the oracle's throughput on the largest group (each group is a plain GEMM)
+        gp = workloads.grouped_moe()
+        p = gp.parts[max(range(len(gp.ms)), key=lambda i: gp.ms[i])]
+        config = {"workload": gp.name, "name": "grouped", "sample_of": "the largest group",
+                  "l2": l2_note(args.l2)}
+    else:
+        p = make_workload(args.workload)
+        config = workload_config(p, args.workload, args.l2)
     budget = max(1.0, 150.0 / max(1, args.steps + args.warmup))  # whole run within a few minutes
     per = []
     for i in range(args.warmup + args.steps):
@@ -603,7 +677,7 @@ def run_reference(args):
         "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": statistics.mean(r["seconds"] for r in per) * 1e3,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-        "data": "synthetic", "config": workload_config(p, args.workload, args.l2),
+        "data": "synthetic", "config": config,
         "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": oracle.num_threads(), "kind": "oracle",
                          "sample": per[-1]["sample"] + " per step"},
         "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},

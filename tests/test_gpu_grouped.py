@@ -89,3 +89,26 @@ def test_grouped_gemm_argument_errors():
         bsg.grouped_gemm(a, b, sa, sb.cpu(), gm)
     with pytest.raises(ValueError):
         bsg.grouped_gemm(a, b, sa, sb, gm.cpu())
+
+
+def test_grouped_moe_workload_sampled():
+    """The bench's grouped workload at full size (8192 rows over 8 experts of
+    4096 x 7168, g = 128), through the same call the bench times: sampled
+    outputs of every group against the oracle run on that group."""
+    from gpu_util import full_rms_from_gpu
+    gp = workloads.grouped_moe()
+    a, b = torch.from_numpy(gp.a).cuda(), torch.from_numpy(gp.b).cuda()
+    sa, sb = torch.from_numpy(gp.sa).cuda(), torch.from_numpy(gp.sb).cuda()
+    out = bsg.grouped_gemm(a, b, sa, sb, torch.tensor(gp.ms, dtype=torch.int32, device="cuda"), gran=gp.gran)
+    torch.cuda.synchronize()
+    assert bsg.get_last_device_status() == 0
+    r = 0
+    for i, (m, p) in enumerate(zip(gp.ms, gp.parts)):
+        if m:
+            og = out[r:r + m]
+            mi, ni = workloads.sample_indices(m, gp.N, 600, seed=i)
+            ref, _ = oracle.bsgemm_at("nt", p.a[:m], p.b, p.sa[:-(-m // gp.gran)], p.sb, m, gp.N, gp.K,
+                                      gp.gran, mi, ni)
+            got = gpu_as_f64(og[torch.from_numpy(mi).cuda(), torch.from_numpy(ni).cuda()])
+            check_close(got, ref, f"grouped MoE group {i} (M={m})", rms=full_rms_from_gpu(og))
+        r += m

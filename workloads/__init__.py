@@ -154,6 +154,50 @@ def long_k(gran=128, seed=0, layout="nt"):
                         name=f"long-K 2048x4096x32768 g={gran}")
 
 
+@dataclasses.dataclass
+class GroupedProblem:
+    """Inputs of one grouped NT call: group i multiplies its M_i rows of A by
+    its own B_i; A's rows and A's scale blocks are stacked group after group."""
+    ms: list            # rows per group
+    N: int
+    K: int
+    gran: int
+    a: np.ndarray       # uint8 [sum M_i, K]
+    sa: np.ndarray      # float32 [sum ceil(M_i/g) + len(ms), Kb] (group i's blocks from row S_i)
+    b: np.ndarray       # uint8 [G, N, K]
+    sb: np.ndarray      # float32 [G, ceil(N/g), Kb]
+    parts: list         # each group's own Problem (its A rows and scales, its B)
+    name: str = ""
+
+    @property
+    def flops(self) -> int:
+        return 2 * sum(self.ms) * self.N * self.K
+
+
+def grouped_moe(seed=0, groups=8, tokens=8192, N=4096, K=7168, gran=128):
+    """A mixture-of-experts up-projection: `tokens` rows routed to `groups`
+    experts in seeded, uneven shares (Dirichlet(1) proportions, multinomial
+    counts), each expert with its own [N, K] weights."""
+    rng = np.random.Generator(np.random.PCG64(seed + 1000))
+    ms = [int(m) for m in rng.multinomial(tokens, rng.dirichlet(np.ones(groups)))]
+    parts = [make_problem(max(m, 1), N, K, gran, "nt", seed + 10 * i) for i, m in enumerate(ms)]
+    kb = -(-K // gran)
+    a = np.zeros((tokens, K), np.uint8)
+    sa = np.ones((-(-tokens // gran) + groups, kb), np.float32)
+    r = sr = 0
+    for m, p in zip(ms, parts):
+        if m:
+            a[r:r + m] = p.a[:m]
+            sa[sr:sr + -(-m // gran)] = p.sa[:-(-m // gran)]
+        r += m
+        sr += -(-m // gran)
+    b = np.stack([p.b for p in parts])
+    sb = np.stack([p.sb for p in parts])
+    return GroupedProblem(ms, N, K, gran, a, sa, b, sb, parts,
+                          f"grouped MoE up-projection: {tokens} rows over {groups} experts, "
+                          f"N={N}, K={K}, g={gran}")
+
+
 def logical_a(p: Problem) -> np.ndarray:
     """A's codes as the logical [M, K] matrix, whatever the storage layout."""
     return np.ascontiguousarray(p.a.T) if a_is_transposed(p.layout) else p.a
