@@ -8,6 +8,8 @@
 //          57344 for E5M2), or 1 when amax is 0;
 //   q    = FP8 code of x / s (FP32 division, correctly rounded), rounded to
 //          nearest with ties to even and saturated to +-FMAX.
+// (For BF16 input the correctly rounded x / s is formed without a division;
+// see quotient() below.)
 // The codes go to q [rows, cols] (row-major, one byte each) and the scales
 // to scales [ceil(rows/g), ceil(cols/g)] (row-major FP32): exactly the
 // operand and scale tensors the GEMM takes.
