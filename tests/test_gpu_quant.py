@@ -37,7 +37,7 @@ def test_quantiser_fp32_bit_exact(fmt, g, rows, cols):
 
 
 @pytest.mark.parametrize("fmt", ["e4m3", "e5m2"])
-@pytest.mark.parametrize("g", [64, 128])
+@pytest.mark.parametrize("g", [64, 128, 256])
 def test_quantiser_bf16_bit_exact(fmt, g):
     x32 = _source(200, 1040, 5)
     xb = torch.from_numpy(x32).to(torch.bfloat16)
@@ -71,7 +71,7 @@ def _every_bf16_up_to(amax_bits, g):
 
 
 @pytest.mark.parametrize("fmt", ["e4m3", "e5m2"])
-@pytest.mark.parametrize("g", [64, 128])
+@pytest.mark.parametrize("g", [64, 128, 256])
 def test_quantiser_bf16_every_value_below_amax(fmt, g):
     """The BF16 path's quotient (a corrected reciprocal product where the
     block scale allows it) against the oracle's division, for every BF16 value
