@@ -458,8 +458,43 @@ def run_e2e(p, dev, stream, tuning, args, world):
     barrier(world)
     e_ms = max_over_ranks(t0.elapsed_time(t1) / args.steps, world)
     h2d = sum(x.numel() * x.element_size() for x in host[0])
+    d2h = hout[0].numel() * hout[0].element_size()
+
+    # the link alone: the same copies, one direction at a time, nothing else running
+    def copy_ms(fn, reps=5):
+        c0 = torch.cuda.Event(enable_timing=True)
+        c1 = torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize()
+        c0.record(stream)
+        with torch.cuda.stream(stream):
+            for _ in range(reps):
+                fn()
+        c1.record(stream)
+        torch.cuda.synchronize()
+        return c0.elapsed_time(c1) / reps
+
+    h2d_ms = copy_ms(lambda: [d.copy_(h, non_blocking=True) for d, h in zip(dbuf[0], host[0])])
+    d2h_ms = copy_ms(lambda: hout[0].copy_(dout[0], non_blocking=True))
+
+    def both():
+        # both directions at once, on the copy-in and copy-out streams
+        s_in.wait_stream(stream)
+        s_out.wait_stream(stream)
+        with torch.cuda.stream(s_in):
+            for d, h in zip(dbuf[0], host[0]):
+                d.copy_(h, non_blocking=True)
+        with torch.cuda.stream(s_out):
+            hout[1].copy_(dout[1], non_blocking=True)
+        stream.wait_stream(s_in)
+        stream.wait_stream(s_out)
+
+    both_ms = copy_ms(both)
     return {"value": world * p.flops / (e_ms * 1e-3) / 1e12, "unit": "TFLOP/s", "ms_per_step": e_ms,
-            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": hout[0].numel() * hout[0].element_size(),
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+            "link_alone": {"h2d_gbs": h2d / (h2d_ms * 1e-3) / 1e9, "d2h_gbs": d2h / (d2h_ms * 1e-3) / 1e9,
+                           "both_directions_ms": both_ms,
+                           "note": "the step's copies with no GEMM: one direction at a time (GB/s), and both "
+                                   "directions at once (ms), which is the per-step floor of the e2e loop"},
             "path": "per step: pinned host -> device copies of A, B and the scales, the GEMM through the "
                     "public binding (its C ABI takes device pointers), device -> pinned host copy of out; "
                     "double-buffered over a copy-in stream, the GEMM stream and a copy-out stream"}
