@@ -15,8 +15,8 @@
 // operand and scale tensors the GEMM takes.
 //
 // One CTA per block for g <= 128; for g = 256 a cluster of four CTAs per
-// block, each taking 64 of its rows, which share their partial maxima through
-// distributed shared memory. Each thread keeps its part of the block in
+// block, each taking 64 of its rows, which exchange their partial maxima
+// through distributed shared memory. Each thread keeps its part of the block in
 // registers between the amax pass and the encode pass. Each thread handles
 // runs of 8 consecutive columns: 32-byte (FP32) or 16-byte (BF16) loads,
 // 8-byte stores of 8 codes. This is HBM-bound work: no tensor cores.
@@ -51,11 +51,9 @@ struct Run {
   uint4 w[BF16_IN ? 1 : 2];
 };
 
-// A float in another CTA's shared memory (a shared::cluster address).
-__device__ __forceinline__ float ld_shared_cluster_f32(uint32_t addr) {
-  float v;
-  asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(addr) : "memory");
-  return v;
+// Store a float to a CTA's shared memory in the cluster (a shared::cluster address).
+__device__ __forceinline__ void st_shared_cluster_f32(uint32_t addr, float v) {
+  asm volatile("st.shared::cluster.f32 [%0], %1;" ::"r"(addr), "f"(v) : "memory");
 }
 
 template <bool BF16_IN>
@@ -149,7 +147,7 @@ __global__ void __launch_bounds__((kThreads<G, BF16_IN>), (kMinCtasPerSm<G, BF16
   constexpr float kFmax = FMT == BSGEMM_FP8_E5M2 ? 57344.0f : 448.0f;
   __shared__ float warp_max[kT / 32];
   __shared__ float block_scale;
-  __shared__ float part_max;   // this CTA's share of a split block's amax
+  __shared__ float part_max[kParts<G>];   // the shares of a split block's amax, one per CTA
 
   // block blk; this CTA takes its rows [part * G / kP, (part + 1) * G / kP)
   // (a cluster is kP consecutive CTAs of the grid, so part is the rank)
@@ -224,17 +222,21 @@ __global__ void __launch_bounds__((kThreads<G, BF16_IN>), (kMinCtasPerSm<G, BF16
     for (int w = 1; w < kT / 32; ++w) cta_max = fmaxf(cta_max, warp_max[w]);
   }
   if constexpr (kP > 1) {
-    // the block's amax: every CTA of the cluster reads all kP shares (every
-    // thread passes both cluster barriers: the second keeps each share alive
-    // until all CTAs have read it)
-    if (threadIdx.x == 0) part_max = cta_max;
-    bsg::cluster_sync_all();
+    // the block's amax: thread 0 of each CTA writes its share into slot
+    // `part` of every CTA of the cluster, its own included. One cluster
+    // barrier (every thread; release then acquire) makes all kP shares
+    // visible in each CTA's own shared memory, and no CTA touches another's
+    // shared memory after it, so any CTA may then run on to its exit.
     if (threadIdx.x == 0) {
-      const uint32_t mine = static_cast<uint32_t>(__cvta_generic_to_shared(&part_max));
+      const uint32_t slot = static_cast<uint32_t>(__cvta_generic_to_shared(&part_max[part]));
 #pragma unroll
-      for (int r = 0; r < kP; ++r) cta_max = fmaxf(cta_max, ld_shared_cluster_f32(bsg::mapa_shared(mine, r)));
+      for (int r = 0; r < kP; ++r) st_shared_cluster_f32(bsg::mapa_shared(slot, r), cta_max);
     }
     bsg::cluster_sync_all();
+    if (threadIdx.x == 0) {
+#pragma unroll
+      for (int r = 0; r < kP; ++r) cta_max = fmaxf(cta_max, part_max[r]);
+    }
   }
   if (threadIdx.x == 0) {
     const float s = cta_max > 0.f ? __fdiv_rn(cta_max, kFmax) : 1.0f;
