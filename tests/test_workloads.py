@@ -67,3 +67,24 @@ def test_outlier_rows_and_block_std():
 def test_sample_indices_in_range():
     mi, ni = workloads.sample_indices(7, 300, 100)
     assert mi.min() >= 0 and mi.max() < 7 and ni.min() >= 0 and ni.max() < 300
+
+
+def test_grouped_moe_stacks_each_group_in_place():
+    """The grouped workload's stacked A rows and A scale blocks are each
+    group's own, at the offsets the grouped call derives from the group sizes
+    (rows R_i = sum of earlier M_i, scale rows S_i = sum of earlier ceil(M_i/g));
+    a small instance keeps the test fast."""
+    gp = workloads.grouped_moe(groups=5, tokens=700, N=64, K=256, gran=64)
+    assert sum(gp.ms) == 700 and len(gp.ms) == 5 and gp.a.shape == (700, 256)
+    assert gp.b.shape == (5, 64, 256) and gp.sb.shape == (5, 1, 4)
+    assert gp.sa.shape[0] >= -(-700 // 64) + 5
+    r = sr = 0
+    for m, p in zip(gp.ms, gp.parts):
+        nb = -(-m // 64)
+        assert np.array_equal(gp.a[r:r + m], p.a[:m])
+        assert np.array_equal(gp.sa[sr:sr + nb], p.sa[:nb])
+        r += m
+        sr += nb
+    again = workloads.grouped_moe(groups=5, tokens=700, N=64, K=256, gran=64)
+    assert again.ms == gp.ms and np.array_equal(again.a, gp.a) and np.array_equal(again.b, gp.b)
+    assert gp.flops == 2 * 700 * 64 * 256
